@@ -1,0 +1,151 @@
+"""B200-native masked attention JVP (Causal-rCM report, Appendix B).
+
+``jvp_attn(q, k, v, dq, dk, dv, mask)`` returns (O, dO, LSE) for softmax
+attention under a temporal mask and its forward-mode tangent along
+(dQ, dK, dV), computed by the CUDA kernels of ``libjvpattn.so``. PyTorch is
+used for device memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+from typing import Optional, Tuple
+
+from . import _lib
+from ._lib import JvpAttnError, MaskDesc
+
+DENSE = 0
+FRAME_CAUSAL = 1
+CHUNK_CAUSAL = 2
+TEACHER_FORCING = 3
+
+__all__ = ["Mask", "jvp_attn", "jvp_attn_fwd", "mask_stats", "tile_classes",
+           "schedule", "check_device_error", "release", "JvpAttnError",
+           "DENSE", "FRAME_CAUSAL", "CHUNK_CAUSAL", "TEACHER_FORCING"]
+
+
+@dataclasses.dataclass(frozen=True)
+class Mask:
+    """Temporal mask descriptor {mode, tokens_per_frame, n_frames, chunk}."""
+    mode: int
+    tokens_per_frame: int
+    n_frames: int
+    chunk: int = 1
+
+    def desc(self) -> MaskDesc:
+        return MaskDesc(self.mode, self.tokens_per_frame, self.n_frames, self.chunk)
+
+    @property
+    def length(self) -> int:
+        ft = self.tokens_per_frame * self.n_frames
+        return 2 * ft if self.mode == TEACHER_FORCING else ft
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return _lib.JVP_BF16
+    if t.dtype == torch.float32:
+        return _lib.JVP_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
+
+
+def jvp_attn_fwd(q, k, v, dq, dk, dv, o, d_o, lse, mask: Mask,
+                 scale: Optional[float] = None, stream: Optional[int] = None) -> None:
+    """Raw call of the C ABI on caller-allocated device tensors (no checks
+    beyond those the library makes). ``stream`` is a cudaStream_t as int;
+    default: the current torch stream of q's device."""
+    import torch
+    B, H, L, d = q.shape
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    rc = _lib.lib().jvp_attn_fwd(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+        dv.data_ptr(), o.data_ptr(), d_o.data_ptr(),
+        ctypes.cast(lse.data_ptr(), ctypes.POINTER(ctypes.c_float)),
+        B, H, L, d, _dtype_code(q), mask.desc(),
+        0.0 if scale is None else float(scale), ctypes.c_void_p(stream))
+    _lib.check(rc, "jvp_attn_fwd")
+
+
+def jvp_attn(q, k, v, dq, dk, dv, mask: Mask, scale: Optional[float] = None,
+             out: Optional[Tuple] = None):
+    """O, dO, LSE of masked attention and its JVP.
+
+    q, k, v, dq, dk, dv: CUDA tensors [B, H, L, d], all bfloat16 or all
+    float32, contiguous. Returns (o, do, lse) with o, do like q and lse
+    float32 [B, H, L]. ``out`` may supply preallocated (o, do, lse).
+    """
+    import torch
+    ts = (q, k, v, dq, dk, dv)
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("jvp_attn expects CUDA tensors")
+        if t.shape != q.shape or t.dtype != q.dtype or t.device != q.device:
+            raise ValueError("q, k, v, dq, dk, dv must share shape, dtype and device")
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous [B, H, L, d]")
+    if q.dim() != 4:
+        raise ValueError("inputs must be [B, H, L, d]")
+    B, H, L, d = q.shape
+    if out is None:
+        o = torch.empty_like(q)
+        d_o = torch.empty_like(q)
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    else:
+        o, d_o, lse = out
+    jvp_attn_fwd(q, k, v, dq, dk, dv, o, d_o, lse, mask, scale)
+    return o, d_o, lse
+
+
+def mask_stats(mask: Mask, L: Optional[int] = None, bm: int = 128, bn: int = 64):
+    """(pairs, full, partial, empty) for the mask on a bm x bn tile grid."""
+    L = mask.length if L is None else L
+    vals = [ctypes.c_int64() for _ in range(4)]
+    rc = _lib.lib().jvp_attn_mask_stats(mask.desc(), L, bm, bn,
+                                         *[ctypes.byref(x) for x in vals])
+    _lib.check(rc, "jvp_attn_mask_stats")
+    return tuple(x.value for x in vals)
+
+
+def tile_classes(mask: Mask, L: Optional[int] = None, bm: int = 128, bn: int = 64):
+    """numpy int8 [n_qt, n_kt] of tile classes (0 empty, 1 full, 2 partial)."""
+    import numpy as np
+    L = mask.length if L is None else L
+    nq, nk = -(-L // bm), -(-L // bn)
+    out = np.zeros((nq, nk), dtype=np.int8)
+    rc = _lib.lib().jvp_attn_tile_classes(
+        mask.desc(), L, bm, bn, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int8)), out.size)
+    _lib.check(rc, "jvp_attn_tile_classes")
+    return out
+
+
+def schedule(mask: Mask, L: Optional[int] = None, bm: int = 128, bn: int = 64):
+    """(qtiles [n, 4], segs [m, 3]) int32 arrays of the tensor-core work list."""
+    import numpy as np
+    L = mask.length if L is None else L
+    nq, ns = ctypes.c_int(), ctypes.c_int()
+    lib = _lib.lib()
+    lib.jvp_attn_schedule(mask.desc(), L, bm, bn, None, 0, None, 0,
+                          ctypes.byref(nq), ctypes.byref(ns))
+    qt = np.zeros((nq.value, 4), dtype=np.int32)
+    sg = np.zeros((ns.value, 3), dtype=np.int32)
+    p32 = ctypes.POINTER(ctypes.c_int32)
+    rc = lib.jvp_attn_schedule(mask.desc(), L, bm, bn, qt.ctypes.data_as(p32), nq.value,
+                               sg.ctypes.data_as(p32), ns.value, ctypes.byref(nq),
+                               ctypes.byref(ns))
+    _lib.check(rc, "jvp_attn_schedule")
+    return qt, sg
+
+
+def check_device_error(stream: Optional[int] = None) -> None:
+    """Synchronise ``stream`` and raise if a kernel recorded a device error."""
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    _lib.check(_lib.lib().jvp_attn_check_device_error(ctypes.c_void_p(stream)),
+               "jvp_attn_check_device_error")
+
+
+def release() -> None:
+    _lib.check(_lib.lib().jvp_attn_release(), "jvp_attn_release")

@@ -1,0 +1,41 @@
+// Internal declarations shared by the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/jvp_attn.h"
+
+namespace jvp {
+
+// Bits of the per-device error word the kernels OR into.
+constexpr unsigned kErrTimeout = 1u;
+constexpr unsigned kErrBounds = 2u;
+
+// Device work list for the tensor-core kernel (see schedule.h).
+struct WorkList {
+  const int4* qtiles = nullptr;  // {qt, seg_begin, seg_count, n_ktiles}
+  const int2* segs = nullptr;    // {kt_begin, (count << 1) | partial}
+  int n_qtiles = 0;
+  int n_segs = 0;
+};
+
+struct LaunchArgs {
+  const void *q, *k, *v, *dq, *dk, *dv;
+  void *o, *d_o;
+  float* lse;
+  int B, H, L, d;
+  jvp_mask_desc mask;
+  float scale;
+  cudaStream_t stream;
+  unsigned* err;  // device error word
+  unsigned long long wait_limit_ns;
+};
+
+// CUDA-core kernel (fp32 arithmetic) for fp32 or bf16 inputs, d in {32,64,96,128}.
+int launch_simt(const LaunchArgs& a, bool bf16);
+
+// Tensor-core kernel: bf16, d = 128, sm_100a.
+int launch_sm100(const LaunchArgs& a, const WorkList& w, int num_sms);
+
+}  // namespace jvp

@@ -1,0 +1,262 @@
+// C ABI of the masked attention JVP library (declared in include/jvp_attn.h).
+//
+// Host-side duties: argument validation, the per-device error word, the
+// cached device work lists built by the tile scheduler, and dispatch to the
+// tensor-core kernel (bf16, d = 128) or the CUDA-core kernel (fp32 / other
+// head dims). No exception crosses the boundary.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <vector>
+
+#include "common.cuh"
+#include "schedule.h"
+
+// One error word per device that loads the library; kernels OR bits in.
+__device__ unsigned g_jvp_error_word;
+
+namespace jvp {
+namespace {
+
+constexpr int kBM = 128, kBN = 64;            // tensor-core tile shape
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
+constexpr int kMaxDevices = 64;
+
+struct DevInfo {
+  bool ready = false;
+  int sms = 0, major = 0, minor = 0;
+  unsigned* err = nullptr;
+};
+
+struct WsKey {
+  int dev, mode, T, F, chunk, L, bm, bn;
+  bool operator<(const WsKey& o) const {
+    return std::tie(dev, mode, T, F, chunk, L, bm, bn) <
+           std::tie(o.dev, o.mode, o.T, o.F, o.chunk, o.L, o.bm, o.bn);
+  }
+};
+
+struct Ws {
+  void* buf = nullptr;
+  WorkList w;
+};
+
+std::mutex g_mu;
+DevInfo g_dev[kMaxDevices];
+std::map<WsKey, Ws> g_ws;
+
+int device_info(DevInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return JVP_ERR_LAUNCH_FAILED;
+  if (dev < 0 || dev >= kMaxDevices) return JVP_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) !=
+            cudaSuccess)
+      return JVP_ERR_LAUNCH_FAILED;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_jvp_error_word) != cudaSuccess) {
+      cudaGetLastError();
+      return JVP_ERR_UNSUPPORTED_DEVICE;  // no sm_100a image for this device
+    }
+    d.err = static_cast<unsigned*>(p);
+    if (cudaMemset(d.err, 0, sizeof(unsigned)) != cudaSuccess) return JVP_ERR_LAUNCH_FAILED;
+    d.ready = true;
+  }
+  *out = &d;
+  return JVP_OK;
+}
+
+int get_worklist(int dev, const jvp_mask_desc& m, int L, WorkList* out) {
+  const WsKey key{dev, m.mode, m.tokens_per_frame, m.n_frames,
+                  m.chunk, L, kBM, kBN};
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_ws.find(key);
+  if (it != g_ws.end()) {
+    *out = it->second.w;
+    return JVP_OK;
+  }
+  const Schedule s = build_schedule(m, L, kBM, kBN);
+  const size_t qbytes = s.qtiles.size() * sizeof(int32_t);
+  const size_t sbytes = s.segs.size() * sizeof(int32_t);
+  const size_t soff = (qbytes + 255) & ~size_t(255);
+  Ws ws;
+  if (cudaMalloc(&ws.buf, soff + sbytes) != cudaSuccess) {
+    cudaGetLastError();
+    return JVP_ERR_OUT_OF_MEMORY;
+  }
+  char* b = static_cast<char*>(ws.buf);
+  if (cudaMemcpy(b, s.qtiles.data(), qbytes, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(b + soff, s.segs.data(), sbytes, cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaFree(ws.buf);
+    return JVP_ERR_LAUNCH_FAILED;
+  }
+  ws.w.qtiles = reinterpret_cast<const int4*>(b);
+  ws.w.segs = reinterpret_cast<const int2*>(b + soff);
+  ws.w.n_qtiles = int(s.qtiles.size() / 4);
+  ws.w.n_segs = int(s.segs.size() / 2);
+  g_ws[key] = ws;
+  *out = ws.w;
+  return JVP_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace jvp
+
+using namespace jvp;
+
+extern "C" {
+
+int jvp_attn_fwd(const void* q, const void* k, const void* v, const void* dq, const void* dk,
+                 const void* dv, void* o, void* d_o, float* lse, int B, int H, int L, int d,
+                 jvp_dtype dtype, jvp_mask_desc mask, float softmax_scale, void* stream) {
+  if (!q || !k || !v || !dq || !dk || !dv || !o || !d_o || !lse) return JVP_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || L <= 0 || d <= 0) return JVP_ERR_INVALID_ARG;
+  if (dtype != JVP_BF16 && dtype != JVP_FP32) return JVP_ERR_INVALID_ARG;
+  if (std::isnan(softmax_scale) || std::isinf(softmax_scale)) return JVP_ERR_INVALID_ARG;
+  int rc = validate_mask(mask, L);
+  if (rc != JVP_OK) return rc;
+  if ((long long)B * H * L >= (1LL << 31) || (long long)B * H >= (1LL << 31) / 2)
+    return JVP_ERR_TOO_LARGE;
+  const bool tensor_core = dtype == JVP_BF16 && d == 128;
+  if (!tensor_core && (d % 32 != 0 || d > 128)) return JVP_ERR_UNSUPPORTED_HEAD_DIM;
+  const void* ptrs[] = {q, k, v, dq, dk, dv, o, d_o, lse};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return JVP_ERR_MISALIGNED;
+
+  DevInfo* di = nullptr;
+  rc = device_info(&di);
+  if (rc != JVP_OK) return rc;
+  if (di->major != 10 || di->minor != 0) return JVP_ERR_UNSUPPORTED_DEVICE;
+
+  LaunchArgs a;
+  a.q = q; a.k = k; a.v = v; a.dq = dq; a.dk = dk; a.dv = dv;
+  a.o = o; a.d_o = d_o; a.lse = lse;
+  a.B = B; a.H = H; a.L = L; a.d = d;
+  a.mask = mask;
+  a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(d));
+  a.stream = static_cast<cudaStream_t>(stream);
+  a.err = di->err;
+  a.wait_limit_ns = kWaitLimitNs;
+  if (!tensor_core) return launch_simt(a, dtype == JVP_BF16);
+
+  int dev = 0;
+  cudaGetDevice(&dev);
+  WorkList w;
+  rc = get_worklist(dev, mask, L, &w);
+  if (rc != JVP_OK) return rc;
+  return launch_sm100(a, w, di->sms);
+}
+
+int jvp_attn_mask_stats(jvp_mask_desc mask, int L, int bm, int bn, int64_t* pairs,
+                        int64_t* full, int64_t* partial, int64_t* empty) {
+  int rc = validate_mask(mask, L);
+  if (rc != JVP_OK) return rc;
+  if (bm < 1 || bn < 1) return JVP_ERR_INVALID_ARG;
+  if (pairs) *pairs = count_pairs(mask, L);
+  if (full || partial || empty) {
+    const int n_qt = (L + bm - 1) / bm, n_kt = (L + bn - 1) / bn;
+    std::vector<int8_t> row(n_kt);
+    int64_t cnt[3] = {0, 0, 0};
+    for (int qt = 0; qt < n_qt; ++qt) {
+      classify_qtile(mask, L, bm, bn, qt, row.data());
+      for (int8_t c : row) ++cnt[c];
+    }
+    if (full) *full = cnt[JVP_TILE_FULL];
+    if (partial) *partial = cnt[JVP_TILE_PARTIAL];
+    if (empty) *empty = cnt[JVP_TILE_EMPTY];
+  }
+  return JVP_OK;
+}
+
+int jvp_attn_tile_classes(jvp_mask_desc mask, int L, int bm, int bn, int8_t* out,
+                          int64_t out_len) {
+  int rc = validate_mask(mask, L);
+  if (rc != JVP_OK) return rc;
+  if (bm < 1 || bn < 1 || !out) return JVP_ERR_INVALID_ARG;
+  const int n_qt = (L + bm - 1) / bm, n_kt = (L + bn - 1) / bn;
+  if (out_len < (int64_t)n_qt * n_kt) return JVP_ERR_INVALID_ARG;
+  for (int qt = 0; qt < n_qt; ++qt) classify_qtile(mask, L, bm, bn, qt, out + (int64_t)qt * n_kt);
+  return JVP_OK;
+}
+
+int jvp_attn_schedule(jvp_mask_desc mask, int L, int bm, int bn, int32_t* qtiles, int qtile_cap,
+                      int32_t* segs, int seg_cap, int* n_qtiles, int* n_segs) {
+  int rc = validate_mask(mask, L);
+  if (rc != JVP_OK) return rc;
+  if (bm < 1 || bn < 1) return JVP_ERR_INVALID_ARG;
+  const Schedule s = build_schedule(mask, L, bm, bn);
+  const int nq = int(s.qtiles.size() / 4), ns = int(s.segs.size() / 2);
+  if (n_qtiles) *n_qtiles = nq;
+  if (n_segs) *n_segs = ns;
+  if (!qtiles || !segs || qtile_cap < nq || seg_cap < ns) return JVP_ERR_INVALID_ARG;
+  std::memcpy(qtiles, s.qtiles.data(), s.qtiles.size() * sizeof(int32_t));
+  for (int i = 0; i < ns; ++i) {
+    segs[3 * i] = s.segs[2 * i];
+    segs[3 * i + 1] = s.segs[2 * i + 1] >> 1;
+    segs[3 * i + 2] = s.segs[2 * i + 1] & 1;
+  }
+  return JVP_OK;
+}
+
+int jvp_attn_check_device_error(void* stream) {
+  DevInfo* di = nullptr;
+  int rc = device_info(&di);
+  if (rc != JVP_OK) return rc;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JVP_ERR_LAUNCH_FAILED;
+  unsigned w = 0;
+  if (cudaMemcpy(&w, di->err, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return JVP_ERR_LAUNCH_FAILED;
+  if (w != 0 && cudaMemset(di->err, 0, sizeof(unsigned)) != cudaSuccess)
+    return JVP_ERR_LAUNCH_FAILED;
+  if (w & kErrTimeout) return JVP_ERR_DEVICE_TIMEOUT;
+  if (w & kErrBounds) return JVP_ERR_DEVICE_BOUNDS;
+  return JVP_OK;
+}
+
+int jvp_attn_release(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int cur = 0;
+  const bool have_dev = cudaGetDevice(&cur) == cudaSuccess;
+  int rc = JVP_OK;
+  for (auto& kv : g_ws) {
+    if (cudaSetDevice(kv.first.dev) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess ||
+        cudaFree(kv.second.buf) != cudaSuccess)
+      rc = JVP_ERR_LAUNCH_FAILED;
+  }
+  g_ws.clear();
+  if (have_dev) cudaSetDevice(cur);
+  return rc;
+}
+
+const char* jvp_attn_strerror(int code) {
+  switch (code) {
+    case JVP_OK: return "success";
+    case JVP_ERR_INVALID_ARG: return "invalid argument";
+    case JVP_ERR_SHAPE_MISMATCH: return "sequence length does not match the mask descriptor";
+    case JVP_ERR_UNSUPPORTED_HEAD_DIM: return "unsupported head dimension";
+    case JVP_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+    case JVP_ERR_LAUNCH_FAILED: return "CUDA launch or runtime error";
+    case JVP_ERR_DEVICE_TIMEOUT: return "kernel gave up on a bounded wait";
+    case JVP_ERR_DEVICE_BOUNDS: return "kernel saw an out-of-range tile index";
+    case JVP_ERR_OUT_OF_MEMORY: return "workspace allocation failed";
+    case JVP_ERR_UNSUPPORTED_DEVICE: return "current device is not sm_100";
+    case JVP_ERR_TOO_LARGE: return "sizes exceed the kernel's index range";
+    default: return "unknown error code";
+  }
+}
+
+int jvp_attn_version(void) { return JVP_ATTN_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,609 @@
+// Tensor-core masked attention JVP for B200 (sm_100a): tcgen05 + TMEM + TMA.
+//
+// Computes, per (batch*head, query tile of 128 rows), in one streaming pass
+// over the admissible key tiles of 64 keys (Causal-rCM report, Appendix B,
+// Eq. 42-45):
+//   S   = Q K^T                         (d-deep MMA, fp32 in TMEM)
+//   dS  = dQ K^T + Q dK^T               (one 2d-deep contraction in TMEM)
+//   e   = 2^(c2 S - m)                  (c2 = scale * log2 e; m = row max)
+//   l  += sum e,  g += sum e dS         (row state in registers)
+//   A1  += e V                          (TMEM accumulator, 128 x 128 fp32)
+//   A23 += (scale e dS) V + e dV        (second TMEM accumulator)
+// finishing with O = A1/l, mu = scale g/l, dO = A23/l - mu O, and
+// LSE = (m + log2 l) ln 2. All accumulators share one running max m and one
+// rescale factor (Appendix B, after Eq. 45); the max is raised lazily, only
+// when a row's new maximum exceeds it by more than 2^8, which is exact
+// because the finish uses ratios only.
+//
+// Warp roles (256 threads, one CTA per SM, persistent over the work list):
+//   warp 0      TMA producer: Q/dQ per query tile, K/dK and V/dV rings of 2
+//   warp 1      TMEM owner and MMA issuer (one thread)
+//   warps 4..7  softmax/JVP state, P write-back to TMEM, epilogue
+// TMEM (512 columns): S/dS double buffer at [0,256): buffer b holds S in
+// columns [128b, 128b+64) and dS in [128b+64, 128b+128); the bf16 operands
+// e and scale*e*dS overwrite the first 32 columns of S and dS of their
+// buffer. A1 at [256,384), A23 at [384,512). MMA order per CTA is
+// S(0) S(1) PV(0) S(2) PV(1) S(3) ..., so the softmax of tile t overlaps
+// PV(t-1) and S(t+1) on the tensor pipe.
+//
+// Every mbarrier wait is bounded: on expiry the CTA records a timeout in the
+// device error word, drains its own TMA copies and MMAs, frees TMEM and
+// exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "mask_rows.cuh"
+#include "sm100_ptx.cuh"
+
+namespace jvp {
+namespace sm100 {
+
+using namespace jvp::ptx;
+
+constexpr int BM = 128;  // query rows per tile = TMEM lanes
+constexpr int BN = 64;   // keys per tile
+constexpr int D = 128;   // head dim
+constexpr int kThreads = 256;
+constexpr float kTau = 8.0f;  // lazy rescale threshold, log2 units
+
+// Shared memory map (byte offsets from a 1024-aligned base). Every operand
+// tile is stored as two 128-byte-swizzled halves (head-dim columns 0-63 and
+// 64-127), each rows x 128 B, exactly as the TMA box {64, rows} lands.
+constexpr uint32_t kQHalf = BM * 128;          // 16 KB
+constexpr uint32_t kKHalf = BN * 128;          //  8 KB
+constexpr uint32_t SM_Q = 0;                   // Q  : 32 KB
+constexpr uint32_t SM_DQ = 2 * kQHalf;         // dQ : 32 KB
+constexpr uint32_t SM_K = 4 * kQHalf;          // K/dK ring: stage s at +32 KB*s
+constexpr uint32_t SM_V = SM_K + 2 * 4 * kKHalf;  // V/dV ring
+constexpr uint32_t kStageBytes = 4 * kKHalf;      // 32 KB: K|dK or V|dV
+constexpr uint32_t SM_BAR = SM_V + 2 * kStageBytes;  // 196608
+constexpr uint32_t kSmemBytes = SM_BAR + 256 + 1024;  // + barriers + align slack
+
+// Barrier slots (8 bytes each) inside SM_BAR.
+enum : uint32_t {
+  B_QFULL = 0,
+  B_QEMPTY = 1,
+  B_KFULL = 2,   // 2 slots
+  B_KEMPTY = 4,  // 2
+  B_VFULL = 6,   // 2
+  B_VEMPTY = 8,  // 2
+  B_SFULL = 10,  // 2
+  B_PFULL = 12,  // 2
+  B_PVDONE = 14,
+  B_AFREE = 15,
+  B_DRAIN = 16,
+  kNumBars = 17
+};
+constexpr uint32_t SM_TMEM_SLOT = SM_BAR + 8 * kNumBars;  // u32: TMEM base
+constexpr uint32_t SM_ABORT = SM_TMEM_SLOT + 4;           // u32: abort flag
+
+// TMEM columns.
+constexpr uint32_t TM_A1 = 256;
+constexpr uint32_t TM_A23 = 384;
+
+constexpr uint32_t IDESC_S = ptx::idesc_bf16(BM, BN, false, false);
+constexpr uint32_t IDESC_PV = ptx::idesc_bf16(BM, D, false, true);
+
+struct Params {
+  const int4* qtiles;  // {qt, seg_begin, seg_count, n_ktiles}
+  const int2* segs;    // {kt_begin, (count << 1) | partial}
+  int n_entries, n_segs, n_items, n_qt, n_kt;
+  int L;
+  jvp_mask_desc mask;
+  float scale, c2;
+  __nv_bfloat16* o;
+  __nv_bfloat16* d_o;
+  float* lse;
+  unsigned* err;
+  unsigned long long wait_limit_ns;
+};
+
+// Walks this CTA's (item, key tile) sequence; every role runs its own copy.
+struct Cursor {
+  int item, item_idx, bh, qt;
+  int seg, seg_end, kt, kt_end;
+  int j, n;
+  uint32_t t;  // ordinal of the tile among this CTA's tiles
+  bool partial, valid;
+
+  __device__ void load_seg(const Params& p) {
+    const int2 s = p.segs[seg];
+    kt = s.x;
+    kt_end = s.x + (s.y >> 1);
+    partial = (s.y & 1) != 0;
+    if (kt < 0 || kt_end > p.n_kt || kt_end <= kt) {
+      atomicOr(p.err, kErrBounds);
+      valid = false;
+    }
+  }
+  __device__ void load_item(const Params& p) {
+    valid = item < p.n_items;
+    if (!valid) return;
+    const int e = item % p.n_entries;
+    bh = item / p.n_entries;
+    const int4 en = p.qtiles[e];
+    qt = en.x;
+    seg = en.y;
+    seg_end = en.y + en.z;
+    n = en.w;
+    j = 0;
+    if (qt < 0 || qt >= p.n_qt || seg < 0 || seg_end > p.n_segs || en.z < 1 || n < 1) {
+      atomicOr(p.err, kErrBounds);
+      valid = false;
+      return;
+    }
+    load_seg(p);
+  }
+  __device__ void start(const Params& p) {
+    item = blockIdx.x;
+    item_idx = 0;
+    t = 0;
+    load_item(p);
+  }
+  __device__ void next(const Params& p) {
+    ++t;
+    ++j;
+    if (++kt < kt_end) return;
+    if (++seg < seg_end) {
+      load_seg(p);
+      return;
+    }
+    item += gridDim.x;
+    ++item_idx;
+    load_item(p);
+  }
+};
+
+// Bounded wait. Returns false (and raises the CTA abort flag) on timeout or
+// when another role has already aborted.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Params& p,
+                                         volatile uint32_t* abort_flag) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 31u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > p.wait_limit_ns) {
+        atomicOr(p.err, kErrTimeout);
+        *abort_flag = 1u;
+        return false;
+      }
+    }
+  }
+}
+
+// Short bounded wait used only while cleaning up after an abort.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try(bar, parity)) {
+    if (globaltimer() - t0 > 100000000ull) return;  // 0.1 s
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_dq,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_dk,
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_dv,
+                      const __grid_constant__ Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // Align the working base to 1024 B (required by the 128-byte swizzle atoms).
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const base_ptr = smem_raw + (base - raw);
+  auto bar = [&](uint32_t slot) { return base + SM_BAR + 8u * slot; };
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + SM_ABORT);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_QFULL), 1);
+    mbar_init(bar(B_QEMPTY), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(B_KFULL + s), 1);
+      mbar_init(bar(B_KEMPTY + s), 1);
+      mbar_init(bar(B_VFULL + s), 1);
+      mbar_init(bar(B_VEMPTY + s), 1);
+      mbar_init(bar(B_SFULL + s), 1);
+      mbar_init(bar(B_PFULL + s), BM);
+    }
+    mbar_init(bar(B_PVDONE), 1);
+    mbar_init(bar(B_AFREE), BM);
+    mbar_init(bar(B_DRAIN), 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tm_q);
+    tma_prefetch_map(&tm_dq);
+    tma_prefetch_map(&tm_k);
+    tma_prefetch_map(&tm_dk);
+    tma_prefetch_map(&tm_v);
+    tma_prefetch_map(&tm_dv);
+  }
+  if (warp == 1) {
+    tmem_alloc(base + SM_TMEM_SLOT, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base_ptr + SM_TMEM_SLOT);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA ----
+    if (lane == 0) {
+      Cursor c;
+      c.start(p);
+      // Parity of the latest arming of each full barrier, for abort cleanup.
+      int q_armed = 0, k_armed[2] = {0, 0}, v_armed[2] = {0, 0};
+      bool ok = true;
+      while (c.valid && ok) {
+        if (c.j == 0) {
+          if (c.item_idx > 0)
+            ok = wait_bar(bar(B_QEMPTY), (c.item_idx - 1) & 1, p, abort_flag);
+          if (!ok) break;
+          mbar_expect_tx(bar(B_QFULL), 4 * kQHalf);
+          ++q_armed;
+          const int y = c.qt * BM;
+          tma_load_3d(base + SM_Q, &tm_q, bar(B_QFULL), 0, y, c.bh);
+          tma_load_3d(base + SM_Q + kQHalf, &tm_q, bar(B_QFULL), 64, y, c.bh);
+          tma_load_3d(base + SM_DQ, &tm_dq, bar(B_QFULL), 0, y, c.bh);
+          tma_load_3d(base + SM_DQ + kQHalf, &tm_dq, bar(B_QFULL), 64, y, c.bh);
+        }
+        const uint32_t s = c.t & 1u, u = c.t >> 1;
+        const int y = c.kt * BN;
+        if (c.t >= 2) ok = wait_bar(bar(B_KEMPTY + s), (u - 1) & 1u, p, abort_flag);
+        if (!ok) break;
+        mbar_expect_tx(bar(B_KFULL + s), kStageBytes);
+        ++k_armed[s];
+        const uint32_t ks = base + SM_K + s * kStageBytes;
+        tma_load_3d(ks, &tm_k, bar(B_KFULL + s), 0, y, c.bh);
+        tma_load_3d(ks + kKHalf, &tm_k, bar(B_KFULL + s), 64, y, c.bh);
+        tma_load_3d(ks + 2 * kKHalf, &tm_dk, bar(B_KFULL + s), 0, y, c.bh);
+        tma_load_3d(ks + 3 * kKHalf, &tm_dk, bar(B_KFULL + s), 64, y, c.bh);
+        if (c.t >= 2) ok = wait_bar(bar(B_VEMPTY + s), (u - 1) & 1u, p, abort_flag);
+        if (!ok) break;
+        mbar_expect_tx(bar(B_VFULL + s), kStageBytes);
+        ++v_armed[s];
+        const uint32_t vs = base + SM_V + s * kStageBytes;
+        tma_load_3d(vs, &tm_v, bar(B_VFULL + s), 0, y, c.bh);
+        tma_load_3d(vs + kKHalf, &tm_v, bar(B_VFULL + s), 64, y, c.bh);
+        tma_load_3d(vs + 2 * kKHalf, &tm_dv, bar(B_VFULL + s), 0, y, c.bh);
+        tma_load_3d(vs + 3 * kKHalf, &tm_dv, bar(B_VFULL + s), 64, y, c.bh);
+        c.next(p);
+      }
+      if (!ok) {
+        // Let copies already issued land before the CTA's smem is released.
+        if (q_armed) drain_wait(bar(B_QFULL), (q_armed - 1) & 1);
+        for (int s = 0; s < 2; ++s) {
+          if (k_armed[s]) drain_wait(bar(B_KFULL + s), (k_armed[s] - 1) & 1);
+          if (v_armed[s]) drain_wait(bar(B_VFULL + s), (v_armed[s] - 1) & 1);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA ----
+    if (lane == 0) {
+      bool ok = true;
+      auto issue_s = [&](const Cursor& c) -> bool {
+        const uint32_t b = c.t & 1u;
+        if (c.j == 0 && !wait_bar(bar(B_QFULL), c.item_idx & 1, p, abort_flag)) return false;
+        if (!wait_bar(bar(B_KFULL + b), (c.t >> 1) & 1u, p, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t d_s = tmem + b * 128u, d_ds = d_s + 64u;
+        const uint32_t kb = base + SM_K + b * kStageBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t oq = (kk >> 2) * kQHalf + (kk & 3) * 32;
+          const uint32_t ok_ = (kk >> 2) * kKHalf + (kk & 3) * 32;
+          mma_ss(d_s, sdesc_sw128(base + SM_Q + oq, 16, 1024),
+                 sdesc_sw128(kb + ok_, 16, 1024), IDESC_S, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t oq = (kk >> 2) * kQHalf + (kk & 3) * 32;
+          const uint32_t ok_ = (kk >> 2) * kKHalf + (kk & 3) * 32;
+          mma_ss(d_ds, sdesc_sw128(base + SM_DQ + oq, 16, 1024),
+                 sdesc_sw128(kb + ok_, 16, 1024), IDESC_S, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t oq = (kk >> 2) * kQHalf + (kk & 3) * 32;
+          const uint32_t ok_ = (kk >> 2) * kKHalf + (kk & 3) * 32;
+          mma_ss(d_ds, sdesc_sw128(base + SM_Q + oq, 16, 1024),
+                 sdesc_sw128(kb + 2 * kKHalf + ok_, 16, 1024), IDESC_S, 1u);
+        }
+        mma_commit(bar(B_KEMPTY + b));
+        mma_commit(bar(B_SFULL + b));
+        if (c.j == c.n - 1) mma_commit(bar(B_QEMPTY));
+        return true;
+      };
+      auto issue_pv = [&](const Cursor& c) -> bool {
+        const uint32_t b = c.t & 1u;
+        if (c.j == 0 && c.item_idx > 0 &&
+            !wait_bar(bar(B_AFREE), (c.item_idx - 1) & 1, p, abort_flag))
+          return false;
+        if (!wait_bar(bar(B_PFULL + b), (c.t >> 1) & 1u, p, abort_flag)) return false;
+        if (!wait_bar(bar(B_VFULL + b), (c.t >> 1) & 1u, p, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t vb = base + SM_V + b * kStageBytes;
+        const uint32_t a_p = tmem + b * 128u, a_pd = a_p + 64u;
+        const uint32_t first = c.j == 0 ? 0u : 1u;
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks)
+          mma_ts(tmem + TM_A1, a_p + ks * 8, sdesc_sw128(vb + ks * 2048, kKHalf, 1024),
+                 IDESC_PV, first | (ks > 0));
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks)
+          mma_ts(tmem + TM_A23, a_pd + ks * 8, sdesc_sw128(vb + ks * 2048, kKHalf, 1024),
+                 IDESC_PV, first | (ks > 0));
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks)
+          mma_ts(tmem + TM_A23, a_p + ks * 8,
+                 sdesc_sw128(vb + 2 * kKHalf + ks * 2048, kKHalf, 1024), IDESC_PV, 1u);
+        mma_commit(bar(B_VEMPTY + b));
+        mma_commit(bar(B_PVDONE));
+        return true;
+      };
+      Cursor cs, cp;
+      cs.start(p);
+      cp.start(p);
+      for (int pre = 0; pre < 2 && cs.valid && ok; ++pre) {
+        ok = issue_s(cs);
+        cs.next(p);
+      }
+      while (cp.valid && ok) {
+        ok = issue_pv(cp);
+        cp.next(p);
+        if (ok && cs.valid) {
+          ok = issue_s(cs);
+          cs.next(p);
+        }
+      }
+      if (!ok) {
+        // Wait for every MMA this thread issued before TMEM is freed.
+        mma_commit(bar(B_DRAIN));
+        drain_wait(bar(B_DRAIN), 0);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ----------------------------------------------------- softmax / JVP ----
+    const int r = threadIdx.x - 128;                 // row within the tile
+    const uint32_t tl = tmem + (uint32_t(r & ~31) << 16);  // this warp's lane quarter
+    const int chunk = p.mask.chunk < 1 ? 1 : p.mask.chunk;
+    Cursor c;
+    c.start(p);
+    float m_ref = -CUDART_INF_F, l = 0.f, g = 0.f;
+    RowKeys rk{0, 0, 0, 0};
+    int grow = 0;
+    bool ok = true;
+    while (c.valid) {
+      if (c.j == 0) {
+        grow = c.qt * BM + r;
+        rk = row_keys(p.mask.mode, p.mask.tokens_per_frame, p.mask.n_frames, chunk, p.L, grow);
+        m_ref = -CUDART_INF_F;
+        l = 0.f;
+        g = 0.f;
+      }
+      const uint32_t b = c.t & 1u;
+      ok = wait_bar(bar(B_SFULL + b), (c.t >> 1) & 1u, p, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      uint32_t sr0[32], sr1[32], dr0[32], dr1[32];
+      tmem_ld32(tl + b * 128u, sr0);
+      tmem_ld32(tl + b * 128u + 32u, sr1);
+      tmem_ld32(tl + b * 128u + 64u, dr0);
+      tmem_ld32(tl + b * 128u + 96u, dr1);
+      tmem_wait_ld();
+      float s[64];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        s[i] = __uint_as_float(sr0[i]);
+        s[32 + i] = __uint_as_float(sr1[i]);
+      }
+      if (c.partial) {
+        const int k0 = c.kt * BN;
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (!key_ok(rk, k0 + i)) s[i] = -CUDART_INF_F;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int i = 1; i < 64; ++i) mx = fmaxf(mx, s[i]);
+      const float mxs = mx * p.c2;
+      float alpha = 1.f;
+      bool need = false;
+      if (m_ref == -CUDART_INF_F) {
+        m_ref = mxs;  // first admitted keys of this row: nothing to rescale yet
+      } else if (mxs > m_ref + kTau) {
+        alpha = ex2(m_ref - mxs);
+        m_ref = mxs;
+        need = true;
+      }
+      if (__any_sync(0xffffffffu, need)) {
+        l *= alpha;
+        g *= alpha;
+        // A1/A23 hold PV(t-1); wait for it, then scale this warp's rows.
+        ok = wait_bar(bar(B_PVDONE), (c.t - 1) & 1u, p, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const uint32_t col = (q4 < 4 ? TM_A1 : TM_A23) + (q4 & 3) * 32u;
+          uint32_t a[32];
+          tmem_ld32(tl + col, a);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) * alpha);
+          tmem_st32(tl + col, a);
+        }
+        tmem_wait_st();
+      }
+      const float mref_use = m_ref == -CUDART_INF_F ? 0.f : m_ref;
+      uint32_t pp[32], pd[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float ds0 = __uint_as_float(i < 16 ? dr0[2 * i] : dr1[2 * i - 32]);
+        const float ds1 = __uint_as_float(i < 16 ? dr0[2 * i + 1] : dr1[2 * i - 31]);
+        const float e0 = ex2(fmaf(s[2 * i], p.c2, -mref_use));
+        const float e1 = ex2(fmaf(s[2 * i + 1], p.c2, -mref_use));
+        const float ed0 = e0 * ds0, ed1 = e1 * ds1;
+        l += e0 + e1;
+        g += ed0 + ed1;
+        pp[i] = pack_bf16(e0, e1);
+        pd[i] = pack_bf16(ed0 * p.scale, ed1 * p.scale);
+      }
+      tmem_st32(tl + b * 128u, pp);
+      tmem_st32(tl + b * 128u + 64u, pd);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_PFULL + b));
+
+      if (c.j == c.n - 1) {
+        // ------------------------------------------------------ epilogue --
+        // PV(t-1) may still be running here, i.e. the barrier may be two
+        // phases short of PV(t); a parity wait is only unambiguous one phase
+        // ahead, so wait for PV(t-1) first, then for PV(t).
+        ok = c.t == 0 || wait_bar(bar(B_PVDONE), (c.t - 1) & 1u, p, abort_flag);
+        ok = ok && wait_bar(bar(B_PVDONE), c.t & 1u, p, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float mu = p.scale * g * inv;
+        const bool row_ok = grow < p.L;
+        const size_t off = (size_t(c.bh) * p.L + (row_ok ? grow : 0)) * D;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t a1[32], a23[32];
+          tmem_ld32(tl + TM_A1 + cc * 32u, a1);
+          tmem_ld32(tl + TM_A23 + cc * 32u, a23);
+          tmem_wait_ld();
+          uint32_t po[16], pdo[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float o0 = __uint_as_float(a1[2 * i]) * inv;
+            const float o1 = __uint_as_float(a1[2 * i + 1]) * inv;
+            const float d0 = __uint_as_float(a23[2 * i]) * inv - mu * o0;
+            const float d1 = __uint_as_float(a23[2 * i + 1]) * inv - mu * o1;
+            po[i] = pack_bf16(o0, o1);
+            pdo[i] = pack_bf16(d0, d1);
+          }
+          if (row_ok) {
+            uint4* go = reinterpret_cast<uint4*>(p.o + off + cc * 32);
+            uint4* gd = reinterpret_cast<uint4*>(p.d_o + off + cc * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              go[i] = make_uint4(po[4 * i], po[4 * i + 1], po[4 * i + 2], po[4 * i + 3]);
+              gd[i] = make_uint4(pdo[4 * i], pdo[4 * i + 1], pdo[4 * i + 2], pdo[4 * i + 3]);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(B_AFREE));
+        if (row_ok)
+          p.lse[size_t(c.bh) * p.L + grow] =
+              l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+      }
+      c.next(p);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- host ----
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [BH, L, 128] bf16 viewed as a 3-D tensor (d innermost); box {64, rows, 1}.
+static bool make_map(CUtensorMap* m, const void* ptr, int L, int BH, int rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(L), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(L) * D * 2};
+  cuuint32_t box[3] = {64, cuuint32_t(rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace sm100
+
+int launch_sm100(const LaunchArgs& a, const WorkList& w, int num_sms) {
+  using namespace sm100;
+  const int BH = a.B * a.H;
+  CUtensorMap mq, mdq, mk, mdk, mv, mdv;
+  if (!make_map(&mq, a.q, a.L, BH, BM) || !make_map(&mdq, a.dq, a.L, BH, BM) ||
+      !make_map(&mk, a.k, a.L, BH, BN) || !make_map(&mdk, a.dk, a.L, BH, BN) ||
+      !make_map(&mv, a.v, a.L, BH, BN) || !make_map(&mdv, a.dv, a.L, BH, BN))
+    return JVP_ERR_LAUNCH_FAILED;
+  Params p;
+  p.qtiles = w.qtiles;
+  p.segs = w.segs;
+  p.n_entries = w.n_qtiles;
+  p.n_segs = w.n_segs;
+  const long long items = (long long)w.n_qtiles * BH;
+  if (items > 0x7fffffffLL) return JVP_ERR_TOO_LARGE;
+  p.n_items = int(items);
+  p.n_qt = (a.L + BM - 1) / BM;
+  p.n_kt = (a.L + BN - 1) / BN;
+  p.L = a.L;
+  p.mask = a.mask;
+  p.scale = a.scale;
+  p.c2 = a.scale * 1.4426950408889634f;
+  p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.d_o = static_cast<__nv_bfloat16*>(a.d_o);
+  p.lse = a.lse;
+  p.err = a.err;
+  p.wait_limit_ns = a.wait_limit_ns;
+  // The dynamic shared-memory opt-in is a per-device function attribute.
+  static std::mutex attr_mu;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return JVP_ERR_LAUNCH_FAILED;
+  {
+    std::lock_guard<std::mutex> lk(attr_mu);
+    if (!attr_done[dev]) {
+      if (cudaFuncSetAttribute(jvp_attn_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kSmemBytes) != cudaSuccess)
+        return JVP_ERR_LAUNCH_FAILED;
+      attr_done[dev] = true;
+    }
+  }
+  const int grid = int(items < num_sms ? items : num_sms);
+  jvp_attn_sm100_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mdq, mk, mdk, mv, mdv, p);
+  return cudaGetLastError() == cudaSuccess ? JVP_OK : JVP_ERR_LAUNCH_FAILED;
+}
+
+}  // namespace jvp

@@ -1,0 +1,122 @@
+// Host-side mask -> tile work list (see schedule.h).
+#include "schedule.h"
+
+#include <algorithm>
+#include <limits>
+
+#include "mask_rows.cuh"
+
+namespace jvp {
+
+int validate_mask(const jvp_mask_desc& m, int L) {
+  if (m.mode < JVP_MASK_DENSE || m.mode > JVP_MASK_TEACHER_FORCING)
+    return JVP_ERR_INVALID_ARG;
+  if (m.tokens_per_frame < 1 || m.n_frames < 1 || L < 1)
+    return JVP_ERR_INVALID_ARG;
+  if (m.chunk < 1 && m.mode != JVP_MASK_DENSE && m.mode != JVP_MASK_FRAME_CAUSAL)
+    return JVP_ERR_INVALID_ARG;
+  const int64_t ft = int64_t(m.tokens_per_frame) * m.n_frames;
+  const int64_t want = m.mode == JVP_MASK_TEACHER_FORCING ? 2 * ft : ft;
+  if (want > std::numeric_limits<int32_t>::max() / 2) return JVP_ERR_TOO_LARGE;
+  if (want != L) return JVP_ERR_SHAPE_MISMATCH;
+  return JVP_OK;
+}
+
+static inline int chunk_of(const jvp_mask_desc& m) {
+  return m.chunk < 1 ? 1 : m.chunk;
+}
+
+int64_t count_pairs(const jvp_mask_desc& m, int L) {
+  int64_t total = 0;
+  for (int i = 0; i < L; ++i) {
+    RowKeys r = row_keys(m.mode, m.tokens_per_frame, m.n_frames, chunk_of(m), L, i);
+    if (r.b0 > r.a0) total += r.b0 - r.a0;
+    if (r.b1 > r.a1) total += r.b1 - r.a1;
+  }
+  return total;
+}
+
+static inline int overlap(int a, int b, int lo, int hi) {
+  const int x = std::max(a, lo), y = std::min(b, hi);
+  return y > x ? y - x : 0;
+}
+
+void classify_qtile(const jvp_mask_desc& m, int L, int bm, int bn, int qt,
+                    int8_t* out) {
+  const int n_kt = (L + bn - 1) / bn;
+  const int r0 = qt * bm;
+  const int r1 = std::min(r0 + bm, L);
+  // Distinct row classes of this query tile (consecutive rows mostly share
+  // their admissible intervals; a tile spans few frames).
+  std::vector<RowKeys> cls;
+  for (int i = r0; i < r1; ++i) {
+    RowKeys r = row_keys(m.mode, m.tokens_per_frame, m.n_frames, chunk_of(m), L, i);
+    if (cls.empty() || cls.back().a0 != r.a0 || cls.back().b0 != r.b0 ||
+        cls.back().a1 != r.a1 || cls.back().b1 != r.b1)
+      cls.push_back(r);
+  }
+  for (int kt = 0; kt < n_kt; ++kt) {
+    const int k0 = kt * bn;
+    const int k1 = std::min(k0 + bn, L);
+    const bool ragged = k0 + bn > L;
+    bool all = !ragged, any = false;
+    for (const RowKeys& r : cls) {
+      const int ov = overlap(r.a0, r.b0, k0, k1) + overlap(r.a1, r.b1, k0, k1);
+      if (ov != k1 - k0) all = false;
+      if (ov > 0) any = true;
+    }
+    out[kt] = all ? JVP_TILE_FULL : (any ? JVP_TILE_PARTIAL : JVP_TILE_EMPTY);
+  }
+}
+
+Schedule build_schedule(const jvp_mask_desc& m, int L, int bm, int bn) {
+  Schedule s;
+  s.L = L;
+  s.bm = bm;
+  s.bn = bn;
+  s.n_qt = (L + bm - 1) / bm;
+  s.n_kt = (L + bn - 1) / bn;
+  std::vector<int8_t> row(s.n_kt);
+  struct Entry {
+    int qt, seg_begin, seg_count, n_kt;
+  };
+  std::vector<Entry> entries;
+  entries.reserve(s.n_qt);
+  for (int qt = 0; qt < s.n_qt; ++qt) {
+    classify_qtile(m, L, bm, bn, qt, row.data());
+    Entry e{qt, int(s.segs.size() / 2), 0, 0};
+    int kt = 0;
+    while (kt < s.n_kt) {
+      const int8_t c = row[kt];
+      if (c == JVP_TILE_EMPTY) {
+        ++s.n_empty;
+        ++kt;
+        continue;
+      }
+      int k2 = kt;
+      while (k2 < s.n_kt && row[k2] == c) ++k2;
+      const int cnt = k2 - kt;
+      s.segs.push_back(kt);
+      s.segs.push_back((cnt << 1) | (c == JVP_TILE_PARTIAL ? 1 : 0));
+      if (c == JVP_TILE_FULL) s.n_full += cnt; else s.n_partial += cnt;
+      e.seg_count += 1;
+      e.n_kt += cnt;
+      kt = k2;
+    }
+    entries.push_back(e);
+    s.max_ktiles = std::max<int64_t>(s.max_ktiles, e.n_kt);
+  }
+  // Longest-processing-time-first order for the persistent grid.
+  std::stable_sort(entries.begin(), entries.end(),
+                   [](const Entry& a, const Entry& b) { return a.n_kt > b.n_kt; });
+  s.qtiles.reserve(entries.size() * 4);
+  for (const Entry& e : entries) {
+    s.qtiles.push_back(e.qt);
+    s.qtiles.push_back(e.seg_begin);
+    s.qtiles.push_back(e.seg_count);
+    s.qtiles.push_back(e.n_kt);
+  }
+  return s;
+}
+
+}  // namespace jvp

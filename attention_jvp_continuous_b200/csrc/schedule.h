@@ -1,0 +1,43 @@
+// Host-side mask -> tile work list.
+//
+// The Causal-rCM report (Appendix B, "Sparse custom-mask representation")
+// streams only admissible query/key rectangles. Here the rectangles are the
+// tiles of one global grid (query tiles of bm rows, key tiles of bn keys,
+// anchored at token 0) and each tile is FULL (every in-range slot admitted),
+// PARTIAL (some) or EMPTY (none, never visited). Keeping the global grid
+// rather than restarting tiles at every range edge wastes fewer slots on
+// ragged frame sizes (1560 = 12*128 + 24 tokens per frame).
+#pragma once
+
+#include <stdint.h>
+
+#include <vector>
+
+#include "../../include/jvp_attn.h"
+
+namespace jvp {
+
+// Returns JVP_OK or the error code for a bad descriptor / length.
+int validate_mask(const jvp_mask_desc& m, int L);
+
+// Admitted (query, key) pairs over all L rows.
+int64_t count_pairs(const jvp_mask_desc& m, int L);
+
+struct Schedule {
+  int L = 0, bm = 0, bn = 0, n_qt = 0, n_kt = 0;
+  int64_t n_full = 0, n_partial = 0, n_empty = 0;
+  int64_t max_ktiles = 0;  // longest query tile, in key tiles
+  // Per query tile, longest first: {qt, seg_begin, seg_count, n_ktiles}.
+  std::vector<int32_t> qtiles;
+  // Segments: {kt_begin, (kt_count << 1) | partial}.
+  std::vector<int32_t> segs;
+};
+
+// Classifies one query tile's key tiles into out[0 .. n_kt).
+void classify_qtile(const jvp_mask_desc& m, int L, int bm, int bn, int qt,
+                    int8_t* out);
+
+// Builds the full schedule. The mask must already be validated.
+Schedule build_schedule(const jvp_mask_desc& m, int L, int bm, int bn);
+
+}  // namespace jvp

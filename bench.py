@@ -1,0 +1,403 @@
+#!/usr/bin/env python
+"""Throughput of the masked attention JVP on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload tf|frame_causal|chunk_tf|tf_long]
+
+One step is one call of the whole hot path (mask -> tile work list, the
+score / score-tangent contractions, the online softmax and JVP state, the
+three PV-type accumulations and the finish) over one synthetic batch of
+the 65,520-token teacher-forcing workload (B=1, H=12, d=128; 21 frames of
+1560 tokens, clean + noisy). Throughput counts 12*d FLOPs per admitted
+(query, key) pair.
+
+Multi-GPU (launched by torch.distributed.run): every rank runs its own,
+independently seeded batch (weak scaling, no collective on the data path);
+the timed region is bracketed by barriers and the slowest rank's time is
+reported. Rank 0 prints one JSON line.
+
+``--impl reference`` times the float64 CPU oracle on this machine's host cores
+instead (rank 0 only), on a bounded sample of query rows per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention-JVP TFLOP/s (12*d per unmasked pair) and % of B200 bf16 tensor peak"
+UNIT = "TFLOP/s"
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+KERNEL_SOURCES = ["attention_jvp_continuous_b200/csrc/jvp_attn_sm100.cu",
+                  "attention_jvp_continuous_b200/csrc/sm100_ptx.cuh",
+                  "attention_jvp_continuous_b200/csrc/mask_rows.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+# ------------------------------------------------------------ host logic --
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken
+    on the current kernel source; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("kernel_hash") != kernel_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def flops_per_step(w, pairs_per_head: int) -> float:
+    return 12.0 * w.d * pairs_per_head * w.B * w.H
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Independent, reproducible input stream per rank."""
+    return base_seed + 1000003 * rank
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, bus_id: str | None):
+        self.bus_id = (bus_id or "").lower()
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], [], set()
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                if self.bus_id and parts[0].lower()[-len(self.bus_id):] != self.bus_id[-12:] \
+                        and not parts[0].lower().endswith(self.bus_id[-12:]):
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(self.NAMES, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ---------------------------------------------------------------- our arm --
+
+def run_ours(args, w):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import attention_jvp_continuous_b200 as ja
+    from attention_jvp_continuous_b200.inputs import make_inputs
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    ja._lib.lib()  # fail loudly if the CUDA library is missing
+    mask = ja.Mask(w.mode, w.tokens_per_frame, w.n_frames, w.chunk)
+    pairs, n_full, n_part, _ = ja.mask_stats(mask)
+    flops = flops_per_step(w, pairs)
+
+    inputs, _ = make_inputs(w, device="cuda", seed=rank_seed(w.seed, rank))
+    q = inputs[0]
+    o = torch.empty_like(q)
+    d_o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=q.device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ja.jvp_attn_fwd(*inputs, o, d_o, lse, mask)
+
+    for _ in range(args.warmup):
+        step()
+    ja.check_device_error()
+
+    # ---- device-timed region (inputs resident in HBM) ----
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    bus = getattr(torch.cuda.get_device_properties(local), "pci_bus_id", None)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(bus) as clk:
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ja.check_device_error()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    total_ms_max = max_over_ranks(total_ms, world)
+    value = flops * args.steps * world / (total_ms_max * 1e-3) / 1e12
+    launch_ms = sum(per) / len(per)
+
+    # ---- end to end through the C ABI: pinned host in, host out ----
+    host_in = [t.cpu().pin_memory() for t in inputs]
+    host_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    host_do = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    host_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    dev_in = [torch.empty_like(t) for t in inputs]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in (host_o, host_do, host_lse))
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        for d, h in zip(dev_in, host_in):
+            d.copy_(h, non_blocking=True)
+        ja.jvp_attn_fwd(*dev_in, o, d_o, lse, mask)
+        host_o.copy_(o, non_blocking=True)
+        host_do.copy_(d_o, non_blocking=True)
+        host_lse.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ja.check_device_error()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+
+    clocks = clk.summary()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (launch_ms * 1e-3) / 1e12
+    traffic = stored_traffic(w.name)
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms_max / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": f"{w.name}: teacher-forcing mask, B={w.B} H={w.H} d={w.d}, "
+                        f"{w.n_frames} frames x {w.tokens_per_frame} tokens x "
+                        f"{{clean,noisy}} = {w.L} tokens, chunk={w.chunk}",
+            "B": w.B, "H": w.H, "L": w.L, "d": w.d, "mode": w.mode,
+            "tokens_per_frame": w.tokens_per_frame, "n_frames": w.n_frames, "chunk": w.chunk,
+            "pairs_per_head": pairs, "flops_per_step": flops,
+            "tiles_128x64_per_head": {"full": n_full, "partial": n_part},
+            "l2": "inputs larger than L2 (%.2f GB read per step vs 126 MB L2); no flush"
+                  % (h2d / 1e9),
+            "parallelism": f"dp{world} (independent problems per rank, no data collective)",
+        },
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "roofline": {
+            "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": UNIT,
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
+            "frac_of_sustained": round(achieved / float(peaks.get(
+                "bf16_tflops_sustained", peak)), 4),
+            "frac_of_nominal_2250": round(achieved / NOMINAL_BF16_TFLOPS, 4),
+            "kernel": "jvp_attn_sm100_kernel", "launch_ms": round(launch_ms, 4),
+        },
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, inputs, rows_per_head=args.cpu_rows)
+    return line
+
+
+# ---------------------------------------------------- oracle on the host --
+
+def oracle_sample(w, host_inputs, rows_per_head: int, seed: int = 1234):
+    """Times the float64 oracle on ``rows_per_head`` seeded query rows of
+    every head; returns (seconds, sampled admitted pairs, threads)."""
+    import numpy as np
+
+    from attention_jvp_continuous_b200.inputs import sample_rows
+    from oracle import MaskSpec, jvp_attention, key_intervals
+
+    spec = MaskSpec(w.mode, w.tokens_per_frame, w.n_frames, w.chunk)
+    rows = sample_rows(w.L, rows_per_head, seed=seed)
+    pairs_per_head = sum(b - a for r in rows for a, b in key_intervals(spec, int(r)))
+    t0 = time.perf_counter()
+    jvp_attention(*host_inputs, spec, rows=rows)
+    dt = time.perf_counter() - t0
+    return dt, pairs_per_head * w.B * w.H
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(w, inputs, rows_per_head: int):
+    host = [t.cpu() for t in inputs]
+    dt, sp = oracle_sample(w, host, rows_per_head)
+    return {"value": round(12.0 * w.d * sp / dt / 1e12, 6), "unit": UNIT,
+            "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{rows_per_head} seeded query rows per head x {w.B * w.H} heads "
+                      f"({sp} admitted pairs, {dt:.1f} s, float64 numpy)"}
+
+
+def run_reference(args, w):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return None
+    from attention_jvp_continuous_b200.inputs import make_inputs
+    inputs, _ = make_inputs(w, device="cpu")
+    rows = args.ref_rows
+    for i in range(args.warmup):
+        oracle_sample(w, inputs, rows, seed=100 + i)
+    times, pairs = [], 0
+    for i in range(args.steps):
+        dt, sp = oracle_sample(w, inputs, rows, seed=1234 + i)
+        times.append(dt)
+        pairs += sp
+    total = sum(times)
+    value = 12.0 * w.d * pairs / total / 1e12
+    cores = blas_threads()
+    sample = f"{rows} seeded query rows per head x {w.B * w.H} heads per step"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / args.steps, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name} (oracle on sampled rows)", "B": w.B, "H": w.H,
+                   "L": w.L, "d": w.d, "mode": w.mode, "chunk": w.chunk,
+                   "parallelism": "host cores, rank 0 only"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__,
+                                 formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="tf",
+                    choices=["tf", "frame_causal", "chunk_tf", "tf_long"])
+    ap.add_argument("--cpu-rows", type=int, default=256,
+                    help="query rows per head in the cpu_baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=32,
+                    help="query rows per head per step of --impl reference")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from attention_jvp_continuous_b200.inputs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    world, rank, _ = dist_setup()
+    if world != args.gpus and args.impl == "ours":
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    line = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
+    if line is not None and rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

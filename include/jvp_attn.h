@@ -1,0 +1,183 @@
+/*
+ * jvp_attn.h -- C ABI of the B200 (sm_100a) masked attention JVP library.
+ *
+ * Operation (Causal-rCM tech report, Appendix B "FlashAttention-2 JVP Kernel
+ * with Custom Masks", Eq. 42-45): for every (batch b, head h) and query row i,
+ * with A_i the keys the temporal mask admits for i and c the softmax scale,
+ *
+ *   O_i   = sum_{j in A_i} p_ij V_j,      p_i = softmax_j( c <Q_i, K_j> )
+ *   dS_ij = c ( <dQ_i, K_j> + <Q_i, dK_j> )                     (Eq. 43)
+ *   dO_i  = sum_j p_ij (dS_ij - mu_i) V_j + sum_j p_ij dV_j,
+ *   mu_i  = sum_j p_ij dS_ij                                     (Eq. 44)
+ *   LSE_i = log sum_{j in A_i} exp(c <Q_i, K_j>)
+ *
+ * i.e. the primal attention output and its forward-mode tangent along
+ * (dQ, dK, dV), computed in one streaming pass. The mask has no tangent.
+ *
+ * Masks (jvp_mask_desc): the token sequence is frame-major with
+ * tokens_per_frame (T) tokens per frame, spatial attention within a frame
+ * always full; a chunk is `chunk` consecutive frames (the last may be short).
+ *   DENSE            L = F*T, every key.
+ *   FRAME_CAUSAL     L = F*T, key frame <= query frame (report Sec. 4.1 c1-1).
+ *   CHUNK_CAUSAL     L = F*T, key chunk <= query chunk: full inside a chunk,
+ *                    causal across chunks (report Sec. 2.3, block-causal).
+ *   TEACHER_FORCING  L = 2*F*T, sequence [clean ; noisy] (report Sec. 3.1.1,
+ *                    Eq. 8 and Table 2 notes). Clean queries see clean keys
+ *                    of chunks <= theirs; noisy queries see clean keys of
+ *                    chunks strictly before theirs plus the noisy keys of
+ *                    their own chunk.
+ * The library turns the descriptor into per-query-tile lists of admissible
+ * key tiles (report Appendix B, "Sparse custom-mask representation") and
+ * never materialises an L x L mask.
+ *
+ * Conventions for every call:
+ *  - Return 0 (JVP_OK) on success, a negative JVP_ERR_* code otherwise. No
+ *    C++ exception crosses this boundary. jvp_attn_strerror() names a code.
+ *  - Tensor pointers are caller-owned DEVICE memory on the current CUDA
+ *    device, contiguous row-major [B, H, L, d] (lse: [B, H, L] float32),
+ *    16-byte aligned. The library keeps no reference after the call returns.
+ *  - Launches are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream). Errors detected on the host are returned before any
+ *    launch; a kernel that gives up on a bounded wait records a device error
+ *    word, read by jvp_attn_check_device_error().
+ */
+#ifndef JVP_ATTN_H
+#define JVP_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define JVP_ATTN_VERSION 100 /* 1.0.0 */
+
+/* ---- error codes --------------------------------------------------------- */
+#define JVP_OK                         0
+#define JVP_ERR_INVALID_ARG           -1  /* null pointer, bad mode, B/H/L/d <= 0 */
+#define JVP_ERR_SHAPE_MISMATCH        -2  /* L inconsistent with the mask descriptor */
+#define JVP_ERR_UNSUPPORTED_HEAD_DIM  -3  /* see jvp_attn_fwd for supported d */
+#define JVP_ERR_MISALIGNED            -4  /* a tensor pointer not 16-byte aligned */
+#define JVP_ERR_LAUNCH_FAILED         -5  /* CUDA launch / runtime error */
+#define JVP_ERR_DEVICE_TIMEOUT        -6  /* a kernel gave up on a bounded wait */
+#define JVP_ERR_DEVICE_BOUNDS         -7  /* a kernel saw an out-of-range tile index */
+#define JVP_ERR_OUT_OF_MEMORY         -8  /* workspace allocation failed */
+#define JVP_ERR_UNSUPPORTED_DEVICE    -9  /* current device is not sm_100 */
+#define JVP_ERR_TOO_LARGE            -10  /* sizes overflow the kernel's index range */
+
+/* ---- mask descriptor ------------------------------------------------------ */
+typedef enum {
+  JVP_MASK_DENSE = 0,
+  JVP_MASK_FRAME_CAUSAL = 1,
+  JVP_MASK_CHUNK_CAUSAL = 2,
+  JVP_MASK_TEACHER_FORCING = 3
+} jvp_mask_mode;
+
+typedef struct {
+  int32_t mode;             /* jvp_mask_mode */
+  int32_t tokens_per_frame; /* T >= 1 */
+  int32_t n_frames;         /* F >= 1 (per half for TEACHER_FORCING) */
+  int32_t chunk;            /* frames per chunk >= 1; ignored by DENSE and
+                               FRAME_CAUSAL (which is chunk = 1) */
+} jvp_mask_desc;
+
+typedef enum { JVP_BF16 = 0, JVP_FP32 = 1 } jvp_dtype;
+
+/* Tile classes reported by jvp_attn_tile_classes(). */
+#define JVP_TILE_EMPTY   0
+#define JVP_TILE_FULL    1
+#define JVP_TILE_PARTIAL 2
+
+/* ---- the operation ------------------------------------------------------- */
+/*
+ * jvp_attn_fwd: O, dO and LSE of masked softmax attention and its JVP
+ * (Appendix B, Eq. 42-45 of the Causal-rCM report).
+ *
+ * q, k, v     primal inputs        [B, H, L, d], dtype `dtype`
+ * dq, dk, dv  tangents             [B, H, L, d], dtype `dtype`
+ * o, d_o      outputs              [B, H, L, d], dtype `dtype`; every row
+ *                                  with index < L is written
+ * lse         output               [B, H, L] float32, natural log of the sum
+ *                                  of exp(scaled scores) over admitted keys
+ * softmax_scale  > 0 uses the value given; <= 0 uses 1/sqrt(d). The same
+ *             scale multiplies the score and the score tangent.
+ *
+ * Supported: dtype JVP_BF16 with d = 128 runs the tcgen05/TMEM tensor-core
+ * kernel (bf16 operands, fp32 accumulation, bf16 outputs); JVP_FP32, and
+ * JVP_BF16 with d in {32, 64, 96}, run a CUDA-core kernel in fp32
+ * arithmetic. Other d give JVP_ERR_UNSUPPORTED_HEAD_DIM. B*H*L must stay
+ * below 2^31 rows.
+ *
+ * Workspace: the admissible tile list for (mask, L) is built on the host
+ * on first use, copied into a device buffer the library allocates, and
+ * cached per (device, mask, L) until jvp_attn_release(). That first call
+ * performs a blocking copy and must not be made during stream capture.
+ *
+ * A row whose admissible set is empty (no descriptor of the four modes
+ * yields one) gets O = dO = 0 and LSE = -inf.
+ */
+int jvp_attn_fwd(const void* q, const void* k, const void* v,
+                 const void* dq, const void* dk, const void* dv,
+                 void* o, void* d_o, float* lse,
+                 int B, int H, int L, int d, jvp_dtype dtype,
+                 jvp_mask_desc mask, float softmax_scale, void* stream);
+
+/* ---- host-side mask / schedule queries (no GPU needed) ------------------- */
+/*
+ * jvp_attn_mask_stats: for the mask on L tokens and a bm x bn tile grid
+ * anchored at (0, 0): *pairs = admitted (query, key) pairs per head;
+ * *full / *partial / *empty = number of tiles in which all / some / none of
+ * the (query < L, key) slots are admitted. Query rows at or past L are
+ * ignored (they are never written); a tile whose key range reaches past L
+ * is never full. Any output pointer may be NULL. Host only.
+ */
+int jvp_attn_mask_stats(jvp_mask_desc mask, int L, int bm, int bn,
+                        int64_t* pairs, int64_t* full, int64_t* partial,
+                        int64_t* empty);
+
+/*
+ * jvp_attn_tile_classes: writes the class (JVP_TILE_*) of every tile of the
+ * bm x bn grid to out[qt * n_kt + kt], n_qt = ceil(L/bm), n_kt = ceil(L/bn).
+ * out_len must be >= n_qt * n_kt, else JVP_ERR_INVALID_ARG. Host only.
+ */
+int jvp_attn_tile_classes(jvp_mask_desc mask, int L, int bm, int bn,
+                          int8_t* out, int64_t out_len);
+
+/*
+ * jvp_attn_schedule: the work list the tensor-core kernel runs, for tests
+ * and tools. Query tiles are bm rows; key tiles bn keys. Writes up to
+ * qtile_cap entries of 4 int32 {query tile, first segment, segment count,
+ * key tiles} to `qtiles`, longest first (ties: lower query tile first), and
+ * up to seg_cap segments of 3 int32 {first key tile, key-tile count,
+ * partial flag} to `segs`, each query tile's segments in increasing key
+ * order. *n_qtiles / *n_segs receive the full counts even if a cap is too
+ * small (then JVP_ERR_INVALID_ARG is returned). Host only.
+ */
+int jvp_attn_schedule(jvp_mask_desc mask, int L, int bm, int bn,
+                      int32_t* qtiles, int qtile_cap, int32_t* segs,
+                      int seg_cap, int* n_qtiles, int* n_segs);
+
+/* ---- device error word, workspace, misc ---------------------------------- */
+/*
+ * jvp_attn_check_device_error: synchronises `stream`, then reads and clears
+ * the current device's error word. Returns JVP_OK, JVP_ERR_DEVICE_TIMEOUT,
+ * JVP_ERR_DEVICE_BOUNDS, or JVP_ERR_LAUNCH_FAILED if the stream itself
+ * reports a CUDA error.
+ */
+int jvp_attn_check_device_error(void* stream);
+
+/* Frees every cached workspace on every device. Synchronises the device(s)
+ * first. Safe to call at any time outside stream capture. */
+int jvp_attn_release(void);
+
+/* Static string naming an error code (never NULL). */
+const char* jvp_attn_strerror(int code);
+
+/* JVP_ATTN_VERSION of the loaded library. */
+int jvp_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JVP_ATTN_H */

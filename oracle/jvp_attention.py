@@ -91,22 +91,27 @@ def jvp_attention_head(q, k, v, dq, dk, dv, spec: MaskSpec,
     for ivs, grp in _group_rows(spec, rows).items():
         if not ivs:
             continue
-        keys = np.concatenate([np.arange(a, b) for a, b in ivs])
-        K, V = k[keys], v[keys]
-        dK, dV = dk[keys], dv[keys]
+        # The admissible keys are the union of the intervals; each interval
+        # is a contiguous slice (a view), and sums over the union are sums
+        # of the per-interval sums.
+        Ks = [k[a:b] for a, b in ivs]
+        Vs = [v[a:b] for a, b in ivs]
+        dKs = [dk[a:b] for a, b in ivs]
+        dVs = [dv[a:b] for a, b in ivs]
         grp = np.asarray(grp)
         for s0 in range(0, len(grp), row_block):
             rr = grp[s0:s0 + row_block]
             Q, dQ = q[rr], dq[rr]
-            s = c * (Q @ K.T)                      # scores, Eq. 42
-            ds = c * (dQ @ K.T + Q @ dK.T)         # score tangent, Eq. 43
-            m = s.max(axis=1, keepdims=True)
-            e = np.exp(s - m)
-            ell = e.sum(axis=1, keepdims=True)
-            p = e / ell                            # masked softmax
-            out_o = p @ V
-            mu = (p * ds).sum(axis=1, keepdims=True)
-            out_do = (p * (ds - mu)) @ V + p @ dV  # Eq. 44
+            s = [c * (Q @ K.T) for K in Ks]                    # Eq. 42
+            ds = [c * (dQ @ K.T + Q @ dK.T) for K, dK in zip(Ks, dKs)]  # Eq. 43
+            m = np.max([x.max(axis=1) for x in s], axis=0)[:, None]
+            e = [np.exp(x - m) for x in s]
+            ell = sum(x.sum(axis=1, keepdims=True) for x in e)
+            p = [x / ell for x in e]                           # masked softmax
+            out_o = sum(pi @ V for pi, V in zip(p, Vs))
+            mu = sum((pi * dsi).sum(axis=1, keepdims=True) for pi, dsi in zip(p, ds))
+            out_do = sum((pi * (dsi - mu)) @ V + pi @ dV       # Eq. 44
+                         for pi, dsi, V, dV in zip(p, ds, Vs, dVs))
             idx = [pos[int(r)] for r in rr]
             o[idx] = out_o
             do[idx] = out_do
