@@ -108,6 +108,15 @@ class ClockSampler:
         self.proc = None
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
 
+    @staticmethod
+    def bus_id_of(props) -> str | None:
+        """'dddddddd:bb:dd.0' from torch device properties, if available."""
+        try:
+            return "%08x:%02x:%02x.0" % (int(props.pci_domain_id), int(props.pci_bus_id),
+                                         int(props.pci_device_id))
+        except (AttributeError, TypeError, ValueError):
+            return None
+
     def __enter__(self):
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
@@ -133,23 +142,36 @@ class ClockSampler:
     def summary(self):
         if self.proc is None or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        sm, mx, reasons = [], [], set()
-        with open(self.path) as f:
+        return self.parse(self.path, self.bus_id)
+
+    @classmethod
+    def parse(cls, path: str, bus_id: str = ""):
+        rows = {}
+        with open(path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
                 if len(parts) < 9:
                     continue
-                if self.bus_id and parts[0].lower()[-len(self.bus_id):] != self.bus_id[-12:] \
-                        and not parts[0].lower().endswith(self.bus_id[-12:]):
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    mx.append(float(parts[2]))
-                except ValueError:
-                    continue
-                for name, val in zip(self.NAMES, parts[5:9]):
-                    if val.lower().startswith("active"):
-                        reasons.add(name)
+                rows.setdefault(parts[0].lower(), []).append(parts)
+        key = None
+        for k in rows:
+            if bus_id and k[-7:] == bus_id[-7:]:
+                key = k
+        if key is None and len(rows) == 1:
+            key = next(iter(rows))
+        if key is None:
+            return {"sm_mhz": None, "sm_max_mhz": None,
+                    "reasons": ["could not match the GPU in nvidia-smi output"]}
+        sm, mx, reasons = [], [], set()
+        for parts in rows[key]:
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(cls.NAMES, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None,
                 "reasons": sorted(reasons), "samples": len(sm)}
@@ -201,7 +223,7 @@ def run_ours(args, w):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    bus = getattr(torch.cuda.get_device_properties(local), "pci_bus_id", None)
+    bus = ClockSampler.bus_id_of(torch.cuda.get_device_properties(local))
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     with ClockSampler(bus) as clk:
         ev[0].record(stream)
@@ -381,7 +403,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="tf",
                     choices=["tf", "frame_causal", "chunk_tf", "tf_long"])
-    ap.add_argument("--cpu-rows", type=int, default=256,
+    ap.add_argument("--cpu-rows", type=int, default=1536,
                     help="query rows per head in the cpu_baseline sample")
     ap.add_argument("--ref-rows", type=int, default=32,
                     help="query rows per head per step of --impl reference")
