@@ -32,7 +32,7 @@ JVP_FP32 = 1
 TILE_EMPTY, TILE_FULL, TILE_PARTIAL = 0, 1, 2
 
 # Exported functions, as declared in include/jvp_attn.h.
-EXPORTS = ("jvp_attn_fwd", "jvp_attn_mask_stats", "jvp_attn_tile_classes",
+EXPORTS = ("jvp_attn_fwd", "jvp_attn_fwd_noalloc", "jvp_attn_mask_stats", "jvp_attn_tile_classes",
            "jvp_attn_schedule", "jvp_attn_check_device_error",
            "jvp_attn_release", "jvp_attn_strerror", "jvp_attn_version")
 
@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.jvp_attn_fwd.argtypes = [vp] * 8 + [ctypes.POINTER(ctypes.c_float)] + \
             [i32] * 5 + [MaskDesc, ctypes.c_float, vp]
         L.jvp_attn_fwd.restype = i32
+        L.jvp_attn_fwd_noalloc.argtypes = L.jvp_attn_fwd.argtypes
+        L.jvp_attn_fwd_noalloc.restype = i32
         L.jvp_attn_mask_stats.argtypes = [MaskDesc, i32, i32, i32, i64p, i64p, i64p, i64p]
         L.jvp_attn_mask_stats.restype = i32
         L.jvp_attn_tile_classes.argtypes = [MaskDesc, i32, i32, i32,

@@ -38,4 +38,8 @@ int launch_simt(const LaunchArgs& a, bool bf16);
 // Tensor-core kernel: bf16, d = 128, sm_100a.
 int launch_sm100(const LaunchArgs& a, const WorkList& w, int num_sms);
 
+// Current device's SM count and error word; JVP_ERR_UNSUPPORTED_DEVICE
+// unless it is an sm_100 device. Allocates nothing.
+int current_device_state(int* sms, unsigned** err);
+
 }  // namespace jvp

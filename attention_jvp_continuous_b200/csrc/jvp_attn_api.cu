@@ -111,6 +111,17 @@ int get_worklist(int dev, const jvp_mask_desc& m, int L, WorkList* out) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
+
+int current_device_state(int* sms, unsigned** err) {
+  DevInfo* di = nullptr;
+  const int rc = device_info(&di);
+  if (rc != JVP_OK) return rc;
+  if (di->major != 10 || di->minor != 0) return JVP_ERR_UNSUPPORTED_DEVICE;
+  *sms = di->sms;
+  *err = di->err;
+  return JVP_OK;
+}
+
 }  // namespace jvp
 
 using namespace jvp;

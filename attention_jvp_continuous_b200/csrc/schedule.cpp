@@ -120,3 +120,76 @@ Schedule build_schedule(const jvp_mask_desc& m, int L, int bm, int bn) {
 }
 
 }  // namespace jvp
+
+namespace jvp {
+
+bool build_schedule_into(const jvp_mask_desc& m, int L, int bm, int bn, int32_t* qtiles,
+                         int64_t qtile_words, int32_t* segs, int64_t seg_words, int* n_qt,
+                         int* n_segs) {
+  const int nq = (L + bm - 1) / bm, nk = (L + bn - 1) / bn;
+  *n_qt = nq;
+  *n_segs = 0;
+  if (bm > 256 || int64_t(nq) * 4 > qtile_words) return false;
+  const int ch = chunk_of(m);
+  RowKeys cls[256];
+  int64_t ns = 0;
+  for (int qt = 0; qt < nq; ++qt) {
+    const int r0 = qt * bm, r1 = std::min(r0 + bm, L);
+    int ncls = 0;
+    for (int i = r0; i < r1; ++i) {
+      const RowKeys r = row_keys(m.mode, m.tokens_per_frame, m.n_frames, ch, L, i);
+      if (ncls == 0 || cls[ncls - 1].a0 != r.a0 || cls[ncls - 1].b0 != r.b0 ||
+          cls[ncls - 1].a1 != r.a1 || cls[ncls - 1].b1 != r.b1)
+        cls[ncls++] = r;
+    }
+    const int64_t seg_begin = ns;
+    int seg_count = 0, total = 0;
+    int run_start = -1, run_class = JVP_TILE_EMPTY;
+    for (int kt = 0; kt <= nk; ++kt) {
+      int c = JVP_TILE_EMPTY;
+      if (kt < nk) {
+        const int k0 = kt * bn, k1 = std::min(k0 + bn, L);
+        bool all = k0 + bn <= L, any = false;
+        for (int x = 0; x < ncls; ++x) {
+          const int ov = overlap(cls[x].a0, cls[x].b0, k0, k1) +
+                         overlap(cls[x].a1, cls[x].b1, k0, k1);
+          if (ov != k1 - k0) all = false;
+          if (ov > 0) any = true;
+        }
+        c = all ? JVP_TILE_FULL : (any ? JVP_TILE_PARTIAL : JVP_TILE_EMPTY);
+      }
+      if (c != run_class) {
+        if (run_class != JVP_TILE_EMPTY) {
+          if (2 * (ns + 1) > seg_words) {
+            *n_segs = int(ns);
+            return false;
+          }
+          const int cnt = kt - run_start;
+          segs[2 * ns] = run_start;
+          segs[2 * ns + 1] = (cnt << 1) | (run_class == JVP_TILE_PARTIAL ? 1 : 0);
+          ++ns;
+          ++seg_count;
+          total += cnt;
+        }
+        run_start = kt;
+        run_class = c;
+      }
+    }
+    qtiles[4 * qt] = qt;
+    qtiles[4 * qt + 1] = int32_t(seg_begin);
+    qtiles[4 * qt + 2] = seg_count;
+    qtiles[4 * qt + 3] = total;
+  }
+  *n_segs = int(ns);
+  // Longest first, ties by query tile: the order build_schedule produces.
+  struct E {
+    int32_t qt, sb, sc, nk;
+  };
+  E* e = reinterpret_cast<E*>(qtiles);
+  std::sort(e, e + nq, [](const E& a, const E& b) {
+    return a.nk != b.nk ? a.nk > b.nk : a.qt < b.qt;
+  });
+  return true;
+}
+
+}  // namespace jvp

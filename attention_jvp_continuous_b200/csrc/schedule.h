@@ -40,4 +40,14 @@ void classify_qtile(const jvp_mask_desc& m, int L, int bm, int bn, int qt,
 // Builds the full schedule. The mask must already be validated.
 Schedule build_schedule(const jvp_mask_desc& m, int L, int bm, int bn);
 
+// The same work list as build_schedule (same entries, same order), written
+// into caller-provided arrays without any heap allocation: entries of 4
+// int32 to `qtiles`, segments of 2 int32 ({kt_begin, (count << 1) |
+// partial}) to `segs`. Capacities are in int32 words. Returns false when a
+// capacity is exceeded (*n_qt / *n_segs then hold what was counted so far).
+// bm must be <= 256. The mask must already be validated.
+bool build_schedule_into(const jvp_mask_desc& m, int L, int bm, int bn, int32_t* qtiles,
+                         int64_t qtile_words, int32_t* segs, int64_t seg_words, int* n_qt,
+                         int* n_segs);
+
 }  // namespace jvp

@@ -122,6 +122,47 @@ int jvp_attn_fwd(const void* q, const void* k, const void* v,
                  int B, int H, int L, int d, jvp_dtype dtype,
                  jvp_mask_desc mask, float softmax_scale, void* stream);
 
+/*
+ * jvp_attn_fwd_noalloc: jvp_attn_fwd for callers that cannot allocate
+ * device memory. The paper has no counterpart: it is a deployment variant.
+ *
+ * jvp_attn_fwd allocates (cudaMalloc) a device buffer for the tile work list
+ * of every new (mask, L). Some callers cannot accept that: a framework whose
+ * device memory all belongs to its own pool or arena, or a deployment that
+ * forbids device allocation after start-up (where a cudaMalloc can also
+ * synchronise the device at a bad moment). This entry point keeps the
+ * work list in a fixed array of the library's own device memory (a
+ * file-scope __device__ array of 65,536 int32 = 256 KiB, held on every GPU
+ * that loads the library until the process exits) and never calls
+ * cudaMalloc, cudaFree or any allocating routine. The caller still passes
+ * the inputs and outputs.
+ *
+ * Arguments, layouts and results are those of jvp_attn_fwd, restricted to
+ * the tensor-core configuration: dtype must be JVP_BF16 (else
+ * JVP_ERR_INVALID_ARG) and d must be 128 (else
+ * JVP_ERR_UNSUPPORTED_HEAD_DIM). A mask whose work list needs more than
+ * 65,536 words (4 per 128-row query tile + 2 per key-tile run; about 81
+ * words per 1000 tokens for the teacher-forcing mask at 1560 tokens per
+ * frame, so roughly 800,000 tokens) returns JVP_ERR_TOO_LARGE before any
+ * device work.
+ *
+ * The first call on a device looks the array's address up
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture. A call whose (mask, L) differs from the list
+ * the array holds rewrites the array with an asynchronous copy on `stream`;
+ * every word the kernel reads is rewritten, so nothing has to start at
+ * zero. All calls on a device share the one array: calls with different
+ * (mask, L) whose work overlaps on the GPU (different streams, no ordering
+ * between them) race on it and give wrong results. Order such calls on one
+ * stream or synchronise between them.
+ */
+int jvp_attn_fwd_noalloc(const void* q, const void* k, const void* v,
+                         const void* dq, const void* dk, const void* dv,
+                         void* o, void* d_o, float* lse,
+                         int B, int H, int L, int d, jvp_dtype dtype,
+                         jvp_mask_desc mask, float softmax_scale,
+                         void* stream);
+
 /* ---- host-side mask / schedule queries (no GPU needed) ------------------- */
 /*
  * jvp_attn_mask_stats: for the mask on L tokens and a bm x bn tile grid
