@@ -20,7 +20,7 @@ CHUNK_CAUSAL = 2
 TEACHER_FORCING = 3
 
 __all__ = ["Mask", "jvp_attn", "jvp_attn_fwd", "mask_stats", "tile_classes",
-           "schedule", "check_device_error", "release", "JvpAttnError",
+           "schedule", "check_device_error", "set_wait_limit", "release", "JvpAttnError",
            "DENSE", "FRAME_CAUSAL", "CHUNK_CAUSAL", "TEACHER_FORCING"]
 
 
@@ -145,6 +145,11 @@ def check_device_error(stream: Optional[int] = None) -> None:
         stream = torch.cuda.current_stream().cuda_stream
     _lib.check(_lib.lib().jvp_attn_check_device_error(ctypes.c_void_p(stream)),
                "jvp_attn_check_device_error")
+
+
+def set_wait_limit(ns: int) -> None:
+    """Per-wait limit of the tensor-core kernel in ns (0 = default, 2 s)."""
+    _lib.check(_lib.lib().jvp_attn_set_wait_limit(int(ns)), "jvp_attn_set_wait_limit")
 
 
 def release() -> None:

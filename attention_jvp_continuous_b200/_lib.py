@@ -34,7 +34,8 @@ TILE_EMPTY, TILE_FULL, TILE_PARTIAL = 0, 1, 2
 # Exported functions, as declared in include/jvp_attn.h.
 EXPORTS = ("jvp_attn_fwd", "jvp_attn_fwd_noalloc", "jvp_attn_mask_stats", "jvp_attn_tile_classes",
            "jvp_attn_schedule", "jvp_attn_check_device_error",
-           "jvp_attn_release", "jvp_attn_strerror", "jvp_attn_version")
+           "jvp_attn_set_wait_limit", "jvp_attn_release", "jvp_attn_strerror",
+           "jvp_attn_version")
 
 
 class MaskDesc(ctypes.Structure):
@@ -84,6 +85,8 @@ def lib() -> ctypes.CDLL:
         L.jvp_attn_schedule.restype = i32
         L.jvp_attn_check_device_error.argtypes = [vp]
         L.jvp_attn_check_device_error.restype = i32
+        L.jvp_attn_set_wait_limit.argtypes = [ctypes.c_uint64]
+        L.jvp_attn_set_wait_limit.restype = i32
         L.jvp_attn_release.argtypes = []
         L.jvp_attn_release.restype = i32
         L.jvp_attn_strerror.argtypes = [i32]

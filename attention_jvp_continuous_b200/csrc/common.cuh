@@ -29,6 +29,10 @@ struct LaunchArgs {
   float scale;
   cudaStream_t stream;
   unsigned* err;  // device error word
+  // Work-item counter of the tensor-core kernel (one u32 of device memory
+  // owned by the caller of launch_sm100, which zeroes it on `stream` before
+  // the launch). Launches that share a counter must be stream-ordered.
+  unsigned* item_ctr = nullptr;
   unsigned long long wait_limit_ns;
 };
 
@@ -37,6 +41,9 @@ int launch_simt(const LaunchArgs& a, bool bf16);
 
 // Tensor-core kernel: bf16, d = 128, sm_100a.
 int launch_sm100(const LaunchArgs& a, const WorkList& w, int num_sms);
+
+// Per-wait limit for the tensor-core kernel (jvp_attn_set_wait_limit).
+unsigned long long wait_limit_ns();
 
 // Current device's SM count and error word; JVP_ERR_UNSUPPORTED_DEVICE
 // unless it is an sm_100 device. Allocates nothing.

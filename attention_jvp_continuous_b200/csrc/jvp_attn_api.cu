@@ -6,6 +6,7 @@
 // head dims). No exception crosses the boundary.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <map>
@@ -23,7 +24,8 @@ namespace jvp {
 namespace {
 
 constexpr int kBM = 128, kBN = 64;            // tensor-core tile shape
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;  // 2 s per wait
+std::atomic<unsigned long long> g_wait_limit{kDefaultWaitLimitNs};
 constexpr int kMaxDevices = 64;
 
 struct DevInfo {
@@ -48,6 +50,9 @@ struct Ws {
 std::mutex g_mu;
 DevInfo g_dev[kMaxDevices];
 std::map<WsKey, Ws> g_ws;
+// Work-item counter of the tensor-core kernel, one per (device, stream):
+// launches on one stream are ordered, so they can share it.
+std::map<std::pair<int, cudaStream_t>, unsigned*> g_ctr;
 
 int device_info(DevInfo** out) {
   int dev = 0;
@@ -108,9 +113,29 @@ int get_worklist(int dev, const jvp_mask_desc& m, int L, WorkList* out) {
   return JVP_OK;
 }
 
+int get_counter(int dev, cudaStream_t st, unsigned** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  const auto key = std::make_pair(dev, st);
+  auto it = g_ctr.find(key);
+  if (it != g_ctr.end()) {
+    *out = it->second;
+    return JVP_OK;
+  }
+  void* p = nullptr;
+  if (cudaMalloc(&p, 256) != cudaSuccess) {
+    cudaGetLastError();
+    return JVP_ERR_OUT_OF_MEMORY;
+  }
+  g_ctr[key] = static_cast<unsigned*>(p);
+  *out = static_cast<unsigned*>(p);
+  return JVP_OK;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
+
+unsigned long long wait_limit_ns() { return g_wait_limit.load(); }
 
 int current_device_state(int* sms, unsigned** err) {
   DevInfo* di = nullptr;
@@ -158,13 +183,15 @@ int jvp_attn_fwd(const void* q, const void* k, const void* v, const void* dq, co
   a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(d));
   a.stream = static_cast<cudaStream_t>(stream);
   a.err = di->err;
-  a.wait_limit_ns = kWaitLimitNs;
+  a.wait_limit_ns = wait_limit_ns();
   if (!tensor_core) return launch_simt(a, dtype == JVP_BF16);
 
   int dev = 0;
   cudaGetDevice(&dev);
   WorkList w;
   rc = get_worklist(dev, mask, L, &w);
+  if (rc != JVP_OK) return rc;
+  rc = get_counter(dev, a.stream, &a.item_ctr);
   if (rc != JVP_OK) return rc;
   return launch_sm100(a, w, di->sms);
 }
@@ -236,6 +263,11 @@ int jvp_attn_check_device_error(void* stream) {
   return JVP_OK;
 }
 
+int jvp_attn_set_wait_limit(uint64_t ns) {
+  g_wait_limit.store(ns == 0 ? kDefaultWaitLimitNs : (unsigned long long)ns);
+  return JVP_OK;
+}
+
 int jvp_attn_release(void) {
   std::lock_guard<std::mutex> lk(g_mu);
   int cur = 0;
@@ -247,6 +279,12 @@ int jvp_attn_release(void) {
       rc = JVP_ERR_LAUNCH_FAILED;
   }
   g_ws.clear();
+  for (auto& kv : g_ctr) {
+    if (cudaSetDevice(kv.first.first) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess ||
+        cudaFree(kv.second) != cudaSuccess)
+      rc = JVP_ERR_LAUNCH_FAILED;
+  }
+  g_ctr.clear();
   if (have_dev) cudaSetDevice(cur);
   return rc;
 }

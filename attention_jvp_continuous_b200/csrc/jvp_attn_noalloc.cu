@@ -23,23 +23,26 @@
 
 namespace {
 
-// Capacity of the work list, in int32 words: 4 per 128-row query tile plus
-// 2 per key-tile segment. The teacher-forcing mask at 1560 tokens per frame
-// needs about 81 words per 1000 tokens, so 65,536 words cover roughly
-// 800,000 tokens.
+// Size of the scratch array, in int32 words. The first kCounterWords hold
+// the kernel's work-item counter (zeroed on the stream before every launch);
+// the work list follows: 4 words per 128-row query tile plus 2 per key-tile
+// segment. The teacher-forcing mask at 1560 tokens per frame needs about 81
+// words per 1000 tokens, so the list fits up to roughly 800,000 tokens.
 constexpr int64_t kNoallocWords = 65536;
+constexpr int64_t kCounterWords = 64;  // keeps the list 256-byte aligned
+constexpr int64_t kListWords = kNoallocWords - kCounterWords;
 constexpr int kBM = 128, kBN = 64;
 constexpr int kMaxDevices = 64;
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 // Device scratch shared by every call on a device.
 static __device__ __align__(256) int32_t g_noalloc_worklist[kNoallocWords];
 // Host staging for the list before it is copied into g_noalloc_worklist.
-static int32_t g_noalloc_host[kNoallocWords];
+static int32_t g_noalloc_host[kListWords];
 
 struct NoallocDev {
   bool ready = false;
   int32_t* scratch = nullptr;  // device address of g_noalloc_worklist
+  int32_t* list = nullptr;     // scratch + kCounterWords
   bool have = false;           // key of the list the scratch currently holds
   int mode = 0, T = 0, F = 0, chunk = 0, L = 0;
   int n_qt = 0, n_segs = 0;
@@ -67,7 +70,7 @@ extern "C" int jvp_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   for (const void* p : ptrs)
     if (reinterpret_cast<uintptr_t>(p) & 15u) return JVP_ERR_MISALIGNED;
   // Query-tile entries alone must fit before the list is worth building.
-  if (4LL * ((L + kBM - 1) / kBM) > kNoallocWords) return JVP_ERR_TOO_LARGE;
+  if (4LL * ((L + kBM - 1) / kBM) > kListWords) return JVP_ERR_TOO_LARGE;
 
   int sms = 0;
   unsigned* err = nullptr;
@@ -79,6 +82,7 @@ extern "C" int jvp_attn_fwd_noalloc(const void* q, const void* k, const void* v,
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   WorkList w;
+  unsigned* counter = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_na_mu);
     NoallocDev& s = g_na[dev];
@@ -89,6 +93,7 @@ extern "C" int jvp_attn_fwd_noalloc(const void* q, const void* k, const void* v,
         return JVP_ERR_LAUNCH_FAILED;
       }
       s.scratch = static_cast<int32_t*>(p);
+      s.list = s.scratch + kCounterWords;
       s.ready = true;
     }
     const bool same = s.have && s.mode == mask.mode && s.T == mask.tokens_per_frame &&
@@ -98,13 +103,13 @@ extern "C" int jvp_attn_fwd_noalloc(const void* q, const void* k, const void* v,
       int nq = 0, ns = 0;
       const int64_t seg_off = 4LL * n_qt;
       if (!build_schedule_into(mask, L, kBM, kBN, g_noalloc_host, seg_off,
-                               g_noalloc_host + seg_off, kNoallocWords - seg_off, &nq, &ns))
+                               g_noalloc_host + seg_off, kListWords - seg_off, &nq, &ns))
         return JVP_ERR_TOO_LARGE;
       // The scratch is rewritten in stream order; it no longer holds the
       // previous list even if this call fails later.
       s.have = false;
       const size_t bytes = size_t(seg_off + 2LL * ns) * sizeof(int32_t);
-      if (cudaMemcpyAsync(s.scratch, g_noalloc_host, bytes, cudaMemcpyHostToDevice, st) !=
+      if (cudaMemcpyAsync(s.list, g_noalloc_host, bytes, cudaMemcpyHostToDevice, st) !=
           cudaSuccess)
         return JVP_ERR_LAUNCH_FAILED;
       s.have = true;
@@ -116,8 +121,9 @@ extern "C" int jvp_attn_fwd_noalloc(const void* q, const void* k, const void* v,
       s.n_qt = nq;
       s.n_segs = ns;
     }
-    w.qtiles = reinterpret_cast<const int4*>(s.scratch);
-    w.segs = reinterpret_cast<const int2*>(s.scratch + 4LL * s.n_qt);
+    w.qtiles = reinterpret_cast<const int4*>(s.list);
+    w.segs = reinterpret_cast<const int2*>(s.list + 4LL * s.n_qt);
+    counter = reinterpret_cast<unsigned*>(s.scratch);
     w.n_qtiles = s.n_qt;
     w.n_segs = s.n_segs;
   }
@@ -130,6 +136,7 @@ extern "C" int jvp_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(d));
   a.stream = st;
   a.err = err;
-  a.wait_limit_ns = kWaitLimitNs;
+  a.item_ctr = counter;
+  a.wait_limit_ns = wait_limit_ns();
   return launch_sm100(a, w, sms);
 }

@@ -15,10 +15,15 @@
 // when a row's new maximum exceeds it by more than 2^8, which is exact
 // because the finish uses ratios only.
 //
-// Warp roles (256 threads, one CTA per SM, persistent over the work list):
-//   warp 0      TMA producer: Q/dQ per query tile, K/dK and V/dV rings of 2
-//   warp 1      TMEM owner and MMA issuer (one thread)
-//   warps 4..7  softmax/JVP state, P write-back to TMEM, epilogue
+// Warp roles (384 threads, one CTA per SM, persistent over the work list):
+//   warp 0       TMA producer: Q/dQ per query tile, K|dK and V|dV rings of 2
+//   warp 1       TMEM owner and MMA issuer (one thread)
+//   warps 4..11  softmax/JVP state, P write-back to TMEM, epilogue: two
+//                warpgroups, each taking 32 of a tile's 64 key columns of
+//                every row (one row per thread), exchanging row maxima
+// MMAs per 64-key tile: [S | Q dK^T] = Q [K ; dK]^T (N = 128), then
+// dS += dQ K^T (N = 64), then [A1 | A23] += P [V | dV] (N = 256, P from
+// TMEM), then A23 += (scale e dS) V (N = 128).
 // TMEM (512 columns): S/dS double buffer at [0,256): buffer b holds S in
 // columns [128b, 128b+64) and dS in [128b+64, 128b+128); the bf16 operands
 // e and scale*e*dS overwrite the first 32 columns of S and dS of their
@@ -48,7 +53,7 @@ using namespace jvp::ptx;
 constexpr int BM = 128;  // query rows per tile = TMEM lanes
 constexpr int BN = 64;   // keys per tile
 constexpr int D = 128;   // head dim
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr float kTau = 8.0f;  // lazy rescale threshold, log2 units
 
 // Shared memory map (byte offsets from a 1024-aligned base). Every operand
@@ -62,7 +67,7 @@ constexpr uint32_t SM_K = 4 * kQHalf;          // K/dK ring: stage s at +32 KB*s
 constexpr uint32_t SM_V = SM_K + 2 * 4 * kKHalf;  // V/dV ring
 constexpr uint32_t kStageBytes = 4 * kKHalf;      // 32 KB: K|dK or V|dV
 constexpr uint32_t SM_BAR = SM_V + 2 * kStageBytes;  // 196608
-constexpr uint32_t kSmemBytes = SM_BAR + 256 + 1024;  // + barriers + align slack
+constexpr uint32_t kSmemBytes = SM_BAR + 512 + 4096 + 1024;  // + barriers, exchange, slack
 
 // Barrier slots (8 bytes each) inside SM_BAR.
 enum : uint32_t {
@@ -77,17 +82,26 @@ enum : uint32_t {
   B_PVDONE = 14,
   B_AFREE = 15,
   B_DRAIN = 16,
-  kNumBars = 17
+  B_XMAX = 17,    // 8 slots: [lane quarter][tile parity], softmax halves' max exchange
+  B_XSUM = 25,    // 4 slots: [lane quarter], end-of-item l/g exchange
+  B_IFULL = 29,   // 4 slots: work-item ring, published
+  B_IEMPTY = 33,  // 4 slots: work-item ring, released
+  kNumBars = 37
 };
 constexpr uint32_t SM_TMEM_SLOT = SM_BAR + 8 * kNumBars;  // u32: TMEM base
 constexpr uint32_t SM_ABORT = SM_TMEM_SLOT + 4;           // u32: abort flag
+constexpr uint32_t SM_RING = SM_ABORT + 4;                // 4 x i32: work-item ring
+constexpr uint32_t SM_XCHG = SM_BAR + 512;                // 4 KB: softmax exchange
+static_assert(SM_RING + 16 <= SM_XCHG, "barrier area overflow");
 
 // TMEM columns.
 constexpr uint32_t TM_A1 = 256;
 constexpr uint32_t TM_A23 = 384;
 
-constexpr uint32_t IDESC_S = ptx::idesc_bf16(BM, BN, false, false);
-constexpr uint32_t IDESC_PV = ptx::idesc_bf16(BM, D, false, true);
+constexpr uint32_t IDESC_S = ptx::idesc_bf16(BM, BN, false, false);       // 128 x 64
+constexpr uint32_t IDESC_SK = ptx::idesc_bf16(BM, 2 * BN, false, false);  // 128 x 128
+constexpr uint32_t IDESC_PV = ptx::idesc_bf16(BM, D, false, true);        // 128 x 128
+constexpr uint32_t IDESC_PVV = ptx::idesc_bf16(BM, 2 * D, false, true);   // 128 x 256
 
 struct Params {
   const int4* qtiles;  // {qt, seg_begin, seg_count, n_ktiles}
@@ -100,63 +114,8 @@ struct Params {
   __nv_bfloat16* d_o;
   float* lse;
   unsigned* err;
+  unsigned* item_ctr;  // zero at launch; CTAs take work items from it in list order
   unsigned long long wait_limit_ns;
-};
-
-// Walks this CTA's (item, key tile) sequence; every role runs its own copy.
-struct Cursor {
-  int item, item_idx, bh, qt;
-  int seg, seg_end, kt, kt_end;
-  int j, n;
-  uint32_t t;  // ordinal of the tile among this CTA's tiles
-  bool partial, valid;
-
-  __device__ void load_seg(const Params& p) {
-    const int2 s = p.segs[seg];
-    kt = s.x;
-    kt_end = s.x + (s.y >> 1);
-    partial = (s.y & 1) != 0;
-    if (kt < 0 || kt_end > p.n_kt || kt_end <= kt) {
-      atomicOr(p.err, kErrBounds);
-      valid = false;
-    }
-  }
-  __device__ void load_item(const Params& p) {
-    valid = item < p.n_items;
-    if (!valid) return;
-    const int e = item % p.n_entries;
-    bh = item / p.n_entries;
-    const int4 en = p.qtiles[e];
-    qt = en.x;
-    seg = en.y;
-    seg_end = en.y + en.z;
-    n = en.w;
-    j = 0;
-    if (qt < 0 || qt >= p.n_qt || seg < 0 || seg_end > p.n_segs || en.z < 1 || n < 1) {
-      atomicOr(p.err, kErrBounds);
-      valid = false;
-      return;
-    }
-    load_seg(p);
-  }
-  __device__ void start(const Params& p) {
-    item = blockIdx.x;
-    item_idx = 0;
-    t = 0;
-    load_item(p);
-  }
-  __device__ void next(const Params& p) {
-    ++t;
-    ++j;
-    if (++kt < kt_end) return;
-    if (++seg < seg_end) {
-      load_seg(p);
-      return;
-    }
-    item += gridDim.x;
-    ++item_idx;
-    load_item(p);
-  }
 };
 
 // Bounded wait. Returns false (and raises the CTA abort flag) on timeout or
@@ -177,6 +136,97 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Pa
     }
   }
 }
+
+// Work items reach the roles through a 4-slot ring in shared memory: the
+// producer takes the next item index from the global counter (dynamic
+// longest-first scheduling) and publishes it; the MMA thread's two cursors
+// and the eight softmax warps read it and release the slot.
+enum Role { kProducer, kConsumerThread, kConsumerWarp };
+constexpr uint32_t kRing = 4;
+constexpr uint32_t kRingReaders = 2 + 8;  // MMA S and PV cursors, softmax warps
+
+struct ItemRing {
+  uint32_t full_bar, empty_bar;  // first slot's mbarrier; slots are 8 B apart
+  volatile int* slots;
+  volatile uint32_t* abort_flag;
+};
+
+// Walks this CTA's (item, key tile) sequence; every role runs its own copy.
+struct Cursor {
+  int item, item_idx, bh, qt;
+  int seg, seg_end, kt, kt_end;
+  int j, n;
+  uint32_t t;  // ordinal of the tile among this CTA's tiles
+  bool partial, valid;
+
+  __device__ void load_seg(const Params& p) {
+    const int2 s = p.segs[seg];
+    kt = s.x;
+    kt_end = s.x + (s.y >> 1);
+    partial = (s.y & 1) != 0;
+    if (kt < 0 || kt_end > p.n_kt || kt_end <= kt) {
+      atomicOr(p.err, kErrBounds);
+      valid = false;
+    }
+  }
+  // Index of this CTA's item number item_idx; false on timeout / abort.
+  __device__ bool acquire(const Params& p, const ItemRing& r, Role role) {
+    const uint32_t slot = uint32_t(item_idx) % kRing, use = uint32_t(item_idx) / kRing;
+    if (role == kProducer) {
+      if (use > 0 && !wait_bar(r.empty_bar + 8 * slot, (use - 1) & 1u, p, r.abort_flag))
+        return false;
+      item = int(atomicAdd(p.item_ctr, 1u));
+      r.slots[slot] = item;
+      mbar_arrive(r.full_bar + 8 * slot);  // release: readers see the slot
+      return true;
+    }
+    bool ok = wait_bar(r.full_bar + 8 * slot, use & 1u, p, r.abort_flag);
+    if (role == kConsumerWarp) ok = __all_sync(0xffffffffu, ok);
+    if (!ok) return false;
+    item = r.slots[slot];
+    if (role == kConsumerWarp) {
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(r.empty_bar + 8 * slot);
+    } else {
+      mbar_arrive(r.empty_bar + 8 * slot);
+    }
+    return true;
+  }
+  __device__ void load_item(const Params& p, const ItemRing& r, Role role) {
+    valid = acquire(p, r, role) && item < p.n_items;
+    if (!valid) return;
+    const int e = item % p.n_entries;
+    bh = item / p.n_entries;
+    const int4 en = p.qtiles[e];
+    qt = en.x;
+    seg = en.y;
+    seg_end = en.y + en.z;
+    n = en.w;
+    j = 0;
+    if (qt < 0 || qt >= p.n_qt || seg < 0 || seg_end > p.n_segs || en.z < 1 || n < 1) {
+      atomicOr(p.err, kErrBounds);
+      valid = false;
+      return;
+    }
+    load_seg(p);
+  }
+  __device__ void start(const Params& p, const ItemRing& r, Role role) {
+    item_idx = 0;
+    t = 0;
+    load_item(p, r, role);
+  }
+  __device__ void next(const Params& p, const ItemRing& r, Role role) {
+    ++t;
+    ++j;
+    if (++kt < kt_end) return;
+    if (++seg < seg_end) {
+      load_seg(p);
+      return;
+    }
+    ++item_idx;
+    load_item(p, r, role);
+  }
+};
 
 // Short bounded wait used only while cleaning up after an abort.
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
@@ -214,11 +264,17 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar(B_VFULL + s), 1);
       mbar_init(bar(B_VEMPTY + s), 1);
       mbar_init(bar(B_SFULL + s), 1);
-      mbar_init(bar(B_PFULL + s), BM);
+      mbar_init(bar(B_PFULL + s), 2 * BM);
     }
     mbar_init(bar(B_PVDONE), 1);
-    mbar_init(bar(B_AFREE), BM);
+    mbar_init(bar(B_AFREE), 2 * BM);
     mbar_init(bar(B_DRAIN), 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bar(B_XMAX + i), 64);
+    for (int i = 0; i < 4; ++i) mbar_init(bar(B_XSUM + i), 64);
+    for (int i = 0; i < int(kRing); ++i) {
+      mbar_init(bar(B_IFULL + i), 1);
+      mbar_init(bar(B_IEMPTY + i), kRingReaders);
+    }
     *abort_flag = 0u;
     fence_mbar_init();
   }
@@ -238,14 +294,17 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base_ptr + SM_TMEM_SLOT);
+  const ItemRing ring{bar(B_IFULL), bar(B_IEMPTY),
+                      reinterpret_cast<volatile int*>(base_ptr + SM_RING), abort_flag};
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA ----
     if (lane == 0) {
       Cursor c;
-      c.start(p);
-      // Parity of the latest arming of each full barrier, for abort cleanup.
-      int q_armed = 0, k_armed[2] = {0, 0}, v_armed[2] = {0, 0};
+      c.start(p, ring, kProducer);
+      // How many times each full barrier was armed, for abort cleanup.
+      // Stage s of a ring is armed by tiles t with t % 2 == s.
+      uint32_t q_armed = 0, k_issued = 0, v_issued = 0;
       bool ok = true;
       while (c.valid && ok) {
         if (c.j == 0) {
@@ -265,29 +324,32 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (c.t >= 2) ok = wait_bar(bar(B_KEMPTY + s), (u - 1) & 1u, p, abort_flag);
         if (!ok) break;
         mbar_expect_tx(bar(B_KFULL + s), kStageBytes);
-        ++k_armed[s];
+        ++k_issued;
+        // [K h0][dK h0][K h1][dK h1]: rows of K then dK are one 128-row
+        // operand per head-dim half.
         const uint32_t ks = base + SM_K + s * kStageBytes;
         tma_load_3d(ks, &tm_k, bar(B_KFULL + s), 0, y, c.bh);
-        tma_load_3d(ks + kKHalf, &tm_k, bar(B_KFULL + s), 64, y, c.bh);
-        tma_load_3d(ks + 2 * kKHalf, &tm_dk, bar(B_KFULL + s), 0, y, c.bh);
+        tma_load_3d(ks + kKHalf, &tm_dk, bar(B_KFULL + s), 0, y, c.bh);
+        tma_load_3d(ks + 2 * kKHalf, &tm_k, bar(B_KFULL + s), 64, y, c.bh);
         tma_load_3d(ks + 3 * kKHalf, &tm_dk, bar(B_KFULL + s), 64, y, c.bh);
         if (c.t >= 2) ok = wait_bar(bar(B_VEMPTY + s), (u - 1) & 1u, p, abort_flag);
         if (!ok) break;
         mbar_expect_tx(bar(B_VFULL + s), kStageBytes);
-        ++v_armed[s];
+        ++v_issued;
         const uint32_t vs = base + SM_V + s * kStageBytes;
         tma_load_3d(vs, &tm_v, bar(B_VFULL + s), 0, y, c.bh);
         tma_load_3d(vs + kKHalf, &tm_v, bar(B_VFULL + s), 64, y, c.bh);
         tma_load_3d(vs + 2 * kKHalf, &tm_dv, bar(B_VFULL + s), 0, y, c.bh);
         tma_load_3d(vs + 3 * kKHalf, &tm_dv, bar(B_VFULL + s), 64, y, c.bh);
-        c.next(p);
+        c.next(p, ring, kProducer);
       }
-      if (!ok) {
+      if (!ok || *abort_flag) {
         // Let copies already issued land before the CTA's smem is released.
-        if (q_armed) drain_wait(bar(B_QFULL), (q_armed - 1) & 1);
-        for (int s = 0; s < 2; ++s) {
-          if (k_armed[s]) drain_wait(bar(B_KFULL + s), (k_armed[s] - 1) & 1);
-          if (v_armed[s]) drain_wait(bar(B_VFULL + s), (v_armed[s] - 1) & 1);
+        if (q_armed) drain_wait(bar(B_QFULL), (q_armed - 1) & 1u);
+        for (uint32_t s = 0; s < 2; ++s) {
+          const uint32_t nk = (k_issued + 1 - s) / 2, nv = (v_issued + 1 - s) / 2;
+          if (nk) drain_wait(bar(B_KFULL + s), (nk - 1) & 1u);
+          if (nv) drain_wait(bar(B_VFULL + s), (nv - 1) & 1u);
         }
       }
     }
@@ -303,26 +365,21 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         tc_fence_after();
         const uint32_t d_s = tmem + b * 128u, d_ds = d_s + 64u;
         const uint32_t kb = base + SM_K + b * kStageBytes;
+        // [S | Q dK^T] = Q [K ; dK]^T: one N=128 MMA per 16-wide k-step.
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t oq = (kk >> 2) * kQHalf + (kk & 3) * 32;
-          const uint32_t ok_ = (kk >> 2) * kKHalf + (kk & 3) * 32;
+          const uint32_t ob = (kk >> 2) * (2 * kKHalf) + (kk & 3) * 32;
           mma_ss(d_s, sdesc_sw128(base + SM_Q + oq, 16, 1024),
-                 sdesc_sw128(kb + ok_, 16, 1024), IDESC_S, kk > 0);
+                 sdesc_sw128(kb + ob, 16, 1024), IDESC_SK, kk > 0);
         }
+        // dS = Q dK^T + dQ K^T: N=64 MMAs accumulate dQ K^T onto it.
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t oq = (kk >> 2) * kQHalf + (kk & 3) * 32;
-          const uint32_t ok_ = (kk >> 2) * kKHalf + (kk & 3) * 32;
+          const uint32_t ob = (kk >> 2) * (2 * kKHalf) + (kk & 3) * 32;
           mma_ss(d_ds, sdesc_sw128(base + SM_DQ + oq, 16, 1024),
-                 sdesc_sw128(kb + ok_, 16, 1024), IDESC_S, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t oq = (kk >> 2) * kQHalf + (kk & 3) * 32;
-          const uint32_t ok_ = (kk >> 2) * kKHalf + (kk & 3) * 32;
-          mma_ss(d_ds, sdesc_sw128(base + SM_Q + oq, 16, 1024),
-                 sdesc_sw128(kb + 2 * kKHalf + ok_, 16, 1024), IDESC_S, 1u);
+                 sdesc_sw128(kb + ob, 16, 1024), IDESC_S, 1u);
         }
         mma_commit(bar(B_KEMPTY + b));
         mma_commit(bar(B_SFULL + b));
@@ -340,38 +397,37 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t vb = base + SM_V + b * kStageBytes;
         const uint32_t a_p = tmem + b * 128u, a_pd = a_p + 64u;
         const uint32_t first = c.j == 0 ? 0u : 1u;
+        // [A1 | A23] += P [V | dV]: one N=256 MMA per 16-key step (A1 and A23
+        // are adjacent in TMEM; V h0, V h1, dV h0, dV h1 are 8 KB apart).
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
           mma_ts(tmem + TM_A1, a_p + ks * 8, sdesc_sw128(vb + ks * 2048, kKHalf, 1024),
-                 IDESC_PV, first | (ks > 0));
+                 IDESC_PVV, first | (ks > 0));
+        // A23 += (scale e dS) V
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
           mma_ts(tmem + TM_A23, a_pd + ks * 8, sdesc_sw128(vb + ks * 2048, kKHalf, 1024),
-                 IDESC_PV, first | (ks > 0));
-#pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts(tmem + TM_A23, a_p + ks * 8,
-                 sdesc_sw128(vb + 2 * kKHalf + ks * 2048, kKHalf, 1024), IDESC_PV, 1u);
+                 IDESC_PV, 1u);
         mma_commit(bar(B_VEMPTY + b));
         mma_commit(bar(B_PVDONE));
         return true;
       };
       Cursor cs, cp;
-      cs.start(p);
-      cp.start(p);
+      cs.start(p, ring, kConsumerThread);
+      cp.start(p, ring, kConsumerThread);
       for (int pre = 0; pre < 2 && cs.valid && ok; ++pre) {
         ok = issue_s(cs);
-        cs.next(p);
+        cs.next(p, ring, kConsumerThread);
       }
       while (cp.valid && ok) {
         ok = issue_pv(cp);
-        cp.next(p);
+        cp.next(p, ring, kConsumerThread);
         if (ok && cs.valid) {
           ok = issue_s(cs);
-          cs.next(p);
+          cs.next(p, ring, kConsumerThread);
         }
       }
-      if (!ok) {
+      if (!ok || *abort_flag) {
         // Wait for every MMA this thread issued before TMEM is freed.
         mma_commit(bar(B_DRAIN));
         drain_wait(bar(B_DRAIN), 0);
@@ -380,11 +436,20 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncwarp();
   } else if (warp >= 4) {
     // ----------------------------------------------------- softmax / JVP ----
-    const int r = threadIdx.x - 128;                 // row within the tile
-    const uint32_t tl = tmem + (uint32_t(r & ~31) << 16);  // this warp's lane quarter
+    // Two warpgroups share each row: warps 4-7 take columns [0, 32) of every
+    // 64-key tile, warps 8-11 columns [32, 64). Warps 4+q and 8+q read the
+    // same TMEM lane quarter q (rows 32q .. 32q+31) and exchange their
+    // partial row maxima through shared memory every tile, so both halves
+    // apply one running max. Their partial l and g are summed at the end.
+    const int hw = (warp - 4) >> 2;                  // column half
+    const int q4 = warp & 3;                         // TMEM lane quarter
+    const int r = q4 * 32 + lane;                    // row within the tile
+    const uint32_t tl = tmem + (uint32_t(q4 * 32) << 16);
     const int chunk = p.mask.chunk < 1 ? 1 : p.mask.chunk;
+    float* const xmax = reinterpret_cast<float*>(base_ptr + SM_XCHG);   // [2][2][128]
+    float* const xsum = xmax + 4 * BM;                                  // [2 (l,g)][2][128]
     Cursor c;
-    c.start(p);
+    c.start(p, ring, kConsumerWarp);
     float m_ref = -CUDART_INF_F, l = 0.f, g = 0.f;
     RowKeys rk{0, 0, 0, 0};
     int grow = 0;
@@ -401,28 +466,40 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       ok = wait_bar(bar(B_SFULL + b), (c.t >> 1) & 1u, p, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      uint32_t sr0[32], sr1[32], dr0[32], dr1[32];
-      tmem_ld32(tl + b * 128u, sr0);
-      tmem_ld32(tl + b * 128u + 32u, sr1);
-      tmem_ld32(tl + b * 128u + 64u, dr0);
-      tmem_ld32(tl + b * 128u + 96u, dr1);
+      uint32_t sr[32], dr[32];
+      tmem_ld32(tl + b * 128u + 32u * hw, sr);
+      tmem_ld32(tl + b * 128u + 64u + 32u * hw, dr);
       tmem_wait_ld();
-      float s[64];
+      float s[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        s[i] = __uint_as_float(sr0[i]);
-        s[32 + i] = __uint_as_float(sr1[i]);
-      }
+      for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(sr[i]);
       if (c.partial) {
-        const int k0 = c.kt * BN;
+        const int k0 = c.kt * BN + 32 * hw;
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
+        for (int i = 0; i < 32; ++i)
           if (!key_ok(rk, k0 + i)) s[i] = -CUDART_INF_F;
       }
-      float mx = s[0];
+      // Partial row max as 8 independent chains, then the partner's half.
+      float m8[8];
 #pragma unroll
-      for (int i = 1; i < 64; ++i) mx = fmaxf(mx, s[i]);
-      const float mxs = mx * p.c2;
+      for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+      for (int i = 8; i < 32; ++i) m8[i & 7] = fmaxf(m8[i & 7], s[i]);
+#pragma unroll
+      for (int w2 = 4; w2 > 0; w2 >>= 1)
+#pragma unroll
+        for (int i = 0; i < w2; ++i) m8[i] = fmaxf(m8[i], m8[i + w2]);
+      const uint32_t xp = b * 2u;  // exchange slot parity = tile parity
+      xmax[(xp + hw) * BM + r] = m8[0];
+      // The exchange also orders TMEM: the partner overwrites half of the S
+      // and dS columns this warp has just read (its P operands), so both
+      // sides fence around it.
+      tc_fence_before();
+      mbar_arrive(bar(B_XMAX + q4 * 2 + b));
+      ok = wait_bar(bar(B_XMAX + q4 * 2 + b), (c.t >> 1) & 1u, p, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const float mxs = fmaxf(m8[0], xmax[(xp + (hw ^ 1)) * BM + r]) * p.c2;
       float alpha = 1.f;
       bool need = false;
       if (m_ref == -CUDART_INF_F) {
@@ -432,16 +509,18 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         m_ref = mxs;
         need = true;
       }
+      // Warps 4+q and 8+q hold the same rows and take the same decision.
       if (__any_sync(0xffffffffu, need)) {
         l *= alpha;
         g *= alpha;
-        // A1/A23 hold PV(t-1); wait for it, then scale this warp's rows.
+        // A1/A23 hold PV(t-1); wait for it, then scale this quarter's rows:
+        // the first warpgroup scales A1, the second A23.
         ok = wait_bar(bar(B_PVDONE), (c.t - 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
 #pragma unroll 1
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const uint32_t col = (q4 < 4 ? TM_A1 : TM_A23) + (q4 & 3) * 32u;
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t col = (hw == 0 ? TM_A1 : TM_A23) + q * 32u;
           uint32_t a[32];
           tmem_ld32(tl + col, a);
           tmem_wait_ld();
@@ -452,21 +531,24 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         tmem_wait_st();
       }
       const float mref_use = m_ref == -CUDART_INF_F ? 0.f : m_ref;
-      uint32_t pp[32], pd[32];
+      uint32_t pp[16], pd[16];
+      float l4[4] = {0.f, 0.f, 0.f, 0.f}, g4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float ds0 = __uint_as_float(i < 16 ? dr0[2 * i] : dr1[2 * i - 32]);
-        const float ds1 = __uint_as_float(i < 16 ? dr0[2 * i + 1] : dr1[2 * i - 31]);
+      for (int i = 0; i < 16; ++i) {
         const float e0 = ex2(fmaf(s[2 * i], p.c2, -mref_use));
         const float e1 = ex2(fmaf(s[2 * i + 1], p.c2, -mref_use));
-        const float ed0 = e0 * ds0, ed1 = e1 * ds1;
-        l += e0 + e1;
-        g += ed0 + ed1;
+        const float ed0 = e0 * __uint_as_float(dr[2 * i]);
+        const float ed1 = e1 * __uint_as_float(dr[2 * i + 1]);
+        l4[i & 3] += e0 + e1;
+        g4[i & 3] += ed0 + ed1;
         pp[i] = pack_bf16(e0, e1);
         pd[i] = pack_bf16(ed0 * p.scale, ed1 * p.scale);
       }
-      tmem_st32(tl + b * 128u, pp);
-      tmem_st32(tl + b * 128u + 64u, pd);
+      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      g += (g4[0] + g4[1]) + (g4[2] + g4[3]);
+      // bf16 e into S columns [16 hw, 16 hw + 16), scale*e*dS into the dS ones.
+      tmem_st16(tl + b * 128u + 16u * hw, pp);
+      tmem_st16(tl + b * 128u + 64u + 16u * hw, pd);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_PFULL + b));
@@ -479,16 +561,26 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         ok = c.t == 0 || wait_bar(bar(B_PVDONE), (c.t - 1) & 1u, p, abort_flag);
         ok = ok && wait_bar(bar(B_PVDONE), c.t & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
+        // Row totals of l and g from both halves.
+        xsum[hw * BM + r] = l;
+        xsum[(2 + hw) * BM + r] = g;
+        mbar_arrive(bar(B_XSUM + q4));
+        ok = wait_bar(bar(B_XSUM + q4), c.item_idx & 1, p, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        const float lt = l + xsum[(hw ^ 1) * BM + r];
+        const float gt = g + xsum[(2 + (hw ^ 1)) * BM + r];
         tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        const float mu = p.scale * g * inv;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const float mu = p.scale * gt * inv;
         const bool row_ok = grow < p.L;
         const size_t off = (size_t(c.bh) * p.L + (row_ok ? grow : 0)) * D;
+        // This warpgroup writes head-dim columns [64 hw, 64 hw + 64).
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < 2; ++cc) {
+          const uint32_t col = 64u * hw + 32u * cc;
           uint32_t a1[32], a23[32];
-          tmem_ld32(tl + TM_A1 + cc * 32u, a1);
-          tmem_ld32(tl + TM_A23 + cc * 32u, a23);
+          tmem_ld32(tl + TM_A1 + col, a1);
+          tmem_ld32(tl + TM_A23 + col, a23);
           tmem_wait_ld();
           uint32_t po[16], pdo[16];
 #pragma unroll
@@ -501,8 +593,8 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             pdo[i] = pack_bf16(d0, d1);
           }
           if (row_ok) {
-            uint4* go = reinterpret_cast<uint4*>(p.o + off + cc * 32);
-            uint4* gd = reinterpret_cast<uint4*>(p.d_o + off + cc * 32);
+            uint4* go = reinterpret_cast<uint4*>(p.o + off + col);
+            uint4* gd = reinterpret_cast<uint4*>(p.d_o + off + col);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               go[i] = make_uint4(po[4 * i], po[4 * i + 1], po[4 * i + 2], po[4 * i + 3]);
@@ -512,11 +604,11 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         tc_fence_before();
         mbar_arrive(bar(B_AFREE));
-        if (row_ok)
+        if (row_ok && hw == 0)
           p.lse[size_t(c.bh) * p.L + grow] =
-              l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+              lt > 0.f ? (m_ref + log2f(lt)) * 0.69314718055994531f : -CUDART_INF_F;
       }
-      c.next(p);
+      c.next(p, ring, kConsumerWarp);
     }
   }
 
@@ -586,6 +678,7 @@ int launch_sm100(const LaunchArgs& a, const WorkList& w, int num_sms) {
   p.d_o = static_cast<__nv_bfloat16*>(a.d_o);
   p.lse = a.lse;
   p.err = a.err;
+  p.item_ctr = a.item_ctr;
   p.wait_limit_ns = a.wait_limit_ns;
   // The dynamic shared-memory opt-in is a per-device function attribute.
   static std::mutex attr_mu;
@@ -602,6 +695,8 @@ int launch_sm100(const LaunchArgs& a, const WorkList& w, int num_sms) {
     }
   }
   const int grid = int(items < num_sms ? items : num_sms);
+  if (!a.item_ctr || cudaMemsetAsync(a.item_ctr, 0, sizeof(unsigned), a.stream) != cudaSuccess)
+    return JVP_ERR_LAUNCH_FAILED;
   jvp_attn_sm100_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mdq, mk, mdk, mv, mdv, p);
   return cudaGetLastError() == cudaSuccess ? JVP_OK : JVP_ERR_LAUNCH_FAILED;
 }

@@ -403,7 +403,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="tf",
                     choices=["tf", "frame_causal", "chunk_tf", "tf_long"])
-    ap.add_argument("--cpu-rows", type=int, default=1536,
+    ap.add_argument("--cpu-rows", type=int, default=3072,
                     help="query rows per head in the cpu_baseline sample")
     ap.add_argument("--ref-rows", type=int, default=32,
                     help="query rows per head per step of --impl reference")

@@ -111,7 +111,10 @@ typedef enum { JVP_BF16 = 0, JVP_FP32 = 1 } jvp_dtype;
  * Workspace: the admissible tile list for (mask, L) is built on the host
  * on first use, copied into a device buffer the library allocates, and
  * cached per (device, mask, L) until jvp_attn_release(). That first call
- * performs a blocking copy and must not be made during stream capture.
+ * performs a blocking copy and must not be made during stream capture. The
+ * tensor-core kernel also takes work items from a 4-byte counter that the
+ * library allocates once per (device, stream) and clears on the stream
+ * before each launch.
  *
  * A row whose admissible set is empty (no descriptor of the four modes
  * yields one) gets O = dO = 0 and LSE = -inf.
@@ -141,20 +144,22 @@ int jvp_attn_fwd(const void* q, const void* k, const void* v,
  * the tensor-core configuration: dtype must be JVP_BF16 (else
  * JVP_ERR_INVALID_ARG) and d must be 128 (else
  * JVP_ERR_UNSUPPORTED_HEAD_DIM). A mask whose work list needs more than
- * 65,536 words (4 per 128-row query tile + 2 per key-tile run; about 81
+ * 65,472 words (4 per 128-row query tile + 2 per key-tile run; about 81
  * words per 1000 tokens for the teacher-forcing mask at 1560 tokens per
  * frame, so roughly 800,000 tokens) returns JVP_ERR_TOO_LARGE before any
  * device work.
  *
  * The first call on a device looks the array's address up
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture. A call whose (mask, L) differs from the list
- * the array holds rewrites the array with an asynchronous copy on `stream`;
- * every word the kernel reads is rewritten, so nothing has to start at
- * zero. All calls on a device share the one array: calls with different
- * (mask, L) whose work overlaps on the GPU (different streams, no ordering
- * between them) race on it and give wrong results. Order such calls on one
- * stream or synchronise between them.
+ * before any stream capture. The array holds the kernel's work-item counter
+ * (its first 64 words, cleared on `stream` before every launch) and the work
+ * list (the rest). A call whose (mask, L) differs from the list the array
+ * holds rewrites the list with an asynchronous copy on `stream`; every word
+ * the kernel reads is rewritten or cleared, so no earlier contents matter.
+ * All calls on a device share the one array: calls whose work overlaps on
+ * the GPU (different streams with no ordering between them) race on it and
+ * give wrong results. Order such calls on one stream or synchronise
+ * between them.
  */
 int jvp_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                          const void* dq, const void* dk, const void* dv,
@@ -206,6 +211,18 @@ int jvp_attn_schedule(jvp_mask_desc mask, int L, int bm, int bn,
  * reports a CUDA error.
  */
 int jvp_attn_check_device_error(void* stream);
+
+/*
+ * jvp_attn_set_wait_limit: upper bound, in nanoseconds, on each wait inside
+ * the tensor-core kernel (for a pipeline stage, a peer warp or a work item).
+ * A wait that runs out makes the kernel record JVP_ERR_DEVICE_TIMEOUT in the
+ * device error word, let its own copies and MMAs finish, free its tensor
+ * memory and exit; the CUDA context stays usable and the outputs of that
+ * launch are undefined. 0 restores the default of 2 s. Process-wide; applies
+ * to launches made after the call. A tiny limit is how the failure path is
+ * tested without faulting a GPU.
+ */
+int jvp_attn_set_wait_limit(uint64_t ns);
 
 /* Frees every cached workspace on every device. Synchronises the device(s)
  * first. Safe to call at any time outside stream capture. */
