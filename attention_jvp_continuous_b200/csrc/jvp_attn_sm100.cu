@@ -74,7 +74,7 @@ enum : uint32_t {
   B_QFULL = 0,
   B_QEMPTY = 1,
   B_KFULL = 2,   // 2 slots
-  B_KEMPTY = 4,  // 2
+  B_KSPARE = 4,  // 2 (unused: S-ready releases the K stage)
   B_VFULL = 6,   // 2
   B_VEMPTY = 8,  // 2
   B_SFULL = 10,  // 2
@@ -118,23 +118,33 @@ struct Params {
   unsigned long long wait_limit_ns;
 };
 
-// Bounded wait. Returns false (and raises the CTA abort flag) on timeout or
-// when another role has already aborted.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Params& p,
-                                         volatile uint32_t* abort_flag) {
-  if (mbar_try(bar, parity)) return true;
+// Slow path of wait_bar, kept out of line so that the hot loops stay small.
+__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity,
+                                           unsigned long long limit_ns, unsigned* err,
+                                           volatile uint32_t* abort_flag) {
   const uint64_t t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
+  for (uint32_t it = 0;; ++it) {
     if (mbar_try(bar, parity)) return true;
-    if ((it & 31u) == 0) {
+    // A try_wait may itself suspend for a while, so the limit is checked
+    // from the first failed poll on.
+    if ((it & 7u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > p.wait_limit_ns) {
-        atomicOr(p.err, kErrTimeout);
+      if (globaltimer() - t0 > limit_ns) {
+        atomicOr(err, kErrTimeout);
         *abort_flag = 1u;
         return false;
       }
     }
   }
+}
+
+// Bounded wait. Returns false (and raises the CTA abort flag) on timeout or
+// when another role has already aborted.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Params& p,
+                                         volatile uint32_t* abort_flag) {
+  // Most waits find the phase already complete: probe without suspending.
+  if (mbar_test(bar, parity)) return true;
+  return wait_bar_slow(bar, parity, p.wait_limit_ns, p.err, abort_flag);
 }
 
 // Work items reach the roles through a 4-slot ring in shared memory: the
@@ -260,7 +270,6 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(bar(B_QEMPTY), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(B_KFULL + s), 1);
-      mbar_init(bar(B_KEMPTY + s), 1);
       mbar_init(bar(B_VFULL + s), 1);
       mbar_init(bar(B_VEMPTY + s), 1);
       mbar_init(bar(B_SFULL + s), 1);
@@ -321,7 +330,9 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         const uint32_t s = c.t & 1u, u = c.t >> 1;
         const int y = c.kt * BN;
-        if (c.t >= 2) ok = wait_bar(bar(B_KEMPTY + s), (u - 1) & 1u, p, abort_flag);
+        // Stage s is free once S(t - 2) is done: the S-ready barrier of that
+        // buffer doubles as the K-stage release.
+        if (c.t >= 2) ok = wait_bar(bar(B_SFULL + s), (u - 1) & 1u, p, abort_flag);
         if (!ok) break;
         mbar_expect_tx(bar(B_KFULL + s), kStageBytes);
         ++k_issued;
@@ -358,31 +369,35 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     // ------------------------------------------------------------ MMA ----
     if (lane == 0) {
       bool ok = true;
+      // Descriptors of the fixed shared-memory operands; an MMA's operand
+      // is the base plus a compile-time byte offset >> 4 (the start-address
+      // field stays below 2^14, so the add never carries out of it).
+      const uint64_t q_desc = sdesc_sw128(base + SM_Q, 16, 1024);
+      const uint64_t dq_desc = sdesc_sw128(base + SM_DQ, 16, 1024);
+      const uint64_t k_desc = sdesc_sw128(base + SM_K, 16, 1024);       // stage 0
+      const uint64_t v_desc = sdesc_sw128(base + SM_V, kKHalf, 1024);   // stage 0
       auto issue_s = [&](const Cursor& c) -> bool {
         const uint32_t b = c.t & 1u;
         if (c.j == 0 && !wait_bar(bar(B_QFULL), c.item_idx & 1, p, abort_flag)) return false;
         if (!wait_bar(bar(B_KFULL + b), (c.t >> 1) & 1u, p, abort_flag)) return false;
         tc_fence_after();
         const uint32_t d_s = tmem + b * 128u, d_ds = d_s + 64u;
-        const uint32_t kb = base + SM_K + b * kStageBytes;
+        const uint64_t kb = k_desc + b * (kStageBytes >> 4);
         // [S | Q dK^T] = Q [K ; dK]^T: one N=128 MMA per 16-wide k-step.
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t oq = (kk >> 2) * kQHalf + (kk & 3) * 32;
-          const uint32_t ob = (kk >> 2) * (2 * kKHalf) + (kk & 3) * 32;
-          mma_ss(d_s, sdesc_sw128(base + SM_Q + oq, 16, 1024),
-                 sdesc_sw128(kb + ob, 16, 1024), IDESC_SK, kk > 0);
+          const uint32_t oq = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
+          const uint32_t ob = ((kk >> 2) * (2 * kKHalf) + (kk & 3) * 32) >> 4;
+          mma_ss(d_s, q_desc + oq, kb + ob, IDESC_SK, kk > 0);
         }
         // dS = Q dK^T + dQ K^T: N=64 MMAs accumulate dQ K^T onto it.
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t oq = (kk >> 2) * kQHalf + (kk & 3) * 32;
-          const uint32_t ob = (kk >> 2) * (2 * kKHalf) + (kk & 3) * 32;
-          mma_ss(d_ds, sdesc_sw128(base + SM_DQ + oq, 16, 1024),
-                 sdesc_sw128(kb + ob, 16, 1024), IDESC_S, 1u);
+          const uint32_t oq = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
+          const uint32_t ob = ((kk >> 2) * (2 * kKHalf) + (kk & 3) * 32) >> 4;
+          mma_ss(d_ds, dq_desc + oq, kb + ob, IDESC_S, 1u);
         }
-        mma_commit(bar(B_KEMPTY + b));
-        mma_commit(bar(B_SFULL + b));
+        mma_commit(bar(B_SFULL + b));  // also releases K stage b to the producer
         if (c.j == c.n - 1) mma_commit(bar(B_QEMPTY));
         return true;
       };
@@ -394,20 +409,19 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!wait_bar(bar(B_PFULL + b), (c.t >> 1) & 1u, p, abort_flag)) return false;
         if (!wait_bar(bar(B_VFULL + b), (c.t >> 1) & 1u, p, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t vb = base + SM_V + b * kStageBytes;
+        const uint64_t vb = v_desc + b * (kStageBytes >> 4);
         const uint32_t a_p = tmem + b * 128u, a_pd = a_p + 64u;
         const uint32_t first = c.j == 0 ? 0u : 1u;
         // [A1 | A23] += P [V | dV]: one N=256 MMA per 16-key step (A1 and A23
         // are adjacent in TMEM; V h0, V h1, dV h0, dV h1 are 8 KB apart).
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts(tmem + TM_A1, a_p + ks * 8, sdesc_sw128(vb + ks * 2048, kKHalf, 1024),
-                 IDESC_PVV, first | (ks > 0));
+          mma_ts(tmem + TM_A1, a_p + ks * 8, vb + ((ks * 2048) >> 4), IDESC_PVV,
+                 first | (ks > 0));
         // A23 += (scale e dS) V
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts(tmem + TM_A23, a_pd + ks * 8, sdesc_sw128(vb + ks * 2048, kKHalf, 1024),
-                 IDESC_PV, 1u);
+          mma_ts(tmem + TM_A23, a_pd + ks * 8, vb + ((ks * 2048) >> 4), IDESC_PV, 1u);
         mma_commit(bar(B_VEMPTY + b));
         mma_commit(bar(B_PVDONE));
         return true;
@@ -531,21 +545,39 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         tmem_wait_st();
       }
       const float mref_use = m_ref == -CUDART_INF_F ? 0.f : m_ref;
+      // Pairs of columns in packed fp32 (f32x2) arithmetic: 2^(c2 s - m),
+      // e dS, the partial sums and scale e dS take one instruction per pair.
+      const uint64_t c2v = f2pack(p.c2, p.c2), mv = f2pack(-mref_use, -mref_use);
+      const uint64_t scv = f2pack(p.scale, p.scale);
+      uint64_t la = 0, lb = 0, ga = 0, gb = 0;  // 0 = two +0.0f
       uint32_t pp[16], pd[16];
-      float l4[4] = {0.f, 0.f, 0.f, 0.f}, g4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float e0 = ex2(fmaf(s[2 * i], p.c2, -mref_use));
-        const float e1 = ex2(fmaf(s[2 * i + 1], p.c2, -mref_use));
-        const float ed0 = e0 * __uint_as_float(dr[2 * i]);
-        const float ed1 = e1 * __uint_as_float(dr[2 * i + 1]);
-        l4[i & 3] += e0 + e1;
-        g4[i & 3] += ed0 + ed1;
+        float x0, x1;
+        f2unpack(fma2(f2pack(s[2 * i], s[2 * i + 1]), c2v, mv), x0, x1);
+        const float e0 = ex2(x0), e1 = ex2(x1);
+        const uint64_t ev = f2pack(e0, e1);
+        const uint64_t edv =
+            mul2(ev, f2pack(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1])));
+        if (i & 1) {
+          lb = add2(lb, ev);
+          gb = add2(gb, edv);
+        } else {
+          la = add2(la, ev);
+          ga = add2(ga, edv);
+        }
         pp[i] = pack_bf16(e0, e1);
-        pd[i] = pack_bf16(ed0 * p.scale, ed1 * p.scale);
+        float q0, q1;
+        f2unpack(mul2(edv, scv), q0, q1);
+        pd[i] = pack_bf16(q0, q1);
       }
-      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-      g += (g4[0] + g4[1]) + (g4[2] + g4[3]);
+      {
+        float u0, u1;
+        f2unpack(add2(la, lb), u0, u1);
+        l += u0 + u1;
+        f2unpack(add2(ga, gb), u0, u1);
+        g += u0 + u1;
+      }
       // bf16 e into S columns [16 hw, 16 hw + 16), scale*e*dS into the dS ones.
       tmem_st16(tl + b * 128u + 16u * hw, pp);
       tmem_st16(tl + b * 128u + 64u + 16u * hw, pd);
