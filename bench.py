@@ -39,6 +39,7 @@ UNIT = "TFLOP/s"
 NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 KERNEL_SOURCES = ["attention_jvp_continuous_b200/csrc/jvp_attn_sm100.cu",
+                  "attention_jvp_continuous_b200/csrc/sm100_pipeline.cuh",
                   "attention_jvp_continuous_b200/csrc/sm100_ptx.cuh",
                   "attention_jvp_continuous_b200/csrc/mask_rows.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")

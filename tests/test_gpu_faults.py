@@ -1,0 +1,47 @@
+"""Failure detection on the GPU without faulting it: every wait inside the
+tensor-core kernel is bounded. With a 1 ns limit the first wait that cannot
+be satisfied at once gives up; the kernel records a timeout in the device
+error word, drains its own copies and MMAs, frees its tensor memory and
+exits. The host reads the error, and the same context then computes correct
+results again."""
+import numpy as np
+import pytest
+import torch
+
+import attention_jvp_continuous_b200 as ja
+from attention_jvp_continuous_b200 import _lib
+from attention_jvp_continuous_b200.inputs import Workload, make_inputs
+from oracle import MaskSpec, jvp_attention
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from attention_jvp_continuous_b200 import build
+    build.build()
+
+
+def test_wait_timeout_is_reported_and_context_recovers():
+    w = Workload("fault_tf", 1, 2, 128, ja.TEACHER_FORCING, 100, 3, 1, "bf16", 0.1)
+    mask = ja.Mask(w.mode, w.tokens_per_frame, w.n_frames, w.chunk)
+    inputs, _ = make_inputs(w, device="cpu")
+    dev = [t.cuda() for t in inputs]
+    ja.check_device_error()  # start clean
+    try:
+        ja.set_wait_limit(1)
+        ja.jvp_attn(*dev, mask)
+        with pytest.raises(ja.JvpAttnError) as e:
+            ja.check_device_error()
+        assert e.value.code == _lib.JVP_ERR_DEVICE_TIMEOUT
+    finally:
+        ja.set_wait_limit(0)
+    ja.check_device_error()  # the word was cleared by the read
+    o, do, _ = ja.jvp_attn(*dev, mask)
+    ja.check_device_error()
+    ref = jvp_attention(*inputs, MaskSpec(w.mode, w.tokens_per_frame, w.n_frames, w.chunk))
+    for got, want in ((o, ref[0]), (do, ref[1])):
+        g = got.float().cpu().numpy().astype(np.float64)
+        assert np.linalg.norm(g - want) <= 5e-3 * np.linalg.norm(want)
