@@ -19,8 +19,9 @@ FRAME_CAUSAL = 1
 CHUNK_CAUSAL = 2
 TEACHER_FORCING = 3
 
-__all__ = ["Mask", "jvp_attn", "jvp_attn_fwd", "mask_stats", "tile_classes",
-           "schedule", "check_device_error", "set_wait_limit", "release", "JvpAttnError",
+__all__ = ["Mask", "jvp_attn", "jvp_attn_fwd", "attn_bwd", "mask_stats", "tile_classes",
+           "schedule", "schedule_kv", "check_device_error", "set_wait_limit", "release",
+           "JvpAttnError",
            "DENSE", "FRAME_CAUSAL", "CHUNK_CAUSAL", "TEACHER_FORCING"]
 
 
@@ -98,6 +99,32 @@ def jvp_attn(q, k, v, dq, dk, dv, mask: Mask, scale: Optional[float] = None,
     return o, d_o, lse
 
 
+def attn_bwd(q, k, v, o, g, lse, mask: Mask, scale: Optional[float] = None,
+             stream: Optional[int] = None):
+    """Gradients (g_q, g_k, g_v) of sum <g, o> for o = masked attention of
+    (q, k, v); o and lse as returned by jvp_attn. bf16 CUDA tensors, d = 128."""
+    import torch
+    ts = (q, k, v, o, g)
+    for t in ts:
+        if not t.is_cuda or t.shape != q.shape or t.dtype != q.dtype or not t.is_contiguous():
+            raise ValueError("q, k, v, o, g must be contiguous CUDA tensors of one shape and dtype")
+    if not lse.is_cuda or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 CUDA tensor [B, H, L]")
+    B, H, L, d = q.shape
+    gq, gk, gv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    scratch = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    fp = ctypes.POINTER(ctypes.c_float)
+    rc = _lib.lib().jvp_attn_bwd(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), g.data_ptr(),
+        ctypes.cast(lse.data_ptr(), fp), gq.data_ptr(), gk.data_ptr(), gv.data_ptr(),
+        ctypes.cast(scratch.data_ptr(), fp), B, H, L, d, _dtype_code(q), mask.desc(),
+        0.0 if scale is None else float(scale), ctypes.c_void_p(stream))
+    _lib.check(rc, "jvp_attn_bwd")
+    return gq, gk, gv
+
+
 def mask_stats(mask: Mask, L: Optional[int] = None, bm: int = 128, bn: int = 64):
     """(pairs, full, partial, empty) for the mask on a bm x bn tile grid."""
     L = mask.length if L is None else L
@@ -136,6 +163,24 @@ def schedule(mask: Mask, L: Optional[int] = None, bm: int = 128, bn: int = 64):
                                ctypes.byref(ns))
     _lib.check(rc, "jvp_attn_schedule")
     return qt, sg
+
+
+def schedule_kv(mask: Mask, L: Optional[int] = None, bq: int = 64, bk: int = 128):
+    """(ktiles [n, 4], segs [m, 3]) int32 arrays of the backward key-pass work list."""
+    import numpy as np
+    L = mask.length if L is None else L
+    nk, ns = ctypes.c_int(), ctypes.c_int()
+    lib = _lib.lib()
+    lib.jvp_attn_schedule_kv(mask.desc(), L, bq, bk, None, 0, None, 0,
+                             ctypes.byref(nk), ctypes.byref(ns))
+    kt = np.zeros((nk.value, 4), dtype=np.int32)
+    sg = np.zeros((ns.value, 3), dtype=np.int32)
+    p32 = ctypes.POINTER(ctypes.c_int32)
+    rc = lib.jvp_attn_schedule_kv(mask.desc(), L, bq, bk, kt.ctypes.data_as(p32), nk.value,
+                                  sg.ctypes.data_as(p32), ns.value, ctypes.byref(nk),
+                                  ctypes.byref(ns))
+    _lib.check(rc, "jvp_attn_schedule_kv")
+    return kt, sg
 
 
 def check_device_error(stream: Optional[int] = None) -> None:

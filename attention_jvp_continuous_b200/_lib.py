@@ -32,8 +32,9 @@ JVP_FP32 = 1
 TILE_EMPTY, TILE_FULL, TILE_PARTIAL = 0, 1, 2
 
 # Exported functions, as declared in include/jvp_attn.h.
-EXPORTS = ("jvp_attn_fwd", "jvp_attn_fwd_noalloc", "jvp_attn_mask_stats", "jvp_attn_tile_classes",
-           "jvp_attn_schedule", "jvp_attn_check_device_error",
+EXPORTS = ("jvp_attn_fwd", "jvp_attn_fwd_noalloc", "jvp_attn_bwd", "jvp_attn_mask_stats",
+           "jvp_attn_tile_classes", "jvp_attn_schedule", "jvp_attn_schedule_kv",
+           "jvp_attn_check_device_error",
            "jvp_attn_set_wait_limit", "jvp_attn_release", "jvp_attn_strerror",
            "jvp_attn_version")
 
@@ -74,6 +75,10 @@ def lib() -> ctypes.CDLL:
         L.jvp_attn_fwd.restype = i32
         L.jvp_attn_fwd_noalloc.argtypes = L.jvp_attn_fwd.argtypes
         L.jvp_attn_fwd_noalloc.restype = i32
+        fp = ctypes.POINTER(ctypes.c_float)
+        L.jvp_attn_bwd.argtypes = [vp] * 5 + [fp] + [vp] * 3 + [fp] + [i32] * 5 + \
+            [MaskDesc, ctypes.c_float, vp]
+        L.jvp_attn_bwd.restype = i32
         L.jvp_attn_mask_stats.argtypes = [MaskDesc, i32, i32, i32, i64p, i64p, i64p, i64p]
         L.jvp_attn_mask_stats.restype = i32
         L.jvp_attn_tile_classes.argtypes = [MaskDesc, i32, i32, i32,
@@ -83,6 +88,8 @@ def lib() -> ctypes.CDLL:
         L.jvp_attn_schedule.argtypes = [MaskDesc, i32, i32, i32, i32p, i32, i32p, i32,
                                         ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
         L.jvp_attn_schedule.restype = i32
+        L.jvp_attn_schedule_kv.argtypes = L.jvp_attn_schedule.argtypes
+        L.jvp_attn_schedule_kv.restype = i32
         L.jvp_attn_check_device_error.argtypes = [vp]
         L.jvp_attn_check_device_error.restype = i32
         L.jvp_attn_set_wait_limit.argtypes = [ctypes.c_uint64]

@@ -42,6 +42,24 @@ int launch_simt(const LaunchArgs& a, bool bf16);
 // Tensor-core kernel: bf16, d = 128, sm_100a.
 int launch_sm100(const LaunchArgs& a, const WorkList& w, int num_sms);
 
+struct BwdArgs {
+  const void *q, *k, *v, *o, *g;  // g: cotangent of o
+  const float* lse;               // forward LSE
+  void *gq, *gk, *gv;
+  float* dvec;                    // scratch [B, H, L]: D = <g, o> per row
+  int B, H, L, d;
+  jvp_mask_desc mask;
+  float scale;
+  cudaStream_t stream;
+  unsigned* err;
+  unsigned* item_ctr;  // two u32 words: one per pass
+  unsigned long long wait_limit_ns;
+};
+
+// Backward passes (dQ, then dK/dV): bf16, d = 128, sm_100a. wq: query-tile
+// work list (128 x 64 grid); wkv: key-tile work list (64 x 128 grid).
+int launch_bwd_sm100(const BwdArgs& a, const WorkList& wq, const WorkList& wkv, int num_sms);
+
 // Per-wait limit for the tensor-core kernel (jvp_attn_set_wait_limit).
 unsigned long long wait_limit_ns();
 

@@ -35,10 +35,10 @@ struct DevInfo {
 };
 
 struct WsKey {
-  int dev, mode, T, F, chunk, L, bm, bn;
+  int dev, mode, T, F, chunk, L, bm, bn, kind;  // kind 0: query-tile list, 1: key-tile list
   bool operator<(const WsKey& o) const {
-    return std::tie(dev, mode, T, F, chunk, L, bm, bn) <
-           std::tie(o.dev, o.mode, o.T, o.F, o.chunk, o.L, o.bm, o.bn);
+    return std::tie(dev, mode, T, F, chunk, L, bm, bn, kind) <
+           std::tie(o.dev, o.mode, o.T, o.F, o.chunk, o.L, o.bm, o.bn, o.kind);
   }
 };
 
@@ -80,16 +80,17 @@ int device_info(DevInfo** out) {
   return JVP_OK;
 }
 
-int get_worklist(int dev, const jvp_mask_desc& m, int L, WorkList* out) {
+int get_worklist(int dev, const jvp_mask_desc& m, int L, WorkList* out, int bm = kBM,
+                 int bn = kBN, int kind = 0) {
   const WsKey key{dev, m.mode, m.tokens_per_frame, m.n_frames,
-                  m.chunk, L, kBM, kBN};
+                  m.chunk, L, bm, bn, kind};
   std::lock_guard<std::mutex> lk(g_mu);
   auto it = g_ws.find(key);
   if (it != g_ws.end()) {
     *out = it->second.w;
     return JVP_OK;
   }
-  const Schedule s = build_schedule(m, L, kBM, kBN);
+  const Schedule s = kind == 0 ? build_schedule(m, L, bm, bn) : build_schedule_kv(m, L, bm, bn);
   const size_t qbytes = s.qtiles.size() * sizeof(int32_t);
   const size_t sbytes = s.segs.size() * sizeof(int32_t);
   const size_t soff = (qbytes + 255) & ~size_t(255);
@@ -194,6 +195,66 @@ int jvp_attn_fwd(const void* q, const void* k, const void* v, const void* dq, co
   rc = get_counter(dev, a.stream, &a.item_ctr);
   if (rc != JVP_OK) return rc;
   return launch_sm100(a, w, di->sms);
+}
+
+int jvp_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* g_o,
+                 const float* lse, void* g_q, void* g_k, void* g_v, float* scratch, int B, int H,
+                 int L, int d, jvp_dtype dtype, jvp_mask_desc mask, float softmax_scale,
+                 void* stream) {
+  if (!q || !k || !v || !o || !g_o || !lse || !g_q || !g_k || !g_v || !scratch)
+    return JVP_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || dtype != JVP_BF16) return JVP_ERR_INVALID_ARG;
+  if (std::isnan(softmax_scale) || std::isinf(softmax_scale)) return JVP_ERR_INVALID_ARG;
+  if (d != 128) return JVP_ERR_UNSUPPORTED_HEAD_DIM;
+  int rc = validate_mask(mask, L);
+  if (rc != JVP_OK) return rc;
+  if ((long long)B * H * L >= (1LL << 31) || (long long)B * H >= (1LL << 31) / 2)
+    return JVP_ERR_TOO_LARGE;
+  const void* ptrs[] = {q, k, v, o, g_o, lse, g_q, g_k, g_v, scratch};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return JVP_ERR_MISALIGNED;
+  DevInfo* di = nullptr;
+  rc = device_info(&di);
+  if (rc != JVP_OK) return rc;
+  if (di->major != 10 || di->minor != 0) return JVP_ERR_UNSUPPORTED_DEVICE;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  BwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.o = o; a.g = g_o; a.lse = lse;
+  a.gq = g_q; a.gk = g_k; a.gv = g_v; a.dvec = scratch;
+  a.B = B; a.H = H; a.L = L; a.d = d;
+  a.mask = mask;
+  a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(d));
+  a.stream = static_cast<cudaStream_t>(stream);
+  a.err = di->err;
+  a.wait_limit_ns = wait_limit_ns();
+  WorkList wq, wkv;
+  rc = get_worklist(dev, mask, L, &wq, 128, 64, 0);
+  if (rc != JVP_OK) return rc;
+  rc = get_worklist(dev, mask, L, &wkv, 64, 128, 1);
+  if (rc != JVP_OK) return rc;
+  rc = get_counter(dev, a.stream, &a.item_ctr);
+  if (rc != JVP_OK) return rc;
+  return launch_bwd_sm100(a, wq, wkv, di->sms);
+}
+
+int jvp_attn_schedule_kv(jvp_mask_desc mask, int L, int bq, int bk, int32_t* ktiles,
+                         int ktile_cap, int32_t* segs, int seg_cap, int* n_ktiles, int* n_segs) {
+  int rc = validate_mask(mask, L);
+  if (rc != JVP_OK) return rc;
+  if (bq < 1 || bk < 1) return JVP_ERR_INVALID_ARG;
+  const Schedule s = build_schedule_kv(mask, L, bq, bk);
+  const int nk = int(s.qtiles.size() / 4), ns = int(s.segs.size() / 2);
+  if (n_ktiles) *n_ktiles = nk;
+  if (n_segs) *n_segs = ns;
+  if (!ktiles || !segs || ktile_cap < nk || seg_cap < ns) return JVP_ERR_INVALID_ARG;
+  std::memcpy(ktiles, s.qtiles.data(), s.qtiles.size() * sizeof(int32_t));
+  for (int i = 0; i < ns; ++i) {
+    segs[3 * i] = s.segs[2 * i];
+    segs[3 * i + 1] = s.segs[2 * i + 1] >> 1;
+    segs[3 * i + 2] = s.segs[2 * i + 1] & 1;
+  }
+  return JVP_OK;
 }
 
 int jvp_attn_mask_stats(jvp_mask_desc mask, int L, int bm, int bn, int64_t* pairs,

@@ -1,0 +1,543 @@
+// Backward pass of masked softmax attention for B200 (sm_100a): the gradient
+// of sum <G, O> with O = softmax(c QK^T + M) V (Causal-rCM report, Eq. 42;
+// the consistency loss is differentiated through the primal output only,
+// Appendix A). With P = exp(c QK^T - LSE) (the forward's LSE), D_i = <g_i, o_i>:
+//   dP = G V^T,  dS = P o (dP - D),  gQ = c dS K,  gK = c dS^T Q,  gV = P^T G.
+//
+// Two persistent tcgen05 kernels over the same admissible-tile work lists:
+//  * dQ pass (query-stationary, 128 query rows per item, 64-key tiles):
+//      S = Q K^T, dP = G V^T   (SS MMAs, N = 64, fp32 in TMEM)
+//      softmax warps: P, dS    (one row per thread, bf16 dS back to TMEM)
+//      gQ += dS K              (TS MMA, N = 128, accumulator in TMEM)
+//    and it writes D_i to a scratch vector for the second pass.
+//  * dK/dV pass (key-stationary, 128 keys per item, 64-query tiles):
+//      S^T = K Q^T, dP^T = V G^T
+//      softmax warps: P^T, dS^T (one key per thread; per-query LSE and D)
+//      gV += P^T G, gK += dS^T Q (TS MMAs, N = 128)
+// Warp roles as in the JVP kernel: warp 0 TMA, warp 1 MMA issue (one
+// thread), warps 4-11 two warpgroups taking 32 of each tile's 64 columns.
+// Each warpgroup writes its bf16 operands into the TMEM columns it has just
+// read itself, so no exchange between the warpgroups is needed.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "mask_rows.cuh"
+#include "sm100_pipeline.cuh"
+#include "sm100_ptx.cuh"
+
+namespace jvp {
+namespace bwd {
+
+using namespace jvp::ptx;
+using pipe::drain_wait;
+using pipe::ItemRing;
+using pipe::kConsumerThread;
+using pipe::kConsumerWarp;
+using pipe::kProducer;
+using pipe::kRing;
+using pipe::kRingReaders;
+using pipe::wait_bar;
+
+constexpr int BR = 128;  // stationary rows per item (TMEM lanes)
+constexpr int BT = 64;   // streamed rows per tile
+constexpr int D = 128;
+constexpr int kThreads = 384;
+
+constexpr uint32_t kRHalf = BR * 128;  // 16 KB: 128 rows x 64 head-dim columns
+constexpr uint32_t kTHalf = BT * 128;  //  8 KB: 64 rows x 64 columns
+constexpr uint32_t kTile = 2 * kTHalf; // 16 KB: one streamed 64-row operand
+
+// Shared memory: two stationary operands (A0, A1), then streamed operands
+// in rings: ring X with 3 stages, ring Y with 2 or 3 stages.
+constexpr uint32_t SM_A0 = 0;
+constexpr uint32_t SM_A1 = 2 * kRHalf;
+constexpr uint32_t SM_X = 4 * kRHalf;         // 3 stages of kTile
+constexpr uint32_t SM_Y = SM_X + 3 * kTile;   // 3 stages of kTile
+constexpr uint32_t SM_BAR = SM_Y + 3 * kTile; // 160 KB
+constexpr uint32_t kSmemBytes = SM_BAR + 512 + 1024;
+
+enum : uint32_t {
+  B_AF = 0,      // stationary operands landed
+  B_AE = 1,      // stationary operands may be overwritten
+  B_XF = 2,      // 3
+  B_XE = 5,      // 3
+  B_YF = 8,      // 3
+  B_YE = 11,     // 3
+  B_SF = 14,     // 2: S / dP buffer ready
+  B_PF = 16,     // 2: bf16 operands written by the softmax warps
+  B_MD = 18,     // accumulating MMA of a tile done
+  B_CF = 19,     // accumulators read by the epilogue
+  B_DRAIN = 20,
+  B_IF = 21,     // 4: work-item ring
+  B_IE = 25,     // 4
+  kNumBars = 29
+};
+constexpr uint32_t SM_TMEM_SLOT = SM_BAR + 8 * kNumBars;
+constexpr uint32_t SM_ABORT = SM_TMEM_SLOT + 4;
+constexpr uint32_t SM_RING = SM_ABORT + 4;
+static_assert(SM_RING + 16 <= SM_BAR + 512, "barrier area overflow");
+
+constexpr uint32_t TM_C0 = 256;  // first accumulator (gQ, or gV)
+constexpr uint32_t TM_C1 = 384;  // second accumulator (gK)
+
+constexpr uint32_t IDESC_N64 = ptx::idesc_bf16(BR, BT, false, false);  // 128 x 64, K-major B
+constexpr uint32_t IDESC_MN = ptx::idesc_bf16(BR, D, false, true);     // 128 x 128, MN-major B
+
+struct Params {
+  const int4* qtiles;  // work entries {outer tile, seg_begin, seg_count, inner tiles}
+  const int2* segs;
+  int n_entries, n_segs, n_items, n_qt, n_kt;  // n_qt: outer tiles, n_kt: inner tiles
+  int L;
+  jvp_mask_desc mask;
+  float scale, c2;
+  const float* lse;     // forward LSE (natural log)
+  float* dvec;          // D_i = <g_i, o_i>: written by the dQ pass, read by the dK/dV pass
+  const __nv_bfloat16* g;  // cotangent, for D (dQ pass)
+  const __nv_bfloat16* o;  // forward output, for D (dQ pass)
+  __nv_bfloat16* out0;     // gQ (dQ pass) or gK (dK/dV pass)
+  __nv_bfloat16* out1;     // gV (dK/dV pass)
+  unsigned* err;
+  unsigned* item_ctr;
+  unsigned long long wait_limit_ns;
+};
+using Cursor = pipe::Cursor<Params>;
+
+// Stationary operand for the stationary-side MMAs (K-major, 128 rows) and
+// streamed operands (64 rows) that serve both as K-major B (first MMAs) and
+// as MN-major B (accumulating MMAs).
+template <bool kKV>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
+           const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
+           const __grid_constant__ Params p) {
+  // dQ pass:  A0 = Q, A1 = G (stationary);  X = K (3 stages), Y = V.
+  // dK/dV:    A0 = K, A1 = V (stationary);  X = Q (3 stages), Y = G.
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const base_ptr = smem_raw + (base - raw);
+  auto bar = [&](uint32_t slot) { return base + SM_BAR + 8u * slot; };
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + SM_ABORT);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_AF), 1);
+    mbar_init(bar(B_AE), 1);
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(bar(B_XF + s), 1);
+      mbar_init(bar(B_XE + s), 1);
+      mbar_init(bar(B_YF + s), 1);
+      mbar_init(bar(B_YE + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(B_SF + b), 1);
+      mbar_init(bar(B_PF + b), 2 * BR);
+    }
+    mbar_init(bar(B_MD), 1);
+    mbar_init(bar(B_CF), 2 * BR);
+    mbar_init(bar(B_DRAIN), 1);
+    for (uint32_t i = 0; i < kRing; ++i) {
+      mbar_init(bar(B_IF + i), 1);
+      mbar_init(bar(B_IE + i), kRingReaders);
+    }
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tm_a0);
+    tma_prefetch_map(&tm_a1);
+    tma_prefetch_map(&tm_x);
+    tma_prefetch_map(&tm_y);
+  }
+  if (warp == 1) {
+    tmem_alloc(base + SM_TMEM_SLOT, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base_ptr + SM_TMEM_SLOT);
+  const ItemRing ring{bar(B_IF), bar(B_IE),
+                      reinterpret_cast<volatile int*>(base_ptr + SM_RING), abort_flag};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA ----
+    if (lane == 0) {
+      Cursor c;
+      c.start(p, ring, kProducer);
+      uint32_t a_armed = 0, x_issued = 0, y_issued = 0;
+      bool ok = true;
+      while (c.valid && ok) {
+        if (c.j == 0) {
+          if (c.item_idx > 0) ok = wait_bar(bar(B_AE), (c.item_idx - 1) & 1, p, abort_flag);
+          if (!ok) break;
+          mbar_expect_tx(bar(B_AF), 4 * kRHalf);
+          ++a_armed;
+          const int y = c.qt * BR;
+          tma_load_3d(base + SM_A0, &tm_a0, bar(B_AF), 0, y, c.bh);
+          tma_load_3d(base + SM_A0 + kRHalf, &tm_a0, bar(B_AF), 64, y, c.bh);
+          tma_load_3d(base + SM_A1, &tm_a1, bar(B_AF), 0, y, c.bh);
+          tma_load_3d(base + SM_A1 + kRHalf, &tm_a1, bar(B_AF), 64, y, c.bh);
+        }
+        const int y = c.kt * BT;
+        const uint32_t sx = c.t % 3, ux = c.t / 3;
+        if (c.t >= 3) ok = wait_bar(bar(B_XE + sx), (ux - 1) & 1u, p, abort_flag);
+        if (!ok) break;
+        mbar_expect_tx(bar(B_XF + sx), kTile);
+        ++x_issued;
+        tma_load_3d(base + SM_X + sx * kTile, &tm_x, bar(B_XF + sx), 0, y, c.bh);
+        tma_load_3d(base + SM_X + sx * kTile + kTHalf, &tm_x, bar(B_XF + sx), 64, y, c.bh);
+        const uint32_t sy = c.t % 3, uy = c.t / 3;
+        if (c.t >= 3) ok = wait_bar(bar(B_YE + sy), (uy - 1) & 1u, p, abort_flag);
+        if (!ok) break;
+        mbar_expect_tx(bar(B_YF + sy), kTile);
+        ++y_issued;
+        tma_load_3d(base + SM_Y + sy * kTile, &tm_y, bar(B_YF + sy), 0, y, c.bh);
+        tma_load_3d(base + SM_Y + sy * kTile + kTHalf, &tm_y, bar(B_YF + sy), 64, y, c.bh);
+        c.next(p, ring, kProducer);
+      }
+      if (!ok || *abort_flag) {
+        if (a_armed) drain_wait(bar(B_AF), (a_armed - 1) & 1u);
+        for (uint32_t s = 0; s < 3; ++s) {
+          const uint32_t nx = (x_issued + 2 - s) / 3, ny = (y_issued + 2 - s) / 3;
+          if (nx) drain_wait(bar(B_XF + s), (nx - 1) & 1u);
+          if (ny) drain_wait(bar(B_YF + s), (ny - 1) & 1u);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA ----
+    if (lane == 0) {
+      bool ok = true;
+      const uint64_t a0_desc = sdesc_sw128(base + SM_A0, 16, 1024);
+      const uint64_t a1_desc = sdesc_sw128(base + SM_A1, 16, 1024);
+      const uint64_t xk_desc = sdesc_sw128(base + SM_X, 16, 1024);       // K-major view
+      const uint64_t xm_desc = sdesc_sw128(base + SM_X, kTHalf, 1024);   // MN-major view
+      const uint64_t yk_desc = sdesc_sw128(base + SM_Y, 16, 1024);
+      const uint64_t ym_desc = sdesc_sw128(base + SM_Y, kTHalf, 1024);
+      // First MMAs of a tile: T0 = A0 X^T into S, T1 = A1 Y^T into dP.
+      auto issue_s = [&](const Cursor& c) -> bool {
+        const uint32_t b = c.t & 1u, sx = c.t % 3, sy = c.t % 3;
+        if (c.j == 0 && !wait_bar(bar(B_AF), c.item_idx & 1, p, abort_flag)) return false;
+        if (!wait_bar(bar(B_XF + sx), (c.t / 3) & 1u, p, abort_flag)) return false;
+        if (!wait_bar(bar(B_YF + sy), (c.t / 3) & 1u, p, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t d_s = tmem + b * 128u, d_p = d_s + 64u;
+        const uint64_t xb = xk_desc + sx * (kTile >> 4), yb = yk_desc + sy * (kTile >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t oa = ((kk >> 2) * kRHalf + (kk & 3) * 32) >> 4;
+          const uint32_t ob = ((kk >> 2) * kTHalf + (kk & 3) * 32) >> 4;
+          mma_ss(d_s, a0_desc + oa, xb + ob, IDESC_N64, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t oa = ((kk >> 2) * kRHalf + (kk & 3) * 32) >> 4;
+          const uint32_t ob = ((kk >> 2) * kTHalf + (kk & 3) * 32) >> 4;
+          mma_ss(d_p, a1_desc + oa, yb + ob, IDESC_N64, kk > 0);
+        }
+        mma_commit(bar(B_SF + b));
+        if (!kKV) mma_commit(bar(B_YE + sy));  // dQ pass: V is used by dP only
+        if (c.j == c.n - 1) mma_commit(bar(B_AE));
+        return true;
+      };
+      // Accumulating MMAs. The bf16 operands of a tile sit in TMEM columns
+      // {0, 8} and {32, 40} (one pair of 16-wide k-steps per warpgroup).
+      auto issue_acc = [&](const Cursor& c) -> bool {
+        const uint32_t b = c.t & 1u, sx = c.t % 3, sy = c.t % 3;
+        if (c.j == 0 && c.item_idx > 0 &&
+            !wait_bar(bar(B_CF), (c.item_idx - 1) & 1, p, abort_flag))
+          return false;
+        if (!wait_bar(bar(B_PF + b), (c.t >> 1) & 1u, p, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t first = c.j == 0 ? 0u : 1u;
+        const uint32_t a_p = tmem + b * 128u;  // dQ pass: dS; dK/dV pass: P^T
+#pragma unroll
+        for (int ks = 0; ks < BT / 16; ++ks) {
+          const uint32_t col = (ks >> 1) * 32u + (ks & 1) * 8u;
+          if (!kKV) {
+            // gQ += dS K
+            mma_ts(tmem + TM_C0, a_p + col, xm_desc + sx * (kTile >> 4) + ((ks * 2048) >> 4),
+                   IDESC_MN, first | (ks > 0));
+          } else {
+            // gV += P^T G ; gK += dS^T Q
+            mma_ts(tmem + TM_C0, a_p + col, ym_desc + sy * (kTile >> 4) + ((ks * 2048) >> 4),
+                   IDESC_MN, first | (ks > 0));
+            mma_ts(tmem + TM_C1, a_p + 64u + col,
+                   xm_desc + sx * (kTile >> 4) + ((ks * 2048) >> 4), IDESC_MN,
+                   first | (ks > 0));
+          }
+        }
+        mma_commit(bar(B_XE + sx));
+        if (kKV) mma_commit(bar(B_YE + sy));
+        mma_commit(bar(B_MD));
+        return true;
+      };
+      Cursor cs, cp;
+      cs.start(p, ring, kConsumerThread);
+      cp.start(p, ring, kConsumerThread);
+      for (int pre = 0; pre < 2 && cs.valid && ok; ++pre) {
+        ok = issue_s(cs);
+        cs.next(p, ring, kConsumerThread);
+      }
+      while (cp.valid && ok) {
+        ok = issue_acc(cp);
+        cp.next(p, ring, kConsumerThread);
+        if (ok && cs.valid) {
+          ok = issue_s(cs);
+          cs.next(p, ring, kConsumerThread);
+        }
+      }
+      if (!ok || *abort_flag) {
+        mma_commit(bar(B_DRAIN));
+        drain_wait(bar(B_DRAIN), 0);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------ softmax warps ----
+    const int hw = (warp - 4) >> 2;
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const uint32_t tl = tmem + (uint32_t(q4 * 32) << 16);
+    const int chunk = p.mask.chunk < 1 ? 1 : p.mask.chunk;
+    const float kLog2e = 1.4426950408889634f;
+    Cursor c;
+    c.start(p, ring, kConsumerWarp);
+    RowKeys rk{0, 0, 0, 0};
+    int grow = 0;
+    float lse2 = 0.f, dval = 0.f;  // dQ pass: this row's LSE (log2) and D
+    bool ok = true;
+    while (c.valid) {
+      if (c.j == 0) {
+        grow = c.qt * BR + r;
+        if (!kKV) {
+          rk = row_keys(p.mask.mode, p.mask.tokens_per_frame, p.mask.n_frames, chunk, p.L, grow);
+          lse2 = -CUDART_INF_F;
+          dval = 0.f;
+          if (grow < p.L) {
+            const size_t roff = size_t(c.bh) * p.L + grow;
+            const float l = p.lse[roff];
+            lse2 = l * kLog2e;
+            // D = <g, o> for this row, both 128-wide rows read as 16 B vectors.
+            const uint4* gr = reinterpret_cast<const uint4*>(p.g + roff * D);
+            const uint4* orow = reinterpret_cast<const uint4*>(p.o + roff * D);
+            float acc = 0.f;
+#pragma unroll 4
+            for (int i = 0; i < D / 8; ++i) {
+              const uint4 a = gr[i], bq = orow[i];
+              const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+              const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bq);
+#pragma unroll
+              for (int k2 = 0; k2 < 4; ++k2) {
+                const float2 fa = __bfloat1622float2(a2[k2]), fb = __bfloat1622float2(b2[k2]);
+                acc = fmaf(fa.x, fb.x, fmaf(fa.y, fb.y, acc));
+              }
+            }
+            dval = acc;
+            if (hw == 0) p.dvec[roff] = dval;
+          }
+        } else {
+          rk = key_queries(p.mask.mode, p.mask.tokens_per_frame, p.mask.n_frames, chunk, p.L,
+                           grow);
+        }
+      }
+      const uint32_t b = c.t & 1u;
+      ok = wait_bar(bar(B_SF + b), (c.t >> 1) & 1u, p, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      uint32_t sr[32], dr[32];
+      tmem_ld32(tl + b * 128u + 32u * hw, sr);
+      tmem_ld32(tl + b * 128u + 64u + 32u * hw, dr);
+      tmem_wait_ld();
+      // Column indices of this thread's 32 elements: keys (dQ pass) or
+      // queries (dK/dV pass) [col0, col0 + 32).
+      const int col0 = c.kt * BT + 32 * hw;
+      uint32_t pp[16], pd[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float e[2], ds[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int ci = col0 + 2 * i + h;
+          const float sv = __uint_as_float(sr[2 * i + h]);
+          const float dp = __uint_as_float(dr[2 * i + h]);
+          float l2, dd;
+          bool keep = !c.partial || key_ok(rk, ci);
+          if (!kKV) {
+            l2 = lse2;
+            dd = dval;
+            keep = keep && lse2 != -CUDART_INF_F;
+          } else {
+            // Per-query LSE and D: the same address for all lanes (broadcast).
+            const size_t qoff = size_t(c.bh) * p.L + (keep ? ci : 0);
+            l2 = keep ? __ldg(p.lse + qoff) * kLog2e : 0.f;
+            dd = keep ? __ldg(p.dvec + qoff) : 0.f;
+          }
+          const float pe = keep ? ex2(fmaf(sv, p.c2, -l2)) : 0.f;
+          e[h] = pe;
+          ds[h] = pe * (dp - dd);
+        }
+        pp[i] = pack_bf16(e[0], e[1]);
+        pd[i] = pack_bf16(ds[0], ds[1]);
+      }
+      if (!kKV) {
+        tmem_st16(tl + b * 128u + 32u * hw, pd);  // dS over this warpgroup's S columns
+      } else {
+        tmem_st16(tl + b * 128u + 32u * hw, pp);        // P^T over its S^T columns
+        tmem_st16(tl + b * 128u + 64u + 32u * hw, pd);  // dS^T over its dP^T columns
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_PF + b));
+
+      if (c.j == c.n - 1) {
+        // ------------------------------------------------------ epilogue --
+        ok = c.t == 0 || wait_bar(bar(B_MD), (c.t - 1) & 1u, p, abort_flag);
+        ok = ok && wait_bar(bar(B_MD), c.t & 1u, p, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
+        const bool row_ok = grow < p.L;
+        const size_t off = (size_t(c.bh) * p.L + (row_ok ? grow : 0)) * D;
+        // Warpgroup hw writes head-dim columns [64 hw, 64 hw + 64) of each output.
+#pragma unroll 1
+        for (int oi = 0; oi < (kKV ? 2 : 1); ++oi) {
+          // dQ pass: gQ = c * C0. dK/dV pass: gK = c * C1, gV = C0.
+          const uint32_t acc_col = !kKV ? TM_C0 : (oi == 0 ? TM_C1 : TM_C0);
+          const float mul = (!kKV || oi == 0) ? p.scale : 1.f;
+          __nv_bfloat16* dst = (!kKV || oi == 0) ? p.out0 : p.out1;
+#pragma unroll 1
+          for (int cc = 0; cc < 2; ++cc) {
+            const uint32_t col = 64u * hw + 32u * cc;
+            uint32_t a[32];
+            tmem_ld32(tl + acc_col + col, a);
+            tmem_wait_ld();
+            uint32_t po[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              po[i] = pack_bf16(__uint_as_float(a[2 * i]) * mul,
+                                __uint_as_float(a[2 * i + 1]) * mul);
+            if (row_ok) {
+              uint4* go = reinterpret_cast<uint4*>(dst + off + col);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                go[i] = make_uint4(po[4 * i], po[4 * i + 1], po[4 * i + 2], po[4 * i + 3]);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(B_CF));
+      }
+      c.next(p, ring, kConsumerWarp);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+static bool make_map(CUtensorMap* m, const void* ptr, int L, int BH, int rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(L), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(L) * D * 2};
+  cuuint32_t box[3] = {64, cuuint32_t(rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool kKV>
+static int launch_pass(const BwdArgs& a, const WorkList& w, int num_sms, unsigned* ctr) {
+  const int BH = a.B * a.H;
+  CUtensorMap m0, m1, mx, my;
+  // dQ pass: stationary Q, G; streamed K, V.  dK/dV: stationary K, V; streamed Q, G.
+  const void* s0 = kKV ? a.k : a.q;
+  const void* s1 = kKV ? a.v : a.g;
+  const void* sx = kKV ? a.q : a.k;
+  const void* sy = kKV ? a.g : a.v;
+  if (!make_map(&m0, s0, a.L, BH, BR) || !make_map(&m1, s1, a.L, BH, BR) ||
+      !make_map(&mx, sx, a.L, BH, BT) || !make_map(&my, sy, a.L, BH, BT))
+    return JVP_ERR_LAUNCH_FAILED;
+  Params p;
+  p.qtiles = w.qtiles;
+  p.segs = w.segs;
+  p.n_entries = w.n_qtiles;
+  p.n_segs = w.n_segs;
+  const long long items = (long long)w.n_qtiles * BH;
+  if (items > 0x7fffffffLL) return JVP_ERR_TOO_LARGE;
+  p.n_items = int(items);
+  p.n_qt = (a.L + BR - 1) / BR;
+  p.n_kt = (a.L + BT - 1) / BT;
+  p.L = a.L;
+  p.mask = a.mask;
+  p.scale = a.scale;
+  p.c2 = a.scale * 1.4426950408889634f;
+  p.lse = a.lse;
+  p.dvec = a.dvec;
+  p.g = static_cast<const __nv_bfloat16*>(a.g);
+  p.o = static_cast<const __nv_bfloat16*>(a.o);
+  p.out0 = static_cast<__nv_bfloat16*>(kKV ? a.gk : a.gq);
+  p.out1 = static_cast<__nv_bfloat16*>(a.gv);
+  p.err = a.err;
+  p.item_ctr = ctr;
+  p.wait_limit_ns = a.wait_limit_ns;
+  static std::mutex attr_mu;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return JVP_ERR_LAUNCH_FAILED;
+  {
+    std::lock_guard<std::mutex> lk(attr_mu);
+    if (!attr_done[dev]) {
+      if (cudaFuncSetAttribute(bwd_kernel<kKV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kSmemBytes) != cudaSuccess)
+        return JVP_ERR_LAUNCH_FAILED;
+      attr_done[dev] = true;
+    }
+  }
+  const int grid = int(items < num_sms ? items : num_sms);
+  if (cudaMemsetAsync(ctr, 0, sizeof(unsigned), a.stream) != cudaSuccess)
+    return JVP_ERR_LAUNCH_FAILED;
+  bwd_kernel<kKV><<<grid, kThreads, kSmemBytes, a.stream>>>(m0, m1, mx, my, p);
+  return cudaGetLastError() == cudaSuccess ? JVP_OK : JVP_ERR_LAUNCH_FAILED;
+}
+
+}  // namespace bwd
+
+int launch_bwd_sm100(const BwdArgs& a, const WorkList& wq, const WorkList& wkv, int num_sms) {
+  if (!a.item_ctr) return JVP_ERR_LAUNCH_FAILED;
+  int rc = bwd::launch_pass<false>(a, wq, num_sms, a.item_ctr);
+  if (rc != JVP_OK) return rc;
+  // The second pass reads D from the first one (stream-ordered) and uses the
+  // second counter word.
+  return bwd::launch_pass<true>(a, wkv, num_sms, a.item_ctr + 1);
+}
+
+}  // namespace jvp

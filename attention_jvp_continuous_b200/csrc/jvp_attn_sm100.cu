@@ -43,6 +43,7 @@
 
 #include "common.cuh"
 #include "mask_rows.cuh"
+#include "sm100_pipeline.cuh"
 #include "sm100_ptx.cuh"
 
 namespace jvp {
@@ -118,133 +119,16 @@ struct Params {
   unsigned long long wait_limit_ns;
 };
 
-// Slow path of wait_bar, kept out of line so that the hot loops stay small.
-__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity,
-                                           unsigned long long limit_ns, unsigned* err,
-                                           volatile uint32_t* abort_flag) {
-  const uint64_t t0 = globaltimer();
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try(bar, parity)) return true;
-    // A try_wait may itself suspend for a while, so the limit is checked
-    // from the first failed poll on.
-    if ((it & 7u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer() - t0 > limit_ns) {
-        atomicOr(err, kErrTimeout);
-        *abort_flag = 1u;
-        return false;
-      }
-    }
-  }
-}
-
-// Bounded wait. Returns false (and raises the CTA abort flag) on timeout or
-// when another role has already aborted.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Params& p,
-                                         volatile uint32_t* abort_flag) {
-  // Most waits find the phase already complete: probe without suspending.
-  if (mbar_test(bar, parity)) return true;
-  return wait_bar_slow(bar, parity, p.wait_limit_ns, p.err, abort_flag);
-}
-
-// Work items reach the roles through a 4-slot ring in shared memory: the
-// producer takes the next item index from the global counter (dynamic
-// longest-first scheduling) and publishes it; the MMA thread's two cursors
-// and the eight softmax warps read it and release the slot.
-enum Role { kProducer, kConsumerThread, kConsumerWarp };
-constexpr uint32_t kRing = 4;
-constexpr uint32_t kRingReaders = 2 + 8;  // MMA S and PV cursors, softmax warps
-
-struct ItemRing {
-  uint32_t full_bar, empty_bar;  // first slot's mbarrier; slots are 8 B apart
-  volatile int* slots;
-  volatile uint32_t* abort_flag;
-};
-
-// Walks this CTA's (item, key tile) sequence; every role runs its own copy.
-struct Cursor {
-  int item, item_idx, bh, qt;
-  int seg, seg_end, kt, kt_end;
-  int j, n;
-  uint32_t t;  // ordinal of the tile among this CTA's tiles
-  bool partial, valid;
-
-  __device__ void load_seg(const Params& p) {
-    const int2 s = p.segs[seg];
-    kt = s.x;
-    kt_end = s.x + (s.y >> 1);
-    partial = (s.y & 1) != 0;
-    if (kt < 0 || kt_end > p.n_kt || kt_end <= kt) {
-      atomicOr(p.err, kErrBounds);
-      valid = false;
-    }
-  }
-  // Index of this CTA's item number item_idx; false on timeout / abort.
-  __device__ bool acquire(const Params& p, const ItemRing& r, Role role) {
-    const uint32_t slot = uint32_t(item_idx) % kRing, use = uint32_t(item_idx) / kRing;
-    if (role == kProducer) {
-      if (use > 0 && !wait_bar(r.empty_bar + 8 * slot, (use - 1) & 1u, p, r.abort_flag))
-        return false;
-      item = int(atomicAdd(p.item_ctr, 1u));
-      r.slots[slot] = item;
-      mbar_arrive(r.full_bar + 8 * slot);  // release: readers see the slot
-      return true;
-    }
-    bool ok = wait_bar(r.full_bar + 8 * slot, use & 1u, p, r.abort_flag);
-    if (role == kConsumerWarp) ok = __all_sync(0xffffffffu, ok);
-    if (!ok) return false;
-    item = r.slots[slot];
-    if (role == kConsumerWarp) {
-      __syncwarp();
-      if ((threadIdx.x & 31) == 0) mbar_arrive(r.empty_bar + 8 * slot);
-    } else {
-      mbar_arrive(r.empty_bar + 8 * slot);
-    }
-    return true;
-  }
-  __device__ void load_item(const Params& p, const ItemRing& r, Role role) {
-    valid = acquire(p, r, role) && item < p.n_items;
-    if (!valid) return;
-    const int e = item % p.n_entries;
-    bh = item / p.n_entries;
-    const int4 en = p.qtiles[e];
-    qt = en.x;
-    seg = en.y;
-    seg_end = en.y + en.z;
-    n = en.w;
-    j = 0;
-    if (qt < 0 || qt >= p.n_qt || seg < 0 || seg_end > p.n_segs || en.z < 1 || n < 1) {
-      atomicOr(p.err, kErrBounds);
-      valid = false;
-      return;
-    }
-    load_seg(p);
-  }
-  __device__ void start(const Params& p, const ItemRing& r, Role role) {
-    item_idx = 0;
-    t = 0;
-    load_item(p, r, role);
-  }
-  __device__ void next(const Params& p, const ItemRing& r, Role role) {
-    ++t;
-    ++j;
-    if (++kt < kt_end) return;
-    if (++seg < seg_end) {
-      load_seg(p);
-      return;
-    }
-    ++item_idx;
-    load_item(p, r, role);
-  }
-};
-
-// Short bounded wait used only while cleaning up after an abort.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try(bar, parity)) {
-    if (globaltimer() - t0 > 100000000ull) return;  // 0.1 s
-  }
-}
+using pipe::wait_bar;
+using pipe::drain_wait;
+using pipe::ItemRing;
+using pipe::Role;
+using pipe::kProducer;
+using pipe::kConsumerThread;
+using pipe::kConsumerWarp;
+using pipe::kRing;
+using pipe::kRingReaders;
+using Cursor = pipe::Cursor<Params>;
 
 __global__ void __launch_bounds__(kThreads, 1)
 jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,

@@ -62,4 +62,46 @@ JVP_HD bool key_ok(const RowKeys& r, int j) {
   return (j >= r.a0 && j < r.b0) || (j >= r.a1 && j < r.b1);
 }
 
+// The transpose: the query rows i whose admissible keys contain key j, again
+// at most two half-open intervals (used by the backward's key/value pass):
+//   DENSE            [0, L)
+//   FRAME/CHUNK      [c0, F*T), c0 = first token of key j's chunk
+//   TEACHER_FORCING  clean key j : clean queries [c0, F*T) and noisy queries
+//                    of later chunks [F*T + c0 + S, 2 F*T)
+//                    noisy key j' = j - F*T, own chunk [c0, c1): noisy
+//                    queries [F*T + c0, F*T + c1)
+// key_ok(row_keys(i), j) == key_ok(key_queries(j), i) for all i, j.
+JVP_HD RowKeys key_queries(int mode, int T, int F, int chunk, int L, int j) {
+  RowKeys r{0, 0, 0, 0};
+  if (j < 0 || j >= L) return r;
+  const int FT = T * F;
+  if (mode == 0) {
+    r.b0 = L;
+    return r;
+  }
+  const int S = (mode == 1 ? 1 : chunk) * T;
+  if (mode == 1 || mode == 2) {
+    r.a0 = (j / S) * S;
+    r.b0 = FT;
+    return r;
+  }
+  if (j < FT) {
+    const int c0 = (j / S) * S;
+    r.a0 = c0;
+    r.b0 = FT;
+    const int n0 = c0 + S;
+    if (n0 < FT) {
+      r.a1 = FT + n0;
+      r.b1 = 2 * FT;
+    }
+    return r;
+  }
+  const int jj = j - FT;
+  const int c0 = (jj / S) * S;
+  const int c1 = (c0 + S < FT) ? c0 + S : FT;
+  r.a0 = FT + c0;
+  r.b0 = FT + c1;
+  return r;
+}
+
 }  // namespace jvp

@@ -193,3 +193,62 @@ bool build_schedule_into(const jvp_mask_desc& m, int L, int bm, int bn, int32_t*
 }
 
 }  // namespace jvp
+
+namespace jvp {
+
+Schedule build_schedule_kv(const jvp_mask_desc& m, int L, int bq, int bk) {
+  Schedule s;
+  s.L = L;
+  s.bm = bq;
+  s.bn = bk;
+  s.n_qt = (L + bq - 1) / bq;
+  s.n_kt = (L + bk - 1) / bk;
+  // Classes on the (bq x bk) grid, then read column by column.
+  std::vector<int8_t> cls(size_t(s.n_qt) * s.n_kt);
+  for (int qt = 0; qt < s.n_qt; ++qt) {
+    int8_t* row = cls.data() + size_t(qt) * s.n_kt;
+    classify_qtile(m, L, bq, bk, qt, row);
+    if ((qt + 1) * bq > L)
+      for (int kt = 0; kt < s.n_kt; ++kt)
+        if (row[kt] == JVP_TILE_FULL) row[kt] = JVP_TILE_PARTIAL;
+  }
+  struct Entry {
+    int kt, seg_begin, seg_count, n_qt;
+  };
+  std::vector<Entry> entries;
+  entries.reserve(s.n_kt);
+  for (int kt = 0; kt < s.n_kt; ++kt) {
+    Entry e{kt, int(s.segs.size() / 2), 0, 0};
+    int qt = 0;
+    while (qt < s.n_qt) {
+      const int8_t c = cls[size_t(qt) * s.n_kt + kt];
+      if (c == JVP_TILE_EMPTY) {
+        ++s.n_empty;
+        ++qt;
+        continue;
+      }
+      int q2 = qt;
+      while (q2 < s.n_qt && cls[size_t(q2) * s.n_kt + kt] == c) ++q2;
+      const int cnt = q2 - qt;
+      s.segs.push_back(qt);
+      s.segs.push_back((cnt << 1) | (c == JVP_TILE_PARTIAL ? 1 : 0));
+      if (c == JVP_TILE_FULL) s.n_full += cnt; else s.n_partial += cnt;
+      e.seg_count += 1;
+      e.n_qt += cnt;
+      qt = q2;
+    }
+    if (e.n_qt > 0) entries.push_back(e);  // a key no query admits has no work
+    s.max_ktiles = std::max<int64_t>(s.max_ktiles, e.n_qt);
+  }
+  std::stable_sort(entries.begin(), entries.end(),
+                   [](const Entry& a, const Entry& b) { return a.n_qt > b.n_qt; });
+  for (const Entry& e : entries) {
+    s.qtiles.push_back(e.kt);
+    s.qtiles.push_back(e.seg_begin);
+    s.qtiles.push_back(e.seg_count);
+    s.qtiles.push_back(e.n_qt);
+  }
+  return s;
+}
+
+}  // namespace jvp

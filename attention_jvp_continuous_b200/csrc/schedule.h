@@ -40,6 +40,14 @@ void classify_qtile(const jvp_mask_desc& m, int L, int bm, int bn, int qt,
 // Builds the full schedule. The mask must already be validated.
 Schedule build_schedule(const jvp_mask_desc& m, int L, int bm, int bn);
 
+// Key-tile-major work list for the backward's key/value pass: one entry per
+// key tile of bk keys, {kt, seg_begin, seg_count, n_qtiles}, longest first,
+// and segments of query tiles of bq rows {qt_begin, (count << 1) | partial}.
+// A tile is FULL only if every (query, key) slot is admitted and neither
+// its queries nor its keys reach past L (query rows past L must be masked
+// here, since the pass reads per-query LSE and D values).
+Schedule build_schedule_kv(const jvp_mask_desc& m, int L, int bq, int bk);
+
 // The same work list as build_schedule (same entries, same order), written
 // into caller-provided arrays without any heap allocation: entries of 4
 // int32 to `qtiles`, segments of 2 int32 ({kt_begin, (count << 1) |

@@ -168,6 +168,32 @@ int jvp_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                          jvp_mask_desc mask, float softmax_scale,
                          void* stream);
 
+/*
+ * jvp_attn_bwd: gradient of sum <G, O> for O = softmax(c QK^T + M) V, the
+ * primal output of jvp_attn_fwd. The consistency loss of the Causal-rCM
+ * report is differentiated through the primal output only (the JVP is taken
+ * at stop-gradient parameters, report Appendix A, around Eq. 26-28), so a
+ * training step pairs jvp_attn_fwd with this backward under the same mask:
+ *
+ *   P = exp(c QK^T - LSE) on admitted pairs,  D_i = <g_i, o_i>,
+ *   dP = G V^T,  dS = P o (dP - D),
+ *   g_q = c dS K,  g_k = c dS^T Q,  g_v = P^T G.
+ *
+ * q, k, v, o, g_o   inputs [B, H, L, d] bf16 (o and lse from jvp_attn_fwd)
+ * lse               input [B, H, L] float32 (natural log)
+ * g_q, g_k, g_v     outputs [B, H, L, d] bf16; every row < L is written
+ * scratch           caller-owned device buffer of B*H*L float32 (receives D)
+ * Supported: JVP_BF16 with d = 128 (two tcgen05 kernels: a query-stationary
+ * pass for g_q and D, then a key-stationary pass for g_k and g_v); other
+ * dtypes give JVP_ERR_INVALID_ARG, other d JVP_ERR_UNSUPPORTED_HEAD_DIM.
+ * Workspace, streams and errors as for jvp_attn_fwd; the key-stationary
+ * work list is cached like the query-stationary one.
+ */
+int jvp_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                 const void* g_o, const float* lse, void* g_q, void* g_k, void* g_v,
+                 float* scratch, int B, int H, int L, int d, jvp_dtype dtype,
+                 jvp_mask_desc mask, float softmax_scale, void* stream);
+
 /* ---- host-side mask / schedule queries (no GPU needed) ------------------- */
 /*
  * jvp_attn_mask_stats: for the mask on L tokens and a bm x bn tile grid
@@ -202,6 +228,19 @@ int jvp_attn_tile_classes(jvp_mask_desc mask, int L, int bm, int bn,
 int jvp_attn_schedule(jvp_mask_desc mask, int L, int bm, int bn,
                       int32_t* qtiles, int qtile_cap, int32_t* segs,
                       int seg_cap, int* n_qtiles, int* n_segs);
+
+/*
+ * jvp_attn_schedule_kv: the key-tile-major work list of jvp_attn_bwd's key
+ * pass, for tests and tools: entries of 4 int32 {key tile, first segment,
+ * segment count, query tiles} (key tiles of bk keys with work, longest
+ * first) and segments of 3 int32 {first query tile, count, partial flag}
+ * over query tiles of bq rows. A tile is full only if all its (query, key)
+ * slots are admitted and it reaches past L in neither direction. Caps and
+ * counts as for jvp_attn_schedule. Host only.
+ */
+int jvp_attn_schedule_kv(jvp_mask_desc mask, int L, int bq, int bk,
+                         int32_t* ktiles, int ktile_cap, int32_t* segs,
+                         int seg_cap, int* n_ktiles, int* n_segs);
 
 /* ---- device error word, workspace, misc ---------------------------------- */
 /*

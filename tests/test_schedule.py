@@ -107,3 +107,27 @@ def test_every_query_tile_has_work():
 def test_schedule_rejects_bad_descriptor():
     with pytest.raises(ja.JvpAttnError):
         ja.mask_stats(ja.Mask(ja.TEACHER_FORCING, 4, 4, 1), L=33)
+
+
+@pytest.mark.parametrize("mode,T,F,ch,bm,bn", CASES[:12])
+def test_key_pass_schedule_is_the_transposed_grid(mode, T, F, ch, bm, bn):
+    # key tiles of bk = bm keys, query tiles of bq = bn rows
+    mk = ja.Mask(mode, T, F, ch)
+    L = mk.length
+    cls = brute_classes(dense(MaskSpec(mode, T, F, ch)), bn, bm)  # [query tile, key tile]
+    nq = cls.shape[0]
+    for qt in range(nq):  # query rows past L must be masked in this pass
+        if (qt + 1) * bn > L:
+            cls[qt][cls[qt] == 1] = 2
+    kt_list, sg = ja.schedule_kv(mk, bq=bn, bk=bm)
+    assert np.all(np.diff(kt_list[:, 3]) <= 0)
+    covered = set()
+    for kt, s0, sc, nqt in kt_list:
+        seen = np.zeros(nq, dtype=np.int8)
+        for qb, cnt, part in sg[s0:s0 + sc]:
+            seen[qb:qb + cnt] = 2 if part else 1
+        np.testing.assert_array_equal(seen, cls[:, kt])
+        assert nqt == int((cls[:, kt] > 0).sum())
+        covered.add(int(kt))
+    # every key tile with an admitted pair has an entry
+    assert covered == {kt for kt in range(cls.shape[1]) if (cls[:, kt] > 0).any()}
