@@ -112,14 +112,17 @@ def attn_bwd(q, k, v, o, g, lse, mask: Mask, scale: Optional[float] = None,
         raise ValueError("lse must be a contiguous float32 CUDA tensor [B, H, L]")
     B, H, L, d = q.shape
     gq, gk, gv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
-    scratch = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    n_scratch = _lib.lib().jvp_attn_bwd_scratch_len(B, H, L)
+    if n_scratch < 0:
+        raise ValueError("invalid shape for jvp_attn_bwd")
+    scratch = torch.empty((n_scratch,), dtype=torch.float32, device=q.device)
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
     fp = ctypes.POINTER(ctypes.c_float)
     rc = _lib.lib().jvp_attn_bwd(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), g.data_ptr(),
         ctypes.cast(lse.data_ptr(), fp), gq.data_ptr(), gk.data_ptr(), gv.data_ptr(),
-        ctypes.cast(scratch.data_ptr(), fp), B, H, L, d, _dtype_code(q), mask.desc(),
+        ctypes.cast(scratch.data_ptr(), fp), n_scratch, B, H, L, d, _dtype_code(q), mask.desc(),
         0.0 if scale is None else float(scale), ctypes.c_void_p(stream))
     _lib.check(rc, "jvp_attn_bwd")
     return gq, gk, gv

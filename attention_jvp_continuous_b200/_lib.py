@@ -32,7 +32,8 @@ JVP_FP32 = 1
 TILE_EMPTY, TILE_FULL, TILE_PARTIAL = 0, 1, 2
 
 # Exported functions, as declared in include/jvp_attn.h.
-EXPORTS = ("jvp_attn_fwd", "jvp_attn_fwd_noalloc", "jvp_attn_bwd", "jvp_attn_mask_stats",
+EXPORTS = ("jvp_attn_fwd", "jvp_attn_fwd_noalloc", "jvp_attn_bwd", "jvp_attn_bwd_scratch_len",
+           "jvp_attn_mask_stats",
            "jvp_attn_tile_classes", "jvp_attn_schedule", "jvp_attn_schedule_kv",
            "jvp_attn_check_device_error",
            "jvp_attn_set_wait_limit", "jvp_attn_release", "jvp_attn_strerror",
@@ -76,9 +77,11 @@ def lib() -> ctypes.CDLL:
         L.jvp_attn_fwd_noalloc.argtypes = L.jvp_attn_fwd.argtypes
         L.jvp_attn_fwd_noalloc.restype = i32
         fp = ctypes.POINTER(ctypes.c_float)
-        L.jvp_attn_bwd.argtypes = [vp] * 5 + [fp] + [vp] * 3 + [fp] + [i32] * 5 + \
-            [MaskDesc, ctypes.c_float, vp]
+        L.jvp_attn_bwd.argtypes = [vp] * 5 + [fp] + [vp] * 3 + [fp, ctypes.c_int64] + \
+            [i32] * 5 + [MaskDesc, ctypes.c_float, vp]
         L.jvp_attn_bwd.restype = i32
+        L.jvp_attn_bwd_scratch_len.argtypes = [i32, i32, i32]
+        L.jvp_attn_bwd_scratch_len.restype = ctypes.c_int64
         L.jvp_attn_mask_stats.argtypes = [MaskDesc, i32, i32, i32, i64p, i64p, i64p, i64p]
         L.jvp_attn_mask_stats.restype = i32
         L.jvp_attn_tile_classes.argtypes = [MaskDesc, i32, i32, i32,

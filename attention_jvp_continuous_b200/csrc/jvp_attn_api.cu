@@ -198,9 +198,9 @@ int jvp_attn_fwd(const void* q, const void* k, const void* v, const void* dq, co
 }
 
 int jvp_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* g_o,
-                 const float* lse, void* g_q, void* g_k, void* g_v, float* scratch, int B, int H,
-                 int L, int d, jvp_dtype dtype, jvp_mask_desc mask, float softmax_scale,
-                 void* stream) {
+                 const float* lse, void* g_q, void* g_k, void* g_v, float* scratch,
+                 int64_t scratch_len, int B, int H, int L, int d, jvp_dtype dtype,
+                 jvp_mask_desc mask, float softmax_scale, void* stream) {
   if (!q || !k || !v || !o || !g_o || !lse || !g_q || !g_k || !g_v || !scratch)
     return JVP_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || dtype != JVP_BF16) return JVP_ERR_INVALID_ARG;
@@ -210,6 +210,7 @@ int jvp_attn_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (rc != JVP_OK) return rc;
   if ((long long)B * H * L >= (1LL << 31) || (long long)B * H >= (1LL << 31) / 2)
     return JVP_ERR_TOO_LARGE;
+  if (scratch_len < jvp_attn_bwd_scratch_len(B, H, L)) return JVP_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, o, g_o, lse, g_q, g_k, g_v, scratch};
   for (const void* p : ptrs)
     if (!aligned16(p)) return JVP_ERR_MISALIGNED;
@@ -221,7 +222,7 @@ int jvp_attn_bwd(const void* q, const void* k, const void* v, const void* o, con
   cudaGetDevice(&dev);
   BwdArgs a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.g = g_o; a.lse = lse;
-  a.gq = g_q; a.gk = g_k; a.gv = g_v; a.dvec = scratch;
+  a.gq = g_q; a.gk = g_k; a.gv = g_v; a.scratch = scratch;
   a.B = B; a.H = H; a.L = L; a.d = d;
   a.mask = mask;
   a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(d));
@@ -236,6 +237,12 @@ int jvp_attn_bwd(const void* q, const void* k, const void* v, const void* o, con
   rc = get_counter(dev, a.stream, &a.item_ctr);
   if (rc != JVP_OK) return rc;
   return launch_bwd_sm100(a, wq, wkv, di->sms);
+}
+
+int64_t jvp_attn_bwd_scratch_len(int B, int H, int L) {
+  if (B <= 0 || H <= 0 || L <= 0) return -1;
+  const int64_t Lp = (int64_t(L) + 127) / 128 * 128;
+  return 2 * int64_t(B) * H * Lp;
 }
 
 int jvp_attn_schedule_kv(jvp_mask_desc mask, int L, int bq, int bk, int32_t* ktiles,

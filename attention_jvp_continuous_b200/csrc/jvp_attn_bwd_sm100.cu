@@ -52,35 +52,45 @@ constexpr uint32_t kRHalf = BR * 128;  // 16 KB: 128 rows x 64 head-dim columns
 constexpr uint32_t kTHalf = BT * 128;  //  8 KB: 64 rows x 64 columns
 constexpr uint32_t kTile = 2 * kTHalf; // 16 KB: one streamed 64-row operand
 
-// Shared memory: two stationary operands (A0, A1), then streamed operands
-// in rings: ring X with 3 stages, ring Y with 2 or 3 stages.
-constexpr uint32_t SM_A0 = 0;
-constexpr uint32_t SM_A1 = 2 * kRHalf;
-constexpr uint32_t SM_X = 4 * kRHalf;         // 3 stages of kTile
-constexpr uint32_t SM_Y = SM_X + 3 * kTile;   // 3 stages of kTile
-constexpr uint32_t SM_BAR = SM_Y + 3 * kTile; // 160 KB
-constexpr uint32_t kSmemBytes = SM_BAR + 512 + 1024;
+// Shared memory: two stationary operands (A0, A1), then the streamed
+// operands in two rings X and Y. A streamed tile that feeds both the first
+// and the accumulating MMAs of a tile stays resident across two tiles (the
+// MMA order is S(t+1) before acc(t)), so such a ring needs 5 stages to keep
+// two loads in flight; V in the dQ pass feeds dP only and needs 4.
+template <bool kKV>
+struct Layout {
+  static constexpr uint32_t NX = 5;            // dQ: K    dK/dV: Q
+  static constexpr uint32_t NY = kKV ? 5 : 4;  // dQ: V    dK/dV: G
+  static constexpr uint32_t A0 = 0;
+  static constexpr uint32_t A1 = 2 * kRHalf;
+  static constexpr uint32_t X = 4 * kRHalf;
+  static constexpr uint32_t Y = X + NX * kTile;
+  static constexpr uint32_t BAR = Y + NY * kTile;  // 208 KB (dQ) / 224 KB (dK/dV)
+  static constexpr uint32_t TMEM_SLOT = BAR + 8 * 40;
+  static constexpr uint32_t ABORT = TMEM_SLOT + 4;
+  static constexpr uint32_t RING = ABORT + 4;
+  static constexpr uint32_t kBytes = BAR + 512 + 1024;  // + alignment slack
+};
+static_assert(Layout<true>::kBytes <= 232448, "shared memory over the per-block limit");
 
 enum : uint32_t {
   B_AF = 0,      // stationary operands landed
   B_AE = 1,      // stationary operands may be overwritten
-  B_XF = 2,      // 3
-  B_XE = 5,      // 3
-  B_YF = 8,      // 3
-  B_YE = 11,     // 3
-  B_SF = 14,     // 2: S / dP buffer ready
-  B_PF = 16,     // 2: bf16 operands written by the softmax warps
-  B_MD = 18,     // accumulating MMA of a tile done
-  B_CF = 19,     // accumulators read by the epilogue
-  B_DRAIN = 20,
-  B_IF = 21,     // 4: work-item ring
-  B_IE = 25,     // 4
-  kNumBars = 29
+  B_XF = 2,      // 5
+  B_XE = 7,      // 5
+  B_YF = 12,     // 5
+  B_YE = 17,     // 5
+  B_SF = 22,     // 2: S / dP buffer ready
+  B_PF = 24,     // 2: bf16 operands written by the softmax warps
+  B_MD = 26,     // accumulating MMA of a tile done
+  B_CF = 27,     // accumulators read by the epilogue
+  B_DRAIN = 28,
+  B_IF = 29,     // 4: work-item ring
+  B_IE = 33,     // 4
+  kNumBars = 37
 };
-constexpr uint32_t SM_TMEM_SLOT = SM_BAR + 8 * kNumBars;
-constexpr uint32_t SM_ABORT = SM_TMEM_SLOT + 4;
-constexpr uint32_t SM_RING = SM_ABORT + 4;
-static_assert(SM_RING + 16 <= SM_BAR + 512, "barrier area overflow");
+static_assert(kNumBars <= 40, "barrier slots");
+static_assert(Layout<false>::RING + 16 <= Layout<false>::BAR + 512, "barrier area overflow");
 
 constexpr uint32_t TM_C0 = 256;  // first accumulator (gQ, or gV)
 constexpr uint32_t TM_C1 = 384;  // second accumulator (gK)
@@ -94,9 +104,11 @@ struct Params {
   int n_entries, n_segs, n_items, n_qt, n_kt;  // n_qt: outer tiles, n_kt: inner tiles
   int L;
   jvp_mask_desc mask;
+  int Lp;  // L rounded up to whole 128-row tiles: row stride of the scratch
   float scale, c2;
   const float* lse;     // forward LSE (natural log)
-  float* dvec;          // D_i = <g_i, o_i>: written by the dQ pass, read by the dK/dV pass
+  float2* sd;           // scratch [B*H, Lp] of {LSE * log2(e), D_i = <g_i, o_i>}: written
+                        // by the dQ pass (rows past L: {+inf, 0}), read by the dK/dV pass
   const __nv_bfloat16* g;  // cotangent, for D (dQ pass)
   const __nv_bfloat16* o;  // forward output, for D (dQ pass)
   __nv_bfloat16* out0;     // gQ (dQ pass) or gK (dK/dV pass)
@@ -117,21 +129,25 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
            const __grid_constant__ Params p) {
   // dQ pass:  A0 = Q, A1 = G (stationary);  X = K (3 stages), Y = V.
   // dK/dV:    A0 = K, A1 = V (stationary);  X = Q (3 stages), Y = G.
+  using LY = Layout<kKV>;
+  constexpr uint32_t NX = LY::NX, NY = LY::NY;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* const base_ptr = smem_raw + (base - raw);
-  auto bar = [&](uint32_t slot) { return base + SM_BAR + 8u * slot; };
-  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + SM_ABORT);
+  auto bar = [&](uint32_t slot) { return base + LY::BAR + 8u * slot; };
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + LY::ABORT);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_AF), 1);
     mbar_init(bar(B_AE), 1);
-    for (int s = 0; s < 3; ++s) {
+    for (uint32_t s = 0; s < NX; ++s) {
       mbar_init(bar(B_XF + s), 1);
       mbar_init(bar(B_XE + s), 1);
+    }
+    for (uint32_t s = 0; s < NY; ++s) {
       mbar_init(bar(B_YF + s), 1);
       mbar_init(bar(B_YE + s), 1);
     }
@@ -156,15 +172,15 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
     tma_prefetch_map(&tm_y);
   }
   if (warp == 1) {
-    tmem_alloc(base + SM_TMEM_SLOT, 512);
+    tmem_alloc(base + LY::TMEM_SLOT, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base_ptr + SM_TMEM_SLOT);
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base_ptr + LY::TMEM_SLOT);
   const ItemRing ring{bar(B_IF), bar(B_IE),
-                      reinterpret_cast<volatile int*>(base_ptr + SM_RING), abort_flag};
+                      reinterpret_cast<volatile int*>(base_ptr + LY::RING), abort_flag};
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA ----
@@ -180,33 +196,37 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
           mbar_expect_tx(bar(B_AF), 4 * kRHalf);
           ++a_armed;
           const int y = c.qt * BR;
-          tma_load_3d(base + SM_A0, &tm_a0, bar(B_AF), 0, y, c.bh);
-          tma_load_3d(base + SM_A0 + kRHalf, &tm_a0, bar(B_AF), 64, y, c.bh);
-          tma_load_3d(base + SM_A1, &tm_a1, bar(B_AF), 0, y, c.bh);
-          tma_load_3d(base + SM_A1 + kRHalf, &tm_a1, bar(B_AF), 64, y, c.bh);
+          tma_load_3d(base + LY::A0, &tm_a0, bar(B_AF), 0, y, c.bh);
+          tma_load_3d(base + LY::A0 + kRHalf, &tm_a0, bar(B_AF), 64, y, c.bh);
+          tma_load_3d(base + LY::A1, &tm_a1, bar(B_AF), 0, y, c.bh);
+          tma_load_3d(base + LY::A1 + kRHalf, &tm_a1, bar(B_AF), 64, y, c.bh);
         }
         const int y = c.kt * BT;
-        const uint32_t sx = c.t % 3, ux = c.t / 3;
-        if (c.t >= 3) ok = wait_bar(bar(B_XE + sx), (ux - 1) & 1u, p, abort_flag);
+        const uint32_t sx = c.t % NX, ux = c.t / NX;
+        if (c.t >= NX) ok = wait_bar(bar(B_XE + sx), (ux - 1) & 1u, p, abort_flag);
         if (!ok) break;
         mbar_expect_tx(bar(B_XF + sx), kTile);
         ++x_issued;
-        tma_load_3d(base + SM_X + sx * kTile, &tm_x, bar(B_XF + sx), 0, y, c.bh);
-        tma_load_3d(base + SM_X + sx * kTile + kTHalf, &tm_x, bar(B_XF + sx), 64, y, c.bh);
-        const uint32_t sy = c.t % 3, uy = c.t / 3;
-        if (c.t >= 3) ok = wait_bar(bar(B_YE + sy), (uy - 1) & 1u, p, abort_flag);
+        tma_load_3d(base + LY::X + sx * kTile, &tm_x, bar(B_XF + sx), 0, y, c.bh);
+        tma_load_3d(base + LY::X + sx * kTile + kTHalf, &tm_x, bar(B_XF + sx), 64, y, c.bh);
+        const uint32_t sy = c.t % NY, uy = c.t / NY;
+        if (c.t >= NY) ok = wait_bar(bar(B_YE + sy), (uy - 1) & 1u, p, abort_flag);
         if (!ok) break;
         mbar_expect_tx(bar(B_YF + sy), kTile);
         ++y_issued;
-        tma_load_3d(base + SM_Y + sy * kTile, &tm_y, bar(B_YF + sy), 0, y, c.bh);
-        tma_load_3d(base + SM_Y + sy * kTile + kTHalf, &tm_y, bar(B_YF + sy), 64, y, c.bh);
+        tma_load_3d(base + LY::Y + sy * kTile, &tm_y, bar(B_YF + sy), 0, y, c.bh);
+        tma_load_3d(base + LY::Y + sy * kTile + kTHalf, &tm_y, bar(B_YF + sy), 64, y, c.bh);
         c.next(p, ring, kProducer);
       }
       if (!ok || *abort_flag) {
         if (a_armed) drain_wait(bar(B_AF), (a_armed - 1) & 1u);
-        for (uint32_t s = 0; s < 3; ++s) {
-          const uint32_t nx = (x_issued + 2 - s) / 3, ny = (y_issued + 2 - s) / 3;
+        // Stage s received ceil((issued - s) / N) loads; wait for the last.
+        for (uint32_t s = 0; s < NX; ++s) {
+          const uint32_t nx = (x_issued + NX - 1 - s) / NX;
           if (nx) drain_wait(bar(B_XF + s), (nx - 1) & 1u);
+        }
+        for (uint32_t s = 0; s < NY; ++s) {
+          const uint32_t ny = (y_issued + NY - 1 - s) / NY;
           if (ny) drain_wait(bar(B_YF + s), (ny - 1) & 1u);
         }
       }
@@ -216,18 +236,18 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
     // ------------------------------------------------------------ MMA ----
     if (lane == 0) {
       bool ok = true;
-      const uint64_t a0_desc = sdesc_sw128(base + SM_A0, 16, 1024);
-      const uint64_t a1_desc = sdesc_sw128(base + SM_A1, 16, 1024);
-      const uint64_t xk_desc = sdesc_sw128(base + SM_X, 16, 1024);       // K-major view
-      const uint64_t xm_desc = sdesc_sw128(base + SM_X, kTHalf, 1024);   // MN-major view
-      const uint64_t yk_desc = sdesc_sw128(base + SM_Y, 16, 1024);
-      const uint64_t ym_desc = sdesc_sw128(base + SM_Y, kTHalf, 1024);
+      const uint64_t a0_desc = sdesc_sw128(base + LY::A0, 16, 1024);
+      const uint64_t a1_desc = sdesc_sw128(base + LY::A1, 16, 1024);
+      const uint64_t xk_desc = sdesc_sw128(base + LY::X, 16, 1024);       // K-major view
+      const uint64_t xm_desc = sdesc_sw128(base + LY::X, kTHalf, 1024);   // MN-major view
+      const uint64_t yk_desc = sdesc_sw128(base + LY::Y, 16, 1024);
+      const uint64_t ym_desc = sdesc_sw128(base + LY::Y, kTHalf, 1024);
       // First MMAs of a tile: T0 = A0 X^T into S, T1 = A1 Y^T into dP.
       auto issue_s = [&](const Cursor& c) -> bool {
-        const uint32_t b = c.t & 1u, sx = c.t % 3, sy = c.t % 3;
+        const uint32_t b = c.t & 1u, sx = c.t % NX, sy = c.t % NY;
         if (c.j == 0 && !wait_bar(bar(B_AF), c.item_idx & 1, p, abort_flag)) return false;
-        if (!wait_bar(bar(B_XF + sx), (c.t / 3) & 1u, p, abort_flag)) return false;
-        if (!wait_bar(bar(B_YF + sy), (c.t / 3) & 1u, p, abort_flag)) return false;
+        if (!wait_bar(bar(B_XF + sx), (c.t / NX) & 1u, p, abort_flag)) return false;
+        if (!wait_bar(bar(B_YF + sy), (c.t / NY) & 1u, p, abort_flag)) return false;
         tc_fence_after();
         const uint32_t d_s = tmem + b * 128u, d_p = d_s + 64u;
         const uint64_t xb = xk_desc + sx * (kTile >> 4), yb = yk_desc + sy * (kTile >> 4);
@@ -251,7 +271,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       // Accumulating MMAs. The bf16 operands of a tile sit in TMEM columns
       // {0, 8} and {32, 40} (one pair of 16-wide k-steps per warpgroup).
       auto issue_acc = [&](const Cursor& c) -> bool {
-        const uint32_t b = c.t & 1u, sx = c.t % 3, sy = c.t % 3;
+        const uint32_t b = c.t & 1u, sx = c.t % NX, sy = c.t % NY;
         if (c.j == 0 && c.item_idx > 0 &&
             !wait_bar(bar(B_CF), (c.item_idx - 1) & 1, p, abort_flag))
           return false;
@@ -313,19 +333,20 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
     c.start(p, ring, kConsumerWarp);
     RowKeys rk{0, 0, 0, 0};
     int grow = 0;
-    float lse2 = 0.f, dval = 0.f;  // dQ pass: this row's LSE (log2) and D
+    // dQ pass: this row's LSE (log2, +inf past L so that P = 0 there) and D.
+    float lse2 = 0.f, dval = 0.f;
     bool ok = true;
     while (c.valid) {
       if (c.j == 0) {
         grow = c.qt * BR + r;
         if (!kKV) {
           rk = row_keys(p.mask.mode, p.mask.tokens_per_frame, p.mask.n_frames, chunk, p.L, grow);
-          lse2 = -CUDART_INF_F;
+          lse2 = CUDART_INF_F;
           dval = 0.f;
+          const size_t roff = size_t(c.bh) * p.L + grow;
           if (grow < p.L) {
-            const size_t roff = size_t(c.bh) * p.L + grow;
             const float l = p.lse[roff];
-            lse2 = l * kLog2e;
+            if (l != -CUDART_INF_F) lse2 = l * kLog2e;
             // D = <g, o> for this row, both 128-wide rows read as 16 B vectors.
             const uint4* gr = reinterpret_cast<const uint4*>(p.g + roff * D);
             const uint4* orow = reinterpret_cast<const uint4*>(p.o + roff * D);
@@ -342,12 +363,25 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
               }
             }
             dval = acc;
-            if (hw == 0) p.dvec[roff] = dval;
           }
+          // grow < Lp always: the last query tile covers the padding rows.
+          if (hw == 0) p.sd[size_t(c.bh) * p.Lp + grow] = make_float2(lse2, dval);
         } else {
           rk = key_queries(p.mask.mode, p.mask.tokens_per_frame, p.mask.n_frames, chunk, p.L,
                            grow);
         }
+      }
+      // Column indices of this thread's 32 elements: keys (dQ pass) or
+      // queries (dK/dV pass) [col0, col0 + 32).
+      const int col0 = c.kt * BT + 32 * hw;
+      // dK/dV pass: {LSE2, D} of the 32 queries, the same for every lane
+      // (col0 + 32 <= Lp, 16-byte aligned since col0 and Lp are even).
+      float4 w[16];
+      if (kKV) {
+        const float4* src =
+            reinterpret_cast<const float4*>(p.sd + size_t(c.bh) * p.Lp + col0);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = __ldg(src + i);
       }
       const uint32_t b = c.t & 1u;
       ok = wait_bar(bar(B_SF + b), (c.t >> 1) & 1u, p, abort_flag);
@@ -357,36 +391,38 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       tmem_ld32(tl + b * 128u + 32u * hw, sr);
       tmem_ld32(tl + b * 128u + 64u + 32u * hw, dr);
       tmem_wait_ld();
-      // Column indices of this thread's 32 elements: keys (dQ pass) or
-      // queries (dK/dV pass) [col0, col0 + 32).
-      const int col0 = c.kt * BT + 32 * hw;
       uint32_t pp[16], pd[16];
+      // Element (2i + h): P = 2^(c2 S - LSE2), dS = P (dP - D); zero where
+      // the mask excludes the pair (only partial tiles test it).
+      auto elem = [&](int i, int h, bool masked, float& e, float& ds) {
+        const float sv = __uint_as_float(sr[2 * i + h]);
+        const float dp = __uint_as_float(dr[2 * i + h]);
+        const float l2 = kKV ? (h ? w[i].z : w[i].x) : lse2;
+        const float dd = kKV ? (h ? w[i].w : w[i].y) : dval;
+        const float pe = ex2(fmaf(sv, p.c2, -l2));
+        const float dsv = pe * (dp - dd);
+        const bool keep = !masked || key_ok(rk, col0 + 2 * i + h);
+        e = keep ? pe : 0.f;
+        ds = keep ? dsv : 0.f;
+      };
+      if (c.partial) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float e[2], ds[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int ci = col0 + 2 * i + h;
-          const float sv = __uint_as_float(sr[2 * i + h]);
-          const float dp = __uint_as_float(dr[2 * i + h]);
-          float l2, dd;
-          bool keep = !c.partial || key_ok(rk, ci);
-          if (!kKV) {
-            l2 = lse2;
-            dd = dval;
-            keep = keep && lse2 != -CUDART_INF_F;
-          } else {
-            // Per-query LSE and D: the same address for all lanes (broadcast).
-            const size_t qoff = size_t(c.bh) * p.L + (keep ? ci : 0);
-            l2 = keep ? __ldg(p.lse + qoff) * kLog2e : 0.f;
-            dd = keep ? __ldg(p.dvec + qoff) : 0.f;
-          }
-          const float pe = keep ? ex2(fmaf(sv, p.c2, -l2)) : 0.f;
-          e[h] = pe;
-          ds[h] = pe * (dp - dd);
+        for (int i = 0; i < 16; ++i) {
+          float e0, e1, d0, d1;
+          elem(i, 0, true, e0, d0);
+          elem(i, 1, true, e1, d1);
+          pp[i] = pack_bf16(e0, e1);
+          pd[i] = pack_bf16(d0, d1);
         }
-        pp[i] = pack_bf16(e[0], e[1]);
-        pd[i] = pack_bf16(ds[0], ds[1]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float e0, e1, d0, d1;
+          elem(i, 0, false, e0, d0);
+          elem(i, 1, false, e1, d1);
+          pp[i] = pack_bf16(e0, e1);
+          pd[i] = pack_bf16(d0, d1);
+        }
       }
       if (!kKV) {
         tmem_st16(tl + b * 128u + 32u * hw, pd);  // dS over this warpgroup's S columns
@@ -501,7 +537,8 @@ static int launch_pass(const BwdArgs& a, const WorkList& w, int num_sms, unsigne
   p.scale = a.scale;
   p.c2 = a.scale * 1.4426950408889634f;
   p.lse = a.lse;
-  p.dvec = a.dvec;
+  p.Lp = (a.L + 127) / 128 * 128;
+  p.sd = reinterpret_cast<float2*>(a.scratch);
   p.g = static_cast<const __nv_bfloat16*>(a.g);
   p.o = static_cast<const __nv_bfloat16*>(a.o);
   p.out0 = static_cast<__nv_bfloat16*>(kKV ? a.gk : a.gq);
@@ -517,7 +554,7 @@ static int launch_pass(const BwdArgs& a, const WorkList& w, int num_sms, unsigne
     std::lock_guard<std::mutex> lk(attr_mu);
     if (!attr_done[dev]) {
       if (cudaFuncSetAttribute(bwd_kernel<kKV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kSmemBytes) != cudaSuccess)
+                               Layout<kKV>::kBytes) != cudaSuccess)
         return JVP_ERR_LAUNCH_FAILED;
       attr_done[dev] = true;
     }
@@ -525,7 +562,7 @@ static int launch_pass(const BwdArgs& a, const WorkList& w, int num_sms, unsigne
   const int grid = int(items < num_sms ? items : num_sms);
   if (cudaMemsetAsync(ctr, 0, sizeof(unsigned), a.stream) != cudaSuccess)
     return JVP_ERR_LAUNCH_FAILED;
-  bwd_kernel<kKV><<<grid, kThreads, kSmemBytes, a.stream>>>(m0, m1, mx, my, p);
+  bwd_kernel<kKV><<<grid, kThreads, Layout<kKV>::kBytes, a.stream>>>(m0, m1, mx, my, p);
   return cudaGetLastError() == cudaSuccess ? JVP_OK : JVP_ERR_LAUNCH_FAILED;
 }
 

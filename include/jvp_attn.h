@@ -182,7 +182,11 @@ int jvp_attn_fwd_noalloc(const void* q, const void* k, const void* v,
  * q, k, v, o, g_o   inputs [B, H, L, d] bf16 (o and lse from jvp_attn_fwd)
  * lse               input [B, H, L] float32 (natural log)
  * g_q, g_k, g_v     outputs [B, H, L, d] bf16; every row < L is written
- * scratch           caller-owned device buffer of B*H*L float32 (receives D)
+ * scratch           caller-owned device buffer of scratch_len float32, at
+ *                   least jvp_attn_bwd_scratch_len(B, H, L) (else
+ *                   JVP_ERR_INVALID_ARG); the first pass writes per-row
+ *                   softmax statistics there for the second; contents on
+ *                   entry are ignored and on return unspecified
  * Supported: JVP_BF16 with d = 128 (two tcgen05 kernels: a query-stationary
  * pass for g_q and D, then a key-stationary pass for g_k and g_v); other
  * dtypes give JVP_ERR_INVALID_ARG, other d JVP_ERR_UNSUPPORTED_HEAD_DIM.
@@ -191,8 +195,14 @@ int jvp_attn_fwd_noalloc(const void* q, const void* k, const void* v,
  */
 int jvp_attn_bwd(const void* q, const void* k, const void* v, const void* o,
                  const void* g_o, const float* lse, void* g_q, void* g_k, void* g_v,
-                 float* scratch, int B, int H, int L, int d, jvp_dtype dtype,
-                 jvp_mask_desc mask, float softmax_scale, void* stream);
+                 float* scratch, int64_t scratch_len, int B, int H, int L, int d,
+                 jvp_dtype dtype, jvp_mask_desc mask, float softmax_scale, void* stream);
+
+/*
+ * jvp_attn_bwd_scratch_len: float32 elements of scratch jvp_attn_bwd needs,
+ * 2 * B * H * ceil(L / 128) * 128; -1 if B, H or L is not positive. Host only.
+ */
+int64_t jvp_attn_bwd_scratch_len(int B, int H, int L);
 
 /* ---- host-side mask / schedule queries (no GPU needed) ------------------- */
 /*
