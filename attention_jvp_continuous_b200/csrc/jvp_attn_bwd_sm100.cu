@@ -6,18 +6,20 @@
 //
 // Two persistent tcgen05 kernels over the same admissible-tile work lists:
 //  * dQ pass (query-stationary, 128 query rows per item, 64-key tiles):
-//      S = Q K^T, dP = G V^T   (SS MMAs, N = 64, fp32 in TMEM)
+//      S = Q K^T, dP = G V^T   (N = 64; Q and G rows held in TMEM as the
+//                               A operands, K and V tiles from shared memory)
 //      softmax warps: P, dS    (one row per thread, bf16 dS back to TMEM)
-//      gQ += dS K              (TS MMA, N = 128, accumulator in TMEM)
-//    and it writes D_i to a scratch vector for the second pass.
+//      gQ += dS K              (A = dS in TMEM, N = 128, accumulator in TMEM)
+//    and it writes {LSE, D_i} per row to a scratch vector for the second pass.
 //  * dK/dV pass (key-stationary, 128 keys per item, 64-query tiles):
-//      S^T = K Q^T, dP^T = V G^T
+//      S^T = K Q^T, dP^T = V G^T (both operands in shared memory: TMEM holds
+//                               the two accumulators and the S/dP buffers)
 //      softmax warps: P^T, dS^T (one key per thread; per-query LSE and D)
-//      gV += P^T G, gK += dS^T Q (TS MMAs, N = 128)
-// Warp roles as in the JVP kernel: warp 0 TMA, warp 1 MMA issue (one
-// thread), warps 4-11 two warpgroups taking 32 of each tile's 64 columns.
-// Each warpgroup writes its bf16 operands into the TMEM columns it has just
-// read itself, so no exchange between the warpgroups is needed.
+//      gV += P^T G, gK += dS^T Q (A in TMEM, N = 128)
+// Warp roles: warp 0 TMA, warps 1 and 2 issue MMAs (one thread each),
+// warps 4-11 two warpgroups taking 32 of each tile's 64 columns. Each
+// warpgroup writes its bf16 operands into the TMEM columns it has just read
+// itself, so no exchange between the warpgroups is needed.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -40,7 +42,6 @@ using pipe::kConsumerThread;
 using pipe::kConsumerWarp;
 using pipe::kProducer;
 using pipe::kRing;
-using pipe::kRingReaders;
 using pipe::wait_bar;
 
 constexpr int BR = 128;  // stationary rows per item (TMEM lanes)
@@ -51,21 +52,24 @@ constexpr int kThreads = 384;
 constexpr uint32_t kRHalf = BR * 128;  // 16 KB: 128 rows x 64 head-dim columns
 constexpr uint32_t kTHalf = BT * 128;  //  8 KB: 64 rows x 64 columns
 constexpr uint32_t kTile = 2 * kTHalf; // 16 KB: one streamed 64-row operand
+// Readers of the work-item ring: issuer A, issuer B's two cursors, 8 softmax warps.
+constexpr uint32_t kReaders = 3 + 8;
 
-// Shared memory: two stationary operands (A0, A1), then the streamed
-// operands in two rings X and Y. A streamed tile that feeds both the first
-// and the accumulating MMAs of a tile stays resident across two tiles (the
-// MMA order is S(t+1) before acc(t)), so such a ring needs 5 stages to keep
-// two loads in flight; V in the dQ pass feeds dP only and needs 4.
+// Shared memory: the dK/dV pass's two stationary operands (A0, A1; the dQ
+// pass keeps its stationary Q and G in TMEM), then the streamed operands in
+// two rings X and Y. A streamed tile that feeds both the first and the
+// accumulating MMAs of a tile stays resident across two tiles (S(t+1) is
+// issued before acc(t)), so such a ring has 5 stages to keep two loads in
+// flight; V in the dQ pass feeds dP only and has 4.
 template <bool kKV>
 struct Layout {
   static constexpr uint32_t NX = 5;            // dQ: K    dK/dV: Q
   static constexpr uint32_t NY = kKV ? 5 : 4;  // dQ: V    dK/dV: G
   static constexpr uint32_t A0 = 0;
-  static constexpr uint32_t A1 = 2 * kRHalf;
-  static constexpr uint32_t X = 4 * kRHalf;
+  static constexpr uint32_t A1 = kKV ? 2 * kRHalf : 0;
+  static constexpr uint32_t X = kKV ? 4 * kRHalf : 0;
   static constexpr uint32_t Y = X + NX * kTile;
-  static constexpr uint32_t BAR = Y + NY * kTile;  // 208 KB (dQ) / 224 KB (dK/dV)
+  static constexpr uint32_t BAR = Y + NY * kTile;  // 144 KB (dQ) / 224 KB (dK/dV)
   static constexpr uint32_t TMEM_SLOT = BAR + 8 * 40;
   static constexpr uint32_t ABORT = TMEM_SLOT + 4;
   static constexpr uint32_t RING = ABORT + 4;
@@ -74,26 +78,31 @@ struct Layout {
 static_assert(Layout<true>::kBytes <= 232448, "shared memory over the per-block limit");
 
 enum : uint32_t {
-  B_AF = 0,      // stationary operands landed
-  B_AE = 1,      // stationary operands may be overwritten
+  B_AF = 0,      // stationary operands ready (TMA bytes, or TMEM rows stored)
+  B_AE = 1,      // dK/dV: stationary smem operands may be overwritten (2 issuers)
   B_XF = 2,      // 5
   B_XE = 7,      // 5
   B_YF = 12,     // 5
   B_YE = 17,     // 5
-  B_SF = 22,     // 2: S / dP buffer ready
+  B_SF = 22,     // 2: S and dP of a buffer complete (one commit per issuer)
   B_PF = 24,     // 2: bf16 operands written by the softmax warps
-  B_MD = 26,     // accumulating MMA of a tile done
-  B_CF = 27,     // accumulators read by the epilogue
-  B_DRAIN = 28,
-  B_IF = 29,     // 4: work-item ring
-  B_IE = 33,     // 4
-  kNumBars = 37
+  B_MD = 26,     // 2: accumulating MMAs of the buffer's last tile complete
+  B_CF = 28,     // accumulators read by the epilogue
+  B_DRAIN = 29,  // 2: one per issuer
+  B_IF = 31,     // 4: work-item ring
+  B_IE = 35,     // 4
+  kNumBars = 39
 };
 static_assert(kNumBars <= 40, "barrier slots");
 static_assert(Layout<false>::RING + 16 <= Layout<false>::BAR + 512, "barrier area overflow");
 
-constexpr uint32_t TM_C0 = 256;  // first accumulator (gQ, or gV)
-constexpr uint32_t TM_C1 = 384;  // second accumulator (gK)
+// TMEM columns: S/dP double buffer [0, 256) (buffer b at 128 b: S or S^T at
+// +0, dP or dP^T at +64), accumulators C0 and C1, and in the dQ pass the
+// stationary bf16 Q and G rows (A operands of the first MMAs) in place of C1.
+constexpr uint32_t TM_C0 = 256;  // gQ, or gV
+constexpr uint32_t TM_C1 = 384;  // gK
+constexpr uint32_t TM_QA = 384;  // dQ pass: Q rows, 64 columns of bf16 pairs
+constexpr uint32_t TM_GA = 448;  // dQ pass: G rows
 
 constexpr uint32_t IDESC_N64 = ptx::idesc_bf16(BR, BT, false, false);  // 128 x 64, K-major B
 constexpr uint32_t IDESC_MN = ptx::idesc_bf16(BR, D, false, true);     // 128 x 128, MN-major B
@@ -109,7 +118,8 @@ struct Params {
   const float* lse;     // forward LSE (natural log)
   float2* sd;           // scratch [B*H, Lp] of {LSE * log2(e), D_i = <g_i, o_i>}: written
                         // by the dQ pass (rows past L: {+inf, 0}), read by the dK/dV pass
-  const __nv_bfloat16* g;  // cotangent, for D (dQ pass)
+  const __nv_bfloat16* q;  // dQ pass: stationary rows, stored into TMEM
+  const __nv_bfloat16* g;  // cotangent: stationary rows and D (dQ pass)
   const __nv_bfloat16* o;  // forward output, for D (dQ pass)
   __nv_bfloat16* out0;     // gQ (dQ pass) or gK (dK/dV pass)
   __nv_bfloat16* out1;     // gV (dK/dV pass)
@@ -119,16 +129,22 @@ struct Params {
 };
 using Cursor = pipe::Cursor<Params>;
 
-// Stationary operand for the stationary-side MMAs (K-major, 128 rows) and
-// streamed operands (64 rows) that serve both as K-major B (first MMAs) and
-// as MN-major B (accumulating MMAs).
+// MMA issue is split over two threads, since one thread issues at most about
+// one tcgen05.mma per ~47 cycles while a 128 x 64 x 16 MMA takes 32:
+//   issuer A (warp 1): S(t) = A0 X(t)^T into buffer t&1, once the
+//                      accumulating MMAs of tile t-2 (same buffer) are done;
+//   issuer B (warp 2): dP(t) = A1 Y(t)^T, and acc(t) once the softmax warps
+//                      have written tile t's bf16 operands. B issues dP(t)
+//                      after acc(t-2), so its own order protects the buffer.
+// The pipe executes each thread's MMAs in issue order; every hand-over
+// between the two threads and the other roles goes through an mbarrier.
 template <bool kKV>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
            const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
            const __grid_constant__ Params p) {
-  // dQ pass:  A0 = Q, A1 = G (stationary);  X = K (3 stages), Y = V.
-  // dK/dV:    A0 = K, A1 = V (stationary);  X = Q (3 stages), Y = G.
+  // dQ pass:  A0 = Q, A1 = G (stationary, TMEM);  X = K, Y = V (smem rings).
+  // dK/dV:    A0 = K, A1 = V (stationary, smem);  X = Q, Y = G.
   using LY = Layout<kKV>;
   constexpr uint32_t NX = LY::NX, NY = LY::NY;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -141,8 +157,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(B_AF), 1);
-    mbar_init(bar(B_AE), 1);
+    // dQ: the 256 softmax threads store Q / G rows and arrive; dK/dV: TMA bytes.
+    mbar_init(bar(B_AF), kKV ? 1 : 2 * BR);
+    mbar_init(bar(B_AE), 2);
     for (uint32_t s = 0; s < NX; ++s) {
       mbar_init(bar(B_XF + s), 1);
       mbar_init(bar(B_XE + s), 1);
@@ -152,22 +169,24 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       mbar_init(bar(B_YE + s), 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(B_SF + b), 1);
+      mbar_init(bar(B_SF + b), 2);
       mbar_init(bar(B_PF + b), 2 * BR);
+      mbar_init(bar(B_MD + b), 1);
+      mbar_init(bar(B_DRAIN + b), 1);
     }
-    mbar_init(bar(B_MD), 1);
     mbar_init(bar(B_CF), 2 * BR);
-    mbar_init(bar(B_DRAIN), 1);
     for (uint32_t i = 0; i < kRing; ++i) {
       mbar_init(bar(B_IF + i), 1);
-      mbar_init(bar(B_IE + i), kRingReaders);
+      mbar_init(bar(B_IE + i), kReaders);
     }
     *abort_flag = 0u;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_map(&tm_a0);
-    tma_prefetch_map(&tm_a1);
+    if (kKV) {
+      tma_prefetch_map(&tm_a0);
+      tma_prefetch_map(&tm_a1);
+    }
     tma_prefetch_map(&tm_x);
     tma_prefetch_map(&tm_y);
   }
@@ -190,7 +209,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       uint32_t a_armed = 0, x_issued = 0, y_issued = 0;
       bool ok = true;
       while (c.valid && ok) {
-        if (c.j == 0) {
+        if (kKV && c.j == 0) {
           if (c.item_idx > 0) ok = wait_bar(bar(B_AE), (c.item_idx - 1) & 1, p, abort_flag);
           if (!ok) break;
           mbar_expect_tx(bar(B_AF), 4 * kRHalf);
@@ -232,44 +251,54 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA ----
+  } else if (warp == 1 || warp == 2) {
+    // ---------------------------------------------------- MMA issuers ----
     if (lane == 0) {
-      bool ok = true;
+      const bool issuer_a = warp == 1;
       const uint64_t a0_desc = sdesc_sw128(base + LY::A0, 16, 1024);
       const uint64_t a1_desc = sdesc_sw128(base + LY::A1, 16, 1024);
       const uint64_t xk_desc = sdesc_sw128(base + LY::X, 16, 1024);       // K-major view
       const uint64_t xm_desc = sdesc_sw128(base + LY::X, kTHalf, 1024);   // MN-major view
       const uint64_t yk_desc = sdesc_sw128(base + LY::Y, 16, 1024);
       const uint64_t ym_desc = sdesc_sw128(base + LY::Y, kTHalf, 1024);
-      // First MMAs of a tile: T0 = A0 X^T into S, T1 = A1 Y^T into dP.
-      auto issue_s = [&](const Cursor& c) -> bool {
-        const uint32_t b = c.t & 1u, sx = c.t % NX, sy = c.t % NY;
+      // First MMAs of tile t: S = A0 X^T (issuer A) or dP = A1 Y^T (issuer B).
+      auto issue_first = [&](const Cursor& c, bool s_mma) -> bool {
+        const uint32_t b = c.t & 1u;
         if (c.j == 0 && !wait_bar(bar(B_AF), c.item_idx & 1, p, abort_flag)) return false;
-        if (!wait_bar(bar(B_XF + sx), (c.t / NX) & 1u, p, abort_flag)) return false;
-        if (!wait_bar(bar(B_YF + sy), (c.t / NY) & 1u, p, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t d_s = tmem + b * 128u, d_p = d_s + 64u;
-        const uint64_t xb = xk_desc + sx * (kTile >> 4), yb = yk_desc + sy * (kTile >> 4);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t oa = ((kk >> 2) * kRHalf + (kk & 3) * 32) >> 4;
-          const uint32_t ob = ((kk >> 2) * kTHalf + (kk & 3) * 32) >> 4;
-          mma_ss(d_s, a0_desc + oa, xb + ob, IDESC_N64, kk > 0);
+        uint32_t stage;
+        uint64_t bdesc;
+        if (s_mma) {
+          // Buffer b last held tile t-2, whose operands acc(t-2) reads.
+          if (c.t >= 2 && !wait_bar(bar(B_MD + b), ((c.t >> 1) - 1) & 1u, p, abort_flag))
+            return false;
+          stage = c.t % NX;
+          if (!wait_bar(bar(B_XF + stage), (c.t / NX) & 1u, p, abort_flag)) return false;
+          bdesc = xk_desc + stage * (kTile >> 4);
+        } else {
+          stage = c.t % NY;
+          if (!wait_bar(bar(B_YF + stage), (c.t / NY) & 1u, p, abort_flag)) return false;
+          bdesc = yk_desc + stage * (kTile >> 4);
         }
+        tc_fence_after();
+        const uint32_t d = tmem + b * 128u + (s_mma ? 0u : 64u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t oa = ((kk >> 2) * kRHalf + (kk & 3) * 32) >> 4;
           const uint32_t ob = ((kk >> 2) * kTHalf + (kk & 3) * 32) >> 4;
-          mma_ss(d_p, a1_desc + oa, yb + ob, IDESC_N64, kk > 0);
+          if (!kKV) {
+            mma_ts(d, tmem + (s_mma ? TM_QA : TM_GA) + 8u * kk, bdesc + ob, IDESC_N64, kk > 0);
+          } else {
+            const uint32_t oa = ((kk >> 2) * kRHalf + (kk & 3) * 32) >> 4;
+            mma_ss(d, (s_mma ? a0_desc : a1_desc) + oa, bdesc + ob, IDESC_N64, kk > 0);
+          }
         }
         mma_commit(bar(B_SF + b));
-        if (!kKV) mma_commit(bar(B_YE + sy));  // dQ pass: V is used by dP only
-        if (c.j == c.n - 1) mma_commit(bar(B_AE));
+        if (!s_mma && !kKV) mma_commit(bar(B_YE + stage));  // dQ pass: V feeds dP only
+        if (kKV && c.j == c.n - 1) mma_commit(bar(B_AE));   // done with A0 (A) / A1 (B)
         return true;
       };
-      // Accumulating MMAs. The bf16 operands of a tile sit in TMEM columns
-      // {0, 8} and {32, 40} (one pair of 16-wide k-steps per warpgroup).
+      // Accumulating MMAs (issuer B). The bf16 operands of a tile sit in
+      // TMEM columns {0, 8} and {32, 40} (one pair of 16-wide k-steps per
+      // warpgroup) of the S part (and, dK/dV pass, of the dP part).
       auto issue_acc = [&](const Cursor& c) -> bool {
         const uint32_t b = c.t & 1u, sx = c.t % NX, sy = c.t % NY;
         if (c.j == 0 && c.item_idx > 0 &&
@@ -295,29 +324,42 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
                    first | (ks > 0));
           }
         }
+        // X(t) was also read by S(t), which completed before the softmax
+        // warps released tile t.
         mma_commit(bar(B_XE + sx));
         if (kKV) mma_commit(bar(B_YE + sy));
-        mma_commit(bar(B_MD));
+        mma_commit(bar(B_MD + b));
         return true;
       };
-      Cursor cs, cp;
-      cs.start(p, ring, kConsumerThread);
-      cp.start(p, ring, kConsumerThread);
-      for (int pre = 0; pre < 2 && cs.valid && ok; ++pre) {
-        ok = issue_s(cs);
-        cs.next(p, ring, kConsumerThread);
-      }
-      while (cp.valid && ok) {
-        ok = issue_acc(cp);
-        cp.next(p, ring, kConsumerThread);
-        if (ok && cs.valid) {
-          ok = issue_s(cs);
+      bool ok = true;
+      if (issuer_a) {
+        Cursor cs;
+        cs.start(p, ring, kConsumerThread);
+        while (cs.valid && ok) {
+          ok = issue_first(cs, true);
           cs.next(p, ring, kConsumerThread);
+        }
+      } else {
+        // dP runs up to two tiles ahead of acc, but not into the next item:
+        // that item's stationary operands (dQ pass) are stored only after
+        // the epilogue of this one, which waits for this item's last acc.
+        Cursor cd, ca;
+        cd.start(p, ring, kConsumerThread);
+        ca.start(p, ring, kConsumerThread);
+        while (ca.valid && ok) {
+          while (ok && cd.valid && cd.t < ca.t + 2 && cd.item_idx == ca.item_idx) {
+            ok = issue_first(cd, false);
+            cd.next(p, ring, kConsumerThread);
+          }
+          if (!ok) break;
+          ok = issue_acc(ca);
+          ca.next(p, ring, kConsumerThread);
         }
       }
       if (!ok || *abort_flag) {
-        mma_commit(bar(B_DRAIN));
-        drain_wait(bar(B_DRAIN), 0);
+        const uint32_t db = bar(B_DRAIN + (issuer_a ? 0 : 1));
+        mma_commit(db);
+        drain_wait(db, 0);
       }
     }
     __syncwarp();
@@ -366,6 +408,34 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
           }
           // grow < Lp always: the last query tile covers the padding rows.
           if (hw == 0) p.sd[size_t(c.bh) * p.Lp + grow] = make_float2(lse2, dval);
+          // The item's stationary rows into TMEM, as bf16 pairs (the A
+          // operands of the first MMAs): warpgroup 0 stores Q, warpgroup 1
+          // G; rows past L are zero. The previous item's S and dP MMAs all
+          // completed before its last tile reached these warps, and neither
+          // issuer starts this item's before B_AF completes.
+          const __nv_bfloat16* src = hw == 0 ? p.q : p.g;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t rv[32];
+            if (grow < p.L) {
+              const uint4* s4 = reinterpret_cast<const uint4*>(src + roff * D) + half * 8;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const uint4 v4 = s4[i];
+                rv[4 * i] = v4.x;
+                rv[4 * i + 1] = v4.y;
+                rv[4 * i + 2] = v4.z;
+                rv[4 * i + 3] = v4.w;
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) rv[i] = 0u;
+            }
+            tmem_st32(tl + (hw == 0 ? TM_QA : TM_GA) + 32u * half, rv);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(B_AF));
         } else {
           rk = key_queries(p.mask.mode, p.mask.tokens_per_frame, p.mask.n_frames, chunk, p.L,
                            grow);
@@ -436,8 +506,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
 
       if (c.j == c.n - 1) {
         // ------------------------------------------------------ epilogue --
-        ok = c.t == 0 || wait_bar(bar(B_MD), (c.t - 1) & 1u, p, abort_flag);
-        ok = ok && wait_bar(bar(B_MD), c.t & 1u, p, abort_flag);
+        // acc(t-2) on the same barrier has completed: S(t) waited for it.
+        ok = wait_bar(bar(B_MD + (c.t & 1u)), (c.t >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
         const bool row_ok = grow < p.L;
@@ -539,6 +609,7 @@ static int launch_pass(const BwdArgs& a, const WorkList& w, int num_sms, unsigne
   p.lse = a.lse;
   p.Lp = (a.L + 127) / 128 * 128;
   p.sd = reinterpret_cast<float2*>(a.scratch);
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.g = static_cast<const __nv_bfloat16*>(a.g);
   p.o = static_cast<const __nv_bfloat16*>(a.o);
   p.out0 = static_cast<__nv_bfloat16*>(kKV ? a.gk : a.gq);
