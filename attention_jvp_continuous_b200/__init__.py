@@ -19,7 +19,8 @@ FRAME_CAUSAL = 1
 CHUNK_CAUSAL = 2
 TEACHER_FORCING = 3
 
-__all__ = ["Mask", "jvp_attn", "jvp_attn_fwd", "attn_bwd", "mask_stats", "tile_classes",
+__all__ = ["Mask", "jvp_attn", "jvp_attn_fwd", "attn_bwd", "jvp_attn_bwd", "bwd_scratch_len",
+           "mask_stats", "tile_classes",
            "schedule", "schedule_kv", "check_device_error", "set_wait_limit", "release",
            "JvpAttnError",
            "DENSE", "FRAME_CAUSAL", "CHUNK_CAUSAL", "TEACHER_FORCING"]
@@ -99,32 +100,50 @@ def jvp_attn(q, k, v, dq, dk, dv, mask: Mask, scale: Optional[float] = None,
     return o, d_o, lse
 
 
-def attn_bwd(q, k, v, o, g, lse, mask: Mask, scale: Optional[float] = None,
-             stream: Optional[int] = None):
-    """Gradients (g_q, g_k, g_v) of sum <g, o> for o = masked attention of
-    (q, k, v); o and lse as returned by jvp_attn. bf16 CUDA tensors, d = 128."""
-    import torch
-    ts = (q, k, v, o, g)
-    for t in ts:
-        if not t.is_cuda or t.shape != q.shape or t.dtype != q.dtype or not t.is_contiguous():
-            raise ValueError("q, k, v, o, g must be contiguous CUDA tensors of one shape and dtype")
-    if not lse.is_cuda or lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous float32 CUDA tensor [B, H, L]")
-    B, H, L, d = q.shape
-    gq, gk, gv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
-    n_scratch = _lib.lib().jvp_attn_bwd_scratch_len(B, H, L)
-    if n_scratch < 0:
+def bwd_scratch_len(B: int, H: int, L: int) -> int:
+    """float32 elements of scratch jvp_attn_bwd needs (jvp_attn_bwd_scratch_len)."""
+    n = _lib.lib().jvp_attn_bwd_scratch_len(B, H, L)
+    if n < 0:
         raise ValueError("invalid shape for jvp_attn_bwd")
-    scratch = torch.empty((n_scratch,), dtype=torch.float32, device=q.device)
+    return int(n)
+
+
+def jvp_attn_bwd(q, k, v, o, g, lse, gq, gk, gv, scratch, mask: Mask,
+                 scale: Optional[float] = None, stream: Optional[int] = None) -> None:
+    """Into preallocated outputs: (gq, gk, gv) = gradients of sum <g, o> for
+    o = masked attention of (q, k, v). bf16 CUDA tensors [B, H, L, 128]; o and
+    lse as returned by jvp_attn; scratch a float32 CUDA tensor of at least
+    bwd_scratch_len(B, H, L) elements. Allocates nothing."""
+    import torch
+    for t in (q, k, v, o, g, gq, gk, gv):
+        if not t.is_cuda or t.shape != q.shape or t.dtype != q.dtype or not t.is_contiguous():
+            raise ValueError("q, k, v, o, g, gq, gk, gv must be contiguous CUDA tensors of "
+                             "one shape and dtype")
+    for t, name in ((lse, "lse"), (scratch, "scratch")):
+        if not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous float32 CUDA tensor")
+    B, H, L, d = q.shape
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
     fp = ctypes.POINTER(ctypes.c_float)
     rc = _lib.lib().jvp_attn_bwd(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), g.data_ptr(),
         ctypes.cast(lse.data_ptr(), fp), gq.data_ptr(), gk.data_ptr(), gv.data_ptr(),
-        ctypes.cast(scratch.data_ptr(), fp), n_scratch, B, H, L, d, _dtype_code(q), mask.desc(),
-        0.0 if scale is None else float(scale), ctypes.c_void_p(stream))
+        ctypes.cast(scratch.data_ptr(), fp), scratch.numel(), B, H, L, d, _dtype_code(q),
+        mask.desc(), 0.0 if scale is None else float(scale), ctypes.c_void_p(stream))
     _lib.check(rc, "jvp_attn_bwd")
+
+
+def attn_bwd(q, k, v, o, g, lse, mask: Mask, scale: Optional[float] = None,
+             stream: Optional[int] = None):
+    """Gradients (g_q, g_k, g_v) of sum <g, o> for o = masked attention of
+    (q, k, v); o and lse as returned by jvp_attn. bf16 CUDA tensors, d = 128.
+    Allocates the outputs and the scratch, then calls jvp_attn_bwd."""
+    import torch
+    B, H, L, d = q.shape
+    gq, gk, gv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    scratch = torch.empty((bwd_scratch_len(B, H, L),), dtype=torch.float32, device=q.device)
+    jvp_attn_bwd(q, k, v, o, g, lse, gq, gk, gv, scratch, mask, scale, stream)
     return gq, gk, gv
 
 

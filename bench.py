@@ -18,6 +18,11 @@ reported. Rank 0 prints one JSON line.
 
 ``--impl reference`` times the float64 CPU oracle on this machine's host cores
 instead (rank 0 only), on a bounded sample of query rows per step.
+
+``--op bwd`` measures the masked attention backward instead (gradients of
+<G, O> for the primal output, jvp_attn_bwd) on the same workload, counting
+10*d FLOPs per admitted pair: S recomputed (2d), dP = G V^T (2d), and the
+three gradient products (2d each); the two passes execute 14*d.
 """
 from __future__ import annotations
 
@@ -35,6 +40,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "attention-JVP TFLOP/s (12*d per unmasked pair) and % of B200 bf16 tensor peak"
+METRIC_BWD = ("masked attention backward TFLOP/s (10*d per unmasked pair) and % of B200 "
+              "bf16 tensor peak")
 UNIT = "TFLOP/s"
 NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
@@ -77,8 +84,12 @@ def stored_traffic(workload: str):
     return e.get("dram_bytes_per_launch")
 
 
-def flops_per_step(w, pairs_per_head: int) -> float:
-    return 12.0 * w.d * pairs_per_head * w.B * w.H
+def flops_per_pair(w, op: str = "jvp") -> float:
+    return (10.0 if op == "bwd" else 12.0) * w.d
+
+
+def flops_per_step(w, pairs_per_head: int, op: str = "jvp") -> float:
+    return flops_per_pair(w, op) * pairs_per_head * w.B * w.H
 
 
 def rank_seed(base_seed: int, rank: int) -> int:
@@ -204,7 +215,8 @@ def run_ours(args, w):
     ja._lib.lib()  # fail loudly if the CUDA library is missing
     mask = ja.Mask(w.mode, w.tokens_per_frame, w.n_frames, w.chunk)
     pairs, n_full, n_part, _ = ja.mask_stats(mask)
-    flops = flops_per_step(w, pairs)
+    bwd = args.op == "bwd"
+    flops = flops_per_step(w, pairs, args.op)
 
     inputs, _ = make_inputs(w, device="cuda", seed=rank_seed(w.seed, rank))
     q = inputs[0]
@@ -213,8 +225,25 @@ def run_ours(args, w):
     lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=q.device)
     stream = torch.cuda.current_stream()
 
-    def step():
+    if bwd:
+        # Backward inputs: q, k, v, the primal output and LSE of the forward
+        # (computed once, outside the timed region) and a seeded N(0, 1)
+        # cotangent G; outputs and scratch preallocated.
+        gen = torch.Generator(device=q.device).manual_seed(rank_seed(w.seed, rank) + 17)
+        g = torch.randn(q.shape, generator=gen, device=q.device).to(q.dtype)
         ja.jvp_attn_fwd(*inputs, o, d_o, lse, mask)
+        grads = [torch.empty_like(q) for _ in range(3)]
+        scratch = torch.empty((ja.bwd_scratch_len(w.B, w.H, w.L),), dtype=torch.float32,
+                              device=q.device)
+        step_in = [inputs[0], inputs[1], inputs[2], o, g, lse]
+
+        def step():
+            ja.jvp_attn_bwd(*step_in, *grads, scratch, mask)
+    else:
+        step_in = list(inputs)
+
+        def step():
+            ja.jvp_attn_fwd(*inputs, o, d_o, lse, mask)
 
     for _ in range(args.warmup):
         step()
@@ -242,22 +271,23 @@ def run_ours(args, w):
     launch_ms = sum(per) / len(per)
 
     # ---- end to end through the C ABI: pinned host in, host out ----
-    host_in = [t.cpu().pin_memory() for t in inputs]
-    host_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    host_do = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    host_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    dev_in = [torch.empty_like(t) for t in inputs]
+    host_in = [t.cpu().pin_memory() for t in step_in]
+    dev_in = [torch.empty_like(t) for t in step_in]
+    dev_out = grads if bwd else [o, d_o, lse]
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in dev_out]
     h2d = sum(t.numel() * t.element_size() for t in host_in)
-    d2h = sum(t.numel() * t.element_size() for t in (host_o, host_do, host_lse))
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
     e2e_steps = max(1, min(args.steps, 5))
 
     def e2e_step():
         for d, h in zip(dev_in, host_in):
             d.copy_(h, non_blocking=True)
-        ja.jvp_attn_fwd(*dev_in, o, d_o, lse, mask)
-        host_o.copy_(o, non_blocking=True)
-        host_do.copy_(d_o, non_blocking=True)
-        host_lse.copy_(lse, non_blocking=True)
+        if bwd:
+            ja.jvp_attn_bwd(*dev_in, *grads, scratch, mask)
+        else:
+            ja.jvp_attn_fwd(*dev_in, o, d_o, lse, mask)
+        for h, d in zip(host_out, dev_out):
+            h.copy_(d, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -285,9 +315,12 @@ def run_ours(args, w):
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
     achieved = flops / (launch_ms * 1e-3) / 1e12
-    traffic = stored_traffic(w.name)
+    traffic = None if bwd else stored_traffic(w.name)
+    kernel = ("bwd_kernel<false> + bwd_kernel<true> (query pass, key/value pass)" if bwd
+              else "jvp_attn_sm100_kernel")
     line = {
-        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "metric": METRIC_BWD if bwd else METRIC, "value": round(value, 2), "unit": UNIT,
+        "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total_ms_max / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -305,7 +338,7 @@ def run_ours(args, w):
         },
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * (2 if bwd else 1),
         "roofline": {
             "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": UNIT,
             "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -313,12 +346,17 @@ def run_ours(args, w):
             "frac_of_sustained": round(achieved / float(peaks.get(
                 "bf16_tflops_sustained", peak)), 4),
             "frac_of_nominal_2250": round(achieved / NOMINAL_BF16_TFLOPS, 4),
-            "kernel": "jvp_attn_sm100_kernel", "launch_ms": round(launch_ms, 4),
+            "kernel": kernel, "launch_ms": round(launch_ms, 4),
         },
         "clocks": clocks,
     }
+    if bwd:
+        line["config"]["cotangent"] = "G ~ N(0, 1), bf16, seeded"
+        line["config"]["executed_flops_per_pair"] = 14 * w.d
     if not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, inputs, rows_per_head=args.cpu_rows)
+        line["cpu_baseline"] = (cpu_baseline_bwd(w, step_in, rows_per_head=args.cpu_rows_bwd)
+                                if bwd else
+                                cpu_baseline(w, inputs, rows_per_head=args.cpu_rows))
     return line
 
 
@@ -361,26 +399,65 @@ def cpu_baseline(w, inputs, rows_per_head: int):
                       f"({sp} admitted pairs, {dt:.1f} s, float64 numpy)"}
 
 
+def oracle_sample_bwd(w, host_in, rows_per_head: int, seed: int = 1234):
+    """Times the float64 backward oracle restricted to ``rows_per_head``
+    seeded query rows of every head (their gradient contributions); returns
+    (seconds, admitted pairs of those rows)."""
+    from attention_jvp_continuous_b200.inputs import sample_rows
+    from oracle import MaskSpec, key_intervals
+    from oracle.attention_backward import attention_backward
+
+    spec = MaskSpec(w.mode, w.tokens_per_frame, w.n_frames, w.chunk)
+    rows = sample_rows(w.L, rows_per_head, seed=seed)
+    pairs_per_head = sum(b - a for r in rows for a, b in key_intervals(spec, int(r)))
+    q, k, v, _, g = host_in[:5]
+    t0 = time.perf_counter()
+    attention_backward(q, k, v, g, spec, rows=[int(r) for r in rows])
+    dt = time.perf_counter() - t0
+    return dt, pairs_per_head * w.B * w.H
+
+
+def cpu_baseline_bwd(w, step_in, rows_per_head: int):
+    host = [t.cpu() for t in step_in]
+    dt, sp = oracle_sample_bwd(w, host, rows_per_head)
+    return {"value": round(flops_per_pair(w, "bwd") * sp / dt / 1e12, 6), "unit": UNIT,
+            "cores": blas_threads(), "kind": "oracle",
+            "sample": f"gradient contributions of {rows_per_head} seeded query rows per "
+                      f"head x {w.B * w.H} heads ({sp} admitted pairs, {dt:.1f} s, "
+                      f"float64 numpy)"}
+
+
 def run_reference(args, w):
     world, rank, _ = dist_setup()
     if rank != 0:
         return None
+    import torch
+
     from attention_jvp_continuous_b200.inputs import make_inputs
     inputs, _ = make_inputs(w, device="cpu")
     rows = args.ref_rows
+    if args.op == "bwd":
+        # The oracle's gradient needs no primal output; a seeded cotangent.
+        gen = torch.Generator().manual_seed(w.seed + 17)
+        g = torch.randn(inputs[0].shape, generator=gen).to(inputs[0].dtype)
+        host = [inputs[0], inputs[1], inputs[2], None, g]
+        run_sample = lambda seed: oracle_sample_bwd(w, host, rows, seed=seed)  # noqa: E731
+    else:
+        run_sample = lambda seed: oracle_sample(w, inputs, rows, seed=seed)  # noqa: E731
     for i in range(args.warmup):
-        oracle_sample(w, inputs, rows, seed=100 + i)
+        run_sample(100 + i)
     times, pairs = [], 0
     for i in range(args.steps):
-        dt, sp = oracle_sample(w, inputs, rows, seed=1234 + i)
+        dt, sp = run_sample(1234 + i)
         times.append(dt)
         pairs += sp
     total = sum(times)
-    value = 12.0 * w.d * pairs / total / 1e12
+    value = flops_per_pair(w, args.op) * pairs / total / 1e12
     cores = blas_threads()
     sample = f"{rows} seeded query rows per head x {w.B * w.H} heads per step"
     return {
-        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "impl": "reference", "metric": METRIC_BWD if args.op == "bwd" else METRIC,
+        "value": round(value, 6), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * total / args.steps, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -408,12 +485,23 @@ def main(argv=None):
                     help="query rows per head in the cpu_baseline sample")
     ap.add_argument("--ref-rows", type=int, default=32,
                     help="query rows per head per step of --impl reference")
+    ap.add_argument("--cpu-rows-bwd", type=int, default=1024,
+                    help="query rows per head in the --op bwd cpu_baseline sample")
+    ap.add_argument("--op", choices=["jvp", "bwd"], default="jvp",
+                    help="jvp: the attention JVP (default); bwd: the masked backward")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the workload's head count (small cases for ncu captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from attention_jvp_continuous_b200.inputs import WORKLOADS
     w = WORKLOADS[args.workload]
+    if args.heads is not None:
+        if args.heads < 1:
+            ap.error("--heads must be >= 1")
+        import dataclasses
+        w = dataclasses.replace(w, H=args.heads)
     world, rank, _ = dist_setup()
     if world != args.gpus and args.impl == "ours":
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)

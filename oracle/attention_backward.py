@@ -27,7 +27,7 @@ softmax; no blocking beyond that.
 from __future__ import annotations
 
 import math
-from typing import Optional
+from typing import Optional, Sequence
 
 import numpy as np
 
@@ -36,11 +36,14 @@ from .masks import MaskSpec
 
 
 def attention_backward_head(q, k, v, g, spec: MaskSpec, scale: Optional[float] = None,
-                            row_block: int = 128):
+                            row_block: int = 128, rows: Optional[Sequence[int]] = None):
     """Gradients (gq, gk, gv) of sum <g, O> for one (batch, head) slice.
 
     q, k, v, g: [L, d]. Returns float64 arrays [L, d] each. Every query row
-    contributes to gk and gv, so all rows are evaluated.
+    contributes to gk and gv, so by default all rows are evaluated. With
+    ``rows``, only those query rows contribute: gq is exact on them and zero
+    elsewhere, gk and gv are the sums of their contributions (the loss
+    restricted to those rows of O). Used to time a bounded sample.
     """
     q, k, v, g = (_as64(t) for t in (q, k, v, g))
     L, d = q.shape
@@ -50,7 +53,7 @@ def attention_backward_head(q, k, v, g, spec: MaskSpec, scale: Optional[float] =
     gq = np.zeros((L, d))
     gk = np.zeros((L, d))
     gv = np.zeros((L, d))
-    for ivs, grp in _group_rows(spec, range(L)).items():
+    for ivs, grp in _group_rows(spec, range(L) if rows is None else rows).items():
         if not ivs:
             continue
         grp = np.asarray(grp)
@@ -72,13 +75,16 @@ def attention_backward_head(q, k, v, g, spec: MaskSpec, scale: Optional[float] =
     return gq, gk, gv
 
 
-def attention_backward(q, k, v, g, spec: MaskSpec, scale: Optional[float] = None):
-    """Oracle over [B, H, L, d] inputs: float64 (gq, gk, gv), each [B, H, L, d]."""
+def attention_backward(q, k, v, g, spec: MaskSpec, scale: Optional[float] = None,
+                       rows: Optional[Sequence[int]] = None):
+    """Oracle over [B, H, L, d] inputs: float64 (gq, gk, gv), each [B, H, L, d].
+    ``rows`` as in attention_backward_head, for every (batch, head)."""
     B, H, L, d = q.shape
     out = [np.zeros((B, H, L, d)) for _ in range(3)]
     for b in range(B):
         for h in range(H):
-            res = attention_backward_head(q[b, h], k[b, h], v[b, h], g[b, h], spec, scale)
+            res = attention_backward_head(q[b, h], k[b, h], v[b, h], g[b, h], spec, scale,
+                                          rows=rows)
             for o, r in zip(out, res):
                 o[b, h] = r
     return tuple(out)

@@ -119,3 +119,24 @@ def test_backward_token_causal_special_case():
     np.testing.assert_allclose(gq, qa.grad.numpy(), atol=1e-11)
     np.testing.assert_allclose(gk, ka.grad.numpy(), atol=1e-11)
     np.testing.assert_allclose(gv, va.grad.numpy(), atol=1e-11)
+
+
+def test_backward_row_subsets_partition():
+    # The loss is a sum over query rows, so the contributions of a partition
+    # of the rows add up to the full gradient; gq is exact on its own rows.
+    spec = MaskSpec(TEACHER_FORCING, 3, 4, 2)
+    q, k, v, g = rand(9, 1, 1, spec.length, 8)
+    full = attention_backward(q, k, v, g, spec)
+    L = spec.length
+    perm = np.random.default_rng(3).permutation(L)
+    parts = [sorted(perm[:7]), sorted(perm[7:15]), sorted(perm[15:])]
+    acc = [np.zeros_like(x) for x in full]
+    for rows in parts:
+        sub = attention_backward(q, k, v, g, spec, rows=rows)
+        rest = np.setdiff1d(np.arange(L), rows)
+        np.testing.assert_allclose(sub[0][:, :, rows], full[0][:, :, rows], atol=1e-12)
+        assert np.all(sub[0][:, :, rest] == 0)
+        for a, x in zip(acc, sub):
+            a += x
+    for a, x in zip(acc, full):
+        np.testing.assert_allclose(a, x, atol=1e-12)
