@@ -132,3 +132,15 @@ def sample_rows(L: int, n: int, seed: int = 1234):
     rng = np.random.default_rng(seed)
     n = min(n, L)
     return np.sort(rng.choice(L, size=n, replace=False)).astype(np.int64)
+
+
+def rope_table(n_pos: int, d: int, base: float = 10000.0, pos0: int = 0, device="cpu"):
+    """cos / sin tables [n_pos, d/2] (float32) for rotary position embedding:
+    row p, pair i holds the angle (pos0 + p) * base^(-2i/d). Built in float64
+    and rounded once; the rotation itself is the caller's (or kernel's)."""
+    import numpy as np
+    i = np.arange(d // 2, dtype=np.float64)
+    ang = (pos0 + np.arange(n_pos, dtype=np.float64))[:, None] * base ** (-2.0 * i / d)[None, :]
+    cos = torch.from_numpy(np.cos(ang).astype(np.float32)).to(device)
+    sin = torch.from_numpy(np.sin(ang).astype(np.float32)).to(device)
+    return cos.contiguous(), sin.contiguous()
