@@ -20,7 +20,7 @@ CHUNK_CAUSAL = 2
 TEACHER_FORCING = 3
 
 __all__ = ["Mask", "jvp_attn", "jvp_attn_fwd", "attn_bwd", "jvp_attn_bwd", "bwd_scratch_len",
-           "mask_stats", "tile_classes",
+           "cache_attn", "rope_copy", "mask_stats", "tile_classes",
            "schedule", "schedule_kv", "check_device_error", "set_wait_limit", "release",
            "JvpAttnError",
            "DENSE", "FRAME_CAUSAL", "CHUNK_CAUSAL", "TEACHER_FORCING"]
@@ -145,6 +145,73 @@ def attn_bwd(q, k, v, o, g, lse, mask: Mask, scale: Optional[float] = None,
     scratch = torch.empty((bwd_scratch_len(B, H, L),), dtype=torch.float32, device=q.device)
     jvp_attn_bwd(q, k, v, o, g, lse, gq, gk, gv, scratch, mask, scale, stream)
     return gq, gk, gv
+
+
+def cache_attn(q, k_cache, v_cache, n_keys: int, o=None, lse=None,
+               scale: Optional[float] = None, stream: Optional[int] = None):
+    """Chunk attention over a key/value cache (jvp_attn_cache_fwd): the
+    queries q [B, H, Lq, 128] attend to rows [0, n_keys) of k_cache, v_cache
+    [B, H, Lcache, 128] (bf16, CUDA). Returns (o [B, H, Lq, 128] bf16,
+    lse [B, H, Lq] float32), into o / lse when given."""
+    import torch
+    B, H, Lq, d = q.shape
+    for t in (q, k_cache, v_cache):
+        if not t.is_cuda or t.dtype != q.dtype or not t.is_contiguous():
+            raise ValueError("q, k_cache, v_cache must be contiguous CUDA tensors of one dtype")
+    if k_cache.shape != v_cache.shape or k_cache.shape[:2] != (B, H) or k_cache.shape[3] != d:
+        raise ValueError("k_cache and v_cache must be [B, H, Lcache, d] matching q")
+    Lcache = k_cache.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    if o.shape != q.shape or o.dtype != q.dtype or not o.is_contiguous():
+        raise ValueError("o must be a contiguous tensor like q")
+    if lse.shape != (B, H, Lq) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor [B, H, Lq]")
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    fp = ctypes.POINTER(ctypes.c_float)
+    rc = _lib.lib().jvp_attn_cache_fwd(
+        q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), o.data_ptr(),
+        ctypes.cast(lse.data_ptr(), fp), B, H, Lq, int(n_keys), Lcache, d, _dtype_code(q),
+        0.0 if scale is None else float(scale), ctypes.c_void_p(stream))
+    _lib.check(rc, "jvp_attn_cache_fwd")
+    return o, lse
+
+
+def rope_copy(src, dst, rows: int, src_row0: int = 0, dst_row0: int = 0, cos=None, sin=None,
+              rope_row0: int = 0, stream: Optional[int] = None) -> None:
+    """Copies rows [src_row0, src_row0 + rows) of src [B, H, Ls, d] to rows
+    [dst_row0, ...) of dst [B, H, Ld, d] (jvp_attn_rope_copy), rotating row j
+    by table row rope_row0 + j of cos / sin (float32 [n, d/2]) when given."""
+    import torch
+    for t in (src, dst):
+        if not t.is_cuda or t.dtype != src.dtype or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("src and dst must be contiguous 4-D CUDA tensors of one dtype")
+    B, H, Ls, d = src.shape
+    if dst.shape[:2] != (B, H) or dst.shape[3] != d:
+        raise ValueError("dst must be [B, H, Ld, d] matching src")
+    fp = ctypes.POINTER(ctypes.c_float)
+    cp = sp = None
+    n_rope = 0
+    if (cos is None) != (sin is None):
+        raise ValueError("give both cos and sin, or neither")
+    if cos is not None:
+        for t in (cos, sin):
+            if not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+                raise ValueError("cos / sin must be contiguous float32 CUDA tensors [n, d/2]")
+        if cos.shape != sin.shape or cos.dim() != 2 or cos.shape[1] * 2 != d:
+            raise ValueError("cos / sin must both be [n, d/2]")
+        cp, sp = ctypes.cast(cos.data_ptr(), fp), ctypes.cast(sin.data_ptr(), fp)
+        n_rope = cos.shape[0]
+    if stream is None:
+        stream = torch.cuda.current_stream(src.device).cuda_stream
+    rc = _lib.lib().jvp_attn_rope_copy(
+        src.data_ptr(), dst.data_ptr(), B, H, Ls, dst.shape[2], int(rows), int(src_row0),
+        int(dst_row0), d, _dtype_code(src), cp, sp, n_rope, int(rope_row0),
+        ctypes.c_void_p(stream))
+    _lib.check(rc, "jvp_attn_rope_copy")
 
 
 def mask_stats(mask: Mask, L: Optional[int] = None, bm: int = 128, bn: int = 64):

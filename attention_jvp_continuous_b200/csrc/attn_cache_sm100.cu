@@ -1,0 +1,590 @@
+// Chunk attention over a key/value cache for B200 (sm_100a): the read-only
+// forward of causal rollout (Causal-rCM report, Sec. 3.2.1 "KV Cache"): the
+// Lq queries of the current chunk attend to the first Lk rows of the cache
+// (the committed prefix the chunk needs, followed by the chunk's own keys
+// at their cache position). O = softmax(c Q K^T) V and LSE per query row.
+//
+// One persistent tcgen05 kernel, one CTA per SM, 384 threads:
+//   warp 0       TMA: Q once per item, K (3 stages) and V (2 stages) of 128
+//                keys; the cache is read through tensor maps whose row
+//                extent is Lk, so rows past the exposed prefix are zero-filled
+//   warp 1       TMEM owner and MMA issuer: S = Q K^T (N = 128) into a
+//                double buffer, O += P V (N = 128, P from TMEM)
+//   warps 4-11   softmax: two warpgroups, each 64 of a tile's 128 keys of
+//                every row, exchanging row maxima; lazy rescale of O (only
+//                when a row max grows by more than 2^8); epilogue
+// Work item = (batch*head, 128-query tile, key split). When the chunk has
+// too few query tiles to fill the GPU the key range is split and every
+// split writes an unnormalised fp32 partial (O, running max, sum) that a
+// second kernel combines; otherwise the epilogue writes O and LSE itself.
+//
+// TMEM: S buffer b at [128 b, 128 b + 128) with the bf16 P packed into its
+// first 64 columns; O at [256, 384). Every mbarrier wait is bounded as in
+// the JVP kernel.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100_pipeline.cuh"
+#include "sm100_ptx.cuh"
+
+namespace jvp {
+namespace cache {
+
+using namespace jvp::ptx;
+using pipe::drain_wait;
+using pipe::ItemRing;
+using pipe::kConsumerThread;
+using pipe::kConsumerWarp;
+using pipe::kProducer;
+using pipe::kRing;
+using pipe::kRingReaders;
+using pipe::wait_bar;
+
+constexpr int BM = 128;  // query rows per tile = TMEM lanes
+constexpr int BN = 128;  // keys per tile
+constexpr int D = 128;
+constexpr int kThreads = 384;
+constexpr float kTau = 8.0f;  // lazy rescale threshold, log2 units
+constexpr uint32_t NK = 3, NV = 2;
+
+constexpr uint32_t kHalf = 128 * 128;   // 16 KB: 128 rows x 64 head-dim columns
+constexpr uint32_t kStage = 2 * kHalf;  // 32 KB: one 128-row operand
+constexpr uint32_t SM_Q = 0;
+constexpr uint32_t SM_K = kStage;
+constexpr uint32_t SM_V = SM_K + NK * kStage;
+constexpr uint32_t SM_BAR = SM_V + NV * kStage;  // 192 KB
+constexpr uint32_t SM_XCHG = SM_BAR + 512;       // softmax exchange
+constexpr uint32_t kSmemBytes = SM_XCHG + 4096 + 1024;
+
+enum : uint32_t {
+  B_QFULL = 0,
+  B_QEMPTY = 1,
+  B_KFULL = 2,    // 3
+  B_KEMPTY = 5,   // 3
+  B_VFULL = 8,    // 2
+  B_VEMPTY = 10,  // 2
+  B_SFULL = 12,   // 2
+  B_PFULL = 14,   // 2
+  B_PVD = 16,     // 2: PV MMAs of the buffer's latest tile complete
+  B_AFREE = 18,   // O read by the epilogue
+  B_DRAIN = 19,
+  B_XMAX = 20,    // 8: [lane quarter][tile parity]
+  B_XSUM = 28,    // 4: [lane quarter]
+  B_IFULL = 32,   // 4
+  B_IEMPTY = 36,  // 4
+  kNumBars = 40
+};
+constexpr uint32_t SM_TMEM_SLOT = SM_BAR + 8 * kNumBars;
+constexpr uint32_t SM_ABORT = SM_TMEM_SLOT + 4;
+constexpr uint32_t SM_RING = SM_ABORT + 4;
+static_assert(SM_RING + 16 <= SM_XCHG, "barrier area overflow");
+static_assert(kSmemBytes <= 232448, "shared memory over the per-block limit");
+
+constexpr uint32_t TM_O = 256;
+constexpr uint32_t IDESC_S = ptx::idesc_bf16(BM, BN, false, false);  // 128 x 128, K-major B
+constexpr uint32_t IDESC_PV = ptx::idesc_bf16(BM, D, false, true);   // 128 x 128, MN-major B
+
+struct Params {
+  const int4* qtiles;  // {qt, seg_begin, seg_count, n_ktiles}; entry = split * n_qt + qt
+  const int2* segs;    // {kt_begin, (count << 1) | partial}
+  int n_entries, n_segs, n_items, n_qt, n_kt;
+  int Lq, Lk;
+  float scale, c2;
+  int split;           // 1: write fp32 partials for the combine kernel
+  __nv_bfloat16* o;    // [B*H, Lq, d]
+  float* lse;          // [B*H, Lq]
+  float* part;         // [n_items, 128, d] unnormalised partial O (split only)
+  float2* ml;          // [n_items, 128] {running max (log2), sum} (split only)
+  unsigned* err;
+  unsigned* item_ctr;
+  unsigned long long wait_limit_ns;
+};
+using Cursor = pipe::Cursor<Params>;
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const base_ptr = smem_raw + (base - raw);
+  auto bar = [&](uint32_t slot) { return base + SM_BAR + 8u * slot; };
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + SM_ABORT);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_QFULL), 1);
+    mbar_init(bar(B_QEMPTY), 1);
+    for (uint32_t s = 0; s < NK; ++s) {
+      mbar_init(bar(B_KFULL + s), 1);
+      mbar_init(bar(B_KEMPTY + s), 1);
+    }
+    for (uint32_t s = 0; s < 2; ++s) {
+      mbar_init(bar(B_VFULL + s), 1);
+      mbar_init(bar(B_VEMPTY + s), 1);
+      mbar_init(bar(B_SFULL + s), 1);
+      mbar_init(bar(B_PFULL + s), 2 * BM);
+      mbar_init(bar(B_PVD + s), 1);
+    }
+    mbar_init(bar(B_AFREE), 2 * BM);
+    mbar_init(bar(B_DRAIN), 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bar(B_XMAX + i), 64);
+    for (int i = 0; i < 4; ++i) mbar_init(bar(B_XSUM + i), 64);
+    for (uint32_t i = 0; i < kRing; ++i) {
+      mbar_init(bar(B_IFULL + i), 1);
+      mbar_init(bar(B_IEMPTY + i), kRingReaders);
+    }
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tm_q);
+    tma_prefetch_map(&tm_k);
+    tma_prefetch_map(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(base + SM_TMEM_SLOT, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base_ptr + SM_TMEM_SLOT);
+  const ItemRing ring{bar(B_IFULL), bar(B_IEMPTY),
+                      reinterpret_cast<volatile int*>(base_ptr + SM_RING), abort_flag};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA ----
+    if (lane == 0) {
+      Cursor c;
+      c.start(p, ring, kProducer);
+      uint32_t q_armed = 0, k_issued = 0, v_issued = 0;
+      bool ok = true;
+      while (c.valid && ok) {
+        if (c.j == 0) {
+          if (c.item_idx > 0) ok = wait_bar(bar(B_QEMPTY), (c.item_idx - 1) & 1, p, abort_flag);
+          if (!ok) break;
+          mbar_expect_tx(bar(B_QFULL), kStage);
+          ++q_armed;
+          const int y = c.qt * BM;
+          tma_load_3d(base + SM_Q, &tm_q, bar(B_QFULL), 0, y, c.bh);
+          tma_load_3d(base + SM_Q + kHalf, &tm_q, bar(B_QFULL), 64, y, c.bh);
+        }
+        const int y = c.kt * BN;
+        const uint32_t sk = c.t % NK, uk = c.t / NK;
+        if (c.t >= NK) ok = wait_bar(bar(B_KEMPTY + sk), (uk - 1) & 1u, p, abort_flag);
+        if (!ok) break;
+        mbar_expect_tx(bar(B_KFULL + sk), kStage);
+        ++k_issued;
+        tma_load_3d(base + SM_K + sk * kStage, &tm_k, bar(B_KFULL + sk), 0, y, c.bh);
+        tma_load_3d(base + SM_K + sk * kStage + kHalf, &tm_k, bar(B_KFULL + sk), 64, y, c.bh);
+        const uint32_t sv = c.t & 1u, uv = c.t >> 1;
+        if (c.t >= NV) ok = wait_bar(bar(B_VEMPTY + sv), (uv - 1) & 1u, p, abort_flag);
+        if (!ok) break;
+        mbar_expect_tx(bar(B_VFULL + sv), kStage);
+        ++v_issued;
+        tma_load_3d(base + SM_V + sv * kStage, &tm_v, bar(B_VFULL + sv), 0, y, c.bh);
+        tma_load_3d(base + SM_V + sv * kStage + kHalf, &tm_v, bar(B_VFULL + sv), 64, y, c.bh);
+        c.next(p, ring, kProducer);
+      }
+      if (!ok || *abort_flag) {
+        if (q_armed) drain_wait(bar(B_QFULL), (q_armed - 1) & 1u);
+        for (uint32_t s = 0; s < NK; ++s) {
+          const uint32_t n = (k_issued + NK - 1 - s) / NK;
+          if (n) drain_wait(bar(B_KFULL + s), (n - 1) & 1u);
+        }
+        for (uint32_t s = 0; s < NV; ++s) {
+          const uint32_t n = (v_issued + NV - 1 - s) / NV;
+          if (n) drain_wait(bar(B_VFULL + s), (n - 1) & 1u);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA ----
+    if (lane == 0) {
+      bool ok = true;
+      const uint64_t q_desc = sdesc_sw128(base + SM_Q, 16, 1024);
+      const uint64_t k_desc = sdesc_sw128(base + SM_K, 16, 1024);     // K-major, stage 0
+      const uint64_t v_desc = sdesc_sw128(base + SM_V, kHalf, 1024);  // MN-major, stage 0
+      auto issue_s = [&](const Cursor& c) -> bool {
+        const uint32_t b = c.t & 1u, sk = c.t % NK;
+        if (c.j == 0 && !wait_bar(bar(B_QFULL), c.item_idx & 1, p, abort_flag)) return false;
+        if (!wait_bar(bar(B_KFULL + sk), (c.t / NK) & 1u, p, abort_flag)) return false;
+        tc_fence_after();
+        const uint64_t kb = k_desc + sk * (kStage >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+          mma_ss(tmem + b * 128u, q_desc + off, kb + off, IDESC_S, kk > 0);
+        }
+        mma_commit(bar(B_SFULL + b));
+        mma_commit(bar(B_KEMPTY + sk));
+        if (c.j == c.n - 1) mma_commit(bar(B_QEMPTY));
+        return true;
+      };
+      auto issue_pv = [&](const Cursor& c) -> bool {
+        const uint32_t b = c.t & 1u;
+        if (c.j == 0 && c.item_idx > 0 &&
+            !wait_bar(bar(B_AFREE), (c.item_idx - 1) & 1, p, abort_flag))
+          return false;
+        if (!wait_bar(bar(B_PFULL + b), (c.t >> 1) & 1u, p, abort_flag)) return false;
+        if (!wait_bar(bar(B_VFULL + b), (c.t >> 1) & 1u, p, abort_flag)) return false;
+        tc_fence_after();
+        const uint64_t vb = v_desc + b * (kStage >> 4);
+        const uint32_t first = c.j == 0 ? 0u : 1u;
+        // O += P V: 8 steps of 16 keys; P's 128 keys are packed in 64 columns.
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks)
+          mma_ts(tmem + TM_O, tmem + b * 128u + ks * 8u, vb + ((ks * 2048) >> 4), IDESC_PV,
+                 first | (ks > 0));
+        mma_commit(bar(B_VEMPTY + b));
+        mma_commit(bar(B_PVD + b));
+        return true;
+      };
+      // Order S(0) S(1) PV(0) S(2) PV(1) ...: S(t+2) overwrites the buffer
+      // whose P PV(t) reads, and one thread's MMAs run in issue order.
+      Cursor cs, cp;
+      cs.start(p, ring, kConsumerThread);
+      cp.start(p, ring, kConsumerThread);
+      for (int pre = 0; pre < 2 && cs.valid && ok; ++pre) {
+        ok = issue_s(cs);
+        cs.next(p, ring, kConsumerThread);
+      }
+      while (cp.valid && ok) {
+        ok = issue_pv(cp);
+        cp.next(p, ring, kConsumerThread);
+        if (ok && cs.valid) {
+          ok = issue_s(cs);
+          cs.next(p, ring, kConsumerThread);
+        }
+      }
+      if (!ok || *abort_flag) {
+        mma_commit(bar(B_DRAIN));
+        drain_wait(bar(B_DRAIN), 0);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ----------------------------------------------------------- softmax ----
+    // Warps 4-7 take keys [0, 64) of every 128-key tile, warps 8-11 keys
+    // [64, 128); warps 4+q and 8+q hold the same rows (TMEM lane quarter q)
+    // and exchange partial row maxima every tile, so both apply one running
+    // max; their partial sums are added at the end.
+    const int hw = (warp - 4) >> 2;
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const uint32_t tl = tmem + (uint32_t(q4 * 32) << 16);
+    float* const xmax = reinterpret_cast<float*>(base_ptr + SM_XCHG);  // [2 parity][2][128]
+    float* const xsum = xmax + 4 * BM;                                 // [2][128]
+    Cursor c;
+    c.start(p, ring, kConsumerWarp);
+    float m_ref = -CUDART_INF_F, l = 0.f;
+    int grow = 0;
+    bool ok = true;
+    while (c.valid) {
+      if (c.j == 0) {
+        grow = c.qt * BM + r;
+        m_ref = -CUDART_INF_F;
+        l = 0.f;
+      }
+      const uint32_t b = c.t & 1u;
+      ok = wait_bar(bar(B_SFULL + b), (c.t >> 1) & 1u, p, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      uint32_t sa[32], sb[32];
+      tmem_ld32(tl + b * 128u + 64u * hw, sa);
+      tmem_ld32(tl + b * 128u + 64u * hw + 32u, sb);
+      tmem_wait_ld();
+      float s[64];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        s[i] = __uint_as_float(sa[i]);
+        s[32 + i] = __uint_as_float(sb[i]);
+      }
+      if (c.partial) {  // the tile holding key Lk - 1: keys past Lk are not in the prefix
+        const int k0 = c.kt * BN + 64 * hw;
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (k0 + i >= p.Lk) s[i] = -CUDART_INF_F;
+      }
+      float m8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+      for (int i = 8; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], s[i]);
+#pragma unroll
+      for (int w2 = 4; w2 > 0; w2 >>= 1)
+#pragma unroll
+        for (int i = 0; i < w2; ++i) m8[i] = fmaxf(m8[i], m8[i + w2]);
+      xmax[(b * 2u + hw) * BM + r] = m8[0];
+      // The exchange also orders TMEM: warpgroup 1 writes its P over S
+      // columns [32, 64) that warpgroup 0 has just read.
+      tc_fence_before();
+      mbar_arrive(bar(B_XMAX + q4 * 2 + b));
+      ok = wait_bar(bar(B_XMAX + q4 * 2 + b), (c.t >> 1) & 1u, p, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const float mxs = fmaxf(m8[0], xmax[(b * 2u + (hw ^ 1)) * BM + r]) * p.c2;
+      float alpha = 1.f;
+      bool need = false;
+      if (m_ref == -CUDART_INF_F) {
+        m_ref = mxs;  // first tile of the item: nothing accumulated yet
+      } else if (mxs > m_ref + kTau) {
+        alpha = ex2(m_ref - mxs);
+        m_ref = mxs;
+        need = true;
+      }
+      if (__any_sync(0xffffffffu, need)) {
+        l *= alpha;
+        // O holds PV(t-1); wait for it, then scale this warpgroup's half.
+        // (PV(t-3), the previous phase of that barrier, completed before
+        // S(t-1) was issued.)
+        ok = wait_bar(bar(B_PVD + ((c.t - 1) & 1u)), ((c.t - 1) >> 1) & 1u, p, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int q = 0; q < 2; ++q) {
+          const uint32_t col = TM_O + 64u * hw + 32u * q;
+          uint32_t a[32];
+          tmem_ld32(tl + col, a);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) * alpha);
+          tmem_st32(tl + col, a);
+        }
+        tmem_wait_st();
+      }
+      // e = 2^(c2 s - m) in packed pairs; bf16 P into this warpgroup's 32
+      // columns of the buffer (keys 64 hw .. 64 hw + 63).
+      const uint64_t c2v = f2pack(p.c2, p.c2), mv = f2pack(-m_ref, -m_ref);
+      uint64_t la = 0, lb = 0;
+      uint32_t pp[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        float x0, x1;
+        f2unpack(fma2(f2pack(s[2 * i], s[2 * i + 1]), c2v, mv), x0, x1);
+        const float e0 = ex2(x0), e1 = ex2(x1);
+        if (i & 1) lb = add2(lb, f2pack(e0, e1));
+        else la = add2(la, f2pack(e0, e1));
+        pp[i] = pack_bf16(e0, e1);
+      }
+      {
+        float u0, u1;
+        f2unpack(add2(la, lb), u0, u1);
+        l += u0 + u1;
+      }
+      tmem_st32(tl + b * 128u + 32u * hw, pp);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_PFULL + b));
+
+      if (c.j == c.n - 1) {
+        // ------------------------------------------------------ epilogue --
+        // PV(t) done; PV(t-2), the previous phase of this barrier, completed
+        // before S(t) was issued.
+        ok = wait_bar(bar(B_PVD + (c.t & 1u)), (c.t >> 1) & 1u, p, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        xsum[hw * BM + r] = l;
+        mbar_arrive(bar(B_XSUM + q4));
+        ok = wait_bar(bar(B_XSUM + q4), c.item_idx & 1, p, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        const float lt = l + xsum[(hw ^ 1) * BM + r];
+        tc_fence_after();
+        const bool row_ok = grow < p.Lq;
+#pragma unroll 1
+        for (int cc = 0; cc < 2; ++cc) {
+          const uint32_t col = 64u * hw + 32u * cc;
+          uint32_t a[32];
+          tmem_ld32(tl + TM_O + col, a);
+          tmem_wait_ld();
+          if (!p.split) {
+            const float inv = lt > 0.f ? 1.f / lt : 0.f;
+            uint32_t po[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              po[i] = pack_bf16(__uint_as_float(a[2 * i]) * inv,
+                                __uint_as_float(a[2 * i + 1]) * inv);
+            if (row_ok) {
+              uint4* go = reinterpret_cast<uint4*>(p.o + (size_t(c.bh) * p.Lq + grow) * D + col);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                go[i] = make_uint4(po[4 * i], po[4 * i + 1], po[4 * i + 2], po[4 * i + 3]);
+            }
+          } else {
+            // Unnormalised partial of this key split, for every row of the
+            // tile (rows past Lq are never combined).
+            float4* dst = reinterpret_cast<float4*>(p.part + (size_t(c.item) * BM + r) * D + col);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(a[4 * i]), __uint_as_float(a[4 * i + 1]),
+                                   __uint_as_float(a[4 * i + 2]), __uint_as_float(a[4 * i + 3]));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(B_AFREE));
+        if (hw == 0) {
+          if (p.split)
+            p.ml[size_t(c.item) * BM + r] = make_float2(m_ref, lt);
+          else if (row_ok)
+            p.lse[size_t(c.bh) * p.Lq + grow] =
+                lt > 0.f ? (m_ref + log2f(lt)) * 0.69314718055994531f : -CUDART_INF_F;
+        }
+      }
+      c.next(p, ring, kConsumerWarp);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Combines the key splits of each query row: with per-split running max m_s
+// (log2 units of the scaled score), sum l_s and unnormalised partial O_s,
+//   M = max m_s,  w_s = 2^(m_s - M),  O = sum w_s O_s / sum w_s l_s,
+//   LSE = (M + log2 sum w_s l_s) ln 2.
+// One warp per (batch*head, query row), 4 head-dim columns per lane.
+__global__ void __launch_bounds__(256)
+attn_cache_combine_kernel(const float* __restrict__ part, const float2* __restrict__ ml,
+                          __nv_bfloat16* __restrict__ o, float* __restrict__ lse, int BH,
+                          int Lq, int n_qt, int n_entries, int splits) {
+  const int lane = threadIdx.x & 31;
+  const long long n_rows = (long long)BH * Lq;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < n_rows;
+       w += warps) {
+    const int bh = int(w / Lq), i = int(w % Lq);
+    const int qt = i / BM, r = i % BM;
+    float M = -CUDART_INF_F;
+    for (int s = 0; s < splits; ++s) {
+      const size_t item = size_t(bh) * n_entries + size_t(s) * n_qt + qt;
+      M = fmaxf(M, ml[item * BM + r].x);
+    }
+    float lsum = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < splits; ++s) {
+      const size_t item = size_t(bh) * n_entries + size_t(s) * n_qt + qt;
+      const float2 v = ml[item * BM + r];
+      const float ws = v.x == -CUDART_INF_F ? 0.f : exp2f(v.x - M);
+      lsum += ws * v.y;
+      const float4 pv = reinterpret_cast<const float4*>(part + (item * BM + r) * D)[lane];
+      acc.x += ws * pv.x;
+      acc.y += ws * pv.y;
+      acc.z += ws * pv.z;
+      acc.w += ws * pv.w;
+    }
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    uint2 packed;
+    packed.x = pack_bf16(acc.x * inv, acc.y * inv);
+    packed.y = pack_bf16(acc.z * inv, acc.w * inv);
+    reinterpret_cast<uint2*>(o + (size_t(bh) * Lq + i) * D)[lane] = packed;
+    if (lane == 0)
+      lse[size_t(bh) * Lq + i] =
+          lsum > 0.f ? (M + log2f(lsum)) * 0.69314718055994531f : -CUDART_INF_F;
+  }
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [BH, rows_alloc, 128] bf16 with `rows` readable rows per (b, h): the map's
+// row extent is `rows`, so reads past it are zero-filled.
+static bool make_map(CUtensorMap* m, const void* ptr, int rows, int rows_alloc, int BH) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(rows), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(rows_alloc) * D * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace cache
+
+int launch_cache_sm100(const CacheArgs& a, const WorkList& w, int splits, int num_sms) {
+  using namespace cache;
+  const int BH = a.B * a.H;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, a.q, a.Lq, a.Lq, BH) || !make_map(&mk, a.k, a.Lk, a.Lcache, BH) ||
+      !make_map(&mv, a.v, a.Lk, a.Lcache, BH))
+    return JVP_ERR_LAUNCH_FAILED;
+  Params p;
+  p.qtiles = w.qtiles;
+  p.segs = w.segs;
+  p.n_entries = w.n_qtiles;
+  p.n_segs = w.n_segs;
+  const long long items = (long long)w.n_qtiles * BH;
+  if (items > 0x7fffffffLL) return JVP_ERR_TOO_LARGE;
+  p.n_items = int(items);
+  p.n_qt = (a.Lq + BM - 1) / BM;
+  p.n_kt = (a.Lk + BN - 1) / BN;
+  p.Lq = a.Lq;
+  p.Lk = a.Lk;
+  p.scale = a.scale;
+  p.c2 = a.scale * 1.4426950408889634f;
+  p.split = splits > 1 ? 1 : 0;
+  p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.lse = a.lse;
+  p.part = a.part;
+  p.ml = reinterpret_cast<float2*>(a.ml);
+  p.err = a.err;
+  p.item_ctr = a.item_ctr;
+  p.wait_limit_ns = a.wait_limit_ns;
+  if (p.split && (!p.part || !p.ml)) return JVP_ERR_LAUNCH_FAILED;
+  static std::mutex attr_mu;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return JVP_ERR_LAUNCH_FAILED;
+  {
+    std::lock_guard<std::mutex> lk(attr_mu);
+    if (!attr_done[dev]) {
+      if (cudaFuncSetAttribute(attn_cache_sm100_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kSmemBytes) != cudaSuccess)
+        return JVP_ERR_LAUNCH_FAILED;
+      attr_done[dev] = true;
+    }
+  }
+  const int grid = int(items < num_sms ? items : num_sms);
+  if (!a.item_ctr || cudaMemsetAsync(a.item_ctr, 0, sizeof(unsigned), a.stream) != cudaSuccess)
+    return JVP_ERR_LAUNCH_FAILED;
+  attn_cache_sm100_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mv, p);
+  if (cudaGetLastError() != cudaSuccess) return JVP_ERR_LAUNCH_FAILED;
+  if (p.split) {
+    const long long rows = (long long)BH * a.Lq;
+    const long long blocks = (rows + 7) / 8;  // 8 warps per block
+    const int cgrid = int(blocks < 8LL * num_sms ? blocks : 8LL * num_sms);
+    attn_cache_combine_kernel<<<cgrid, 256, 0, a.stream>>>(p.part, p.ml, p.o, p.lse, BH, a.Lq,
+                                                           p.n_qt, p.n_entries, splits);
+    if (cudaGetLastError() != cudaSuccess) return JVP_ERR_LAUNCH_FAILED;
+  }
+  return JVP_OK;
+}
+
+}  // namespace jvp

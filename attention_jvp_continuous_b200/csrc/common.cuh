@@ -61,6 +61,36 @@ struct BwdArgs {
 // work list (128 x 64 grid); wkv: key-tile work list (64 x 128 grid).
 int launch_bwd_sm100(const BwdArgs& a, const WorkList& wq, const WorkList& wkv, int num_sms);
 
+// Chunk attention over a key/value cache (jvp_attn_cache_fwd): bf16, d = 128.
+struct CacheArgs {
+  const void *q, *k, *v;  // q [B, H, Lq, d]; k, v caches [B, H, Lcache, d]
+  void* o;                // [B, H, Lq, d]
+  float* lse;             // [B, H, Lq]
+  int B, H, Lq, Lk, Lcache;
+  float scale;
+  cudaStream_t stream;
+  unsigned* err;
+  unsigned* item_ctr;
+  unsigned long long wait_limit_ns;
+  float* part;  // split > 1: [items, 128, 128] fp32 partial outputs
+  float* ml;    // split > 1: [items, 128] {max, sum} pairs
+};
+
+// w: dense split work list (build_schedule_dense with 128 x 128 tiles).
+int launch_cache_sm100(const CacheArgs& a, const WorkList& w, int splits, int num_sms);
+
+// Row copy with optional rotary embedding (jvp_attn_rope_copy).
+struct RopeArgs {
+  const void* src;
+  void* dst;
+  int B, H, src_rows, dst_rows, rows, src_row0, dst_row0, d;
+  bool bf16;
+  const float *cos, *sin;  // both null: plain copy
+  int rope_row0;
+  cudaStream_t stream;
+};
+int launch_rope_copy(const RopeArgs& a, int num_sms);
+
 // Per-wait limit for the tensor-core kernel (jvp_attn_set_wait_limit).
 unsigned long long wait_limit_ns();
 

@@ -35,7 +35,9 @@ struct DevInfo {
 };
 
 struct WsKey {
-  int dev, mode, T, F, chunk, L, bm, bn, kind;  // kind 0: query-tile list, 1: key-tile list
+  // kind 0: query-tile list, 1: key-tile list (mask fields), 2: dense split
+  // list for cache attention (T = splits, chunk = Lq, L = Lk).
+  int dev, mode, T, F, chunk, L, bm, bn, kind;
   bool operator<(const WsKey& o) const {
     return std::tie(dev, mode, T, F, chunk, L, bm, bn, kind) <
            std::tie(o.dev, o.mode, o.T, o.F, o.chunk, o.L, o.bm, o.bn, o.kind);
@@ -53,6 +55,9 @@ std::map<WsKey, Ws> g_ws;
 // Work-item counter of the tensor-core kernel, one per (device, stream):
 // launches on one stream are ordered, so they can share it.
 std::map<std::pair<int, cudaStream_t>, unsigned*> g_ctr;
+// Split-K partial results of cache attention, per (device, stream), grown
+// on demand: {buffer, bytes}.
+std::map<std::pair<int, cudaStream_t>, std::pair<void*, size_t>> g_part;
 
 int device_info(DevInfo** out) {
   int dev = 0;
@@ -80,17 +85,9 @@ int device_info(DevInfo** out) {
   return JVP_OK;
 }
 
-int get_worklist(int dev, const jvp_mask_desc& m, int L, WorkList* out, int bm = kBM,
-                 int bn = kBN, int kind = 0) {
-  const WsKey key{dev, m.mode, m.tokens_per_frame, m.n_frames,
-                  m.chunk, L, bm, bn, kind};
-  std::lock_guard<std::mutex> lk(g_mu);
-  auto it = g_ws.find(key);
-  if (it != g_ws.end()) {
-    *out = it->second.w;
-    return JVP_OK;
-  }
-  const Schedule s = kind == 0 ? build_schedule(m, L, bm, bn) : build_schedule_kv(m, L, bm, bn);
+// Copies a host schedule into a new device buffer and caches it under key.
+// Caller holds g_mu.
+int upload_schedule(const WsKey& key, const Schedule& s, WorkList* out) {
   const size_t qbytes = s.qtiles.size() * sizeof(int32_t);
   const size_t sbytes = s.segs.size() * sizeof(int32_t);
   const size_t soff = (qbytes + 255) & ~size_t(255);
@@ -112,6 +109,74 @@ int get_worklist(int dev, const jvp_mask_desc& m, int L, WorkList* out, int bm =
   g_ws[key] = ws;
   *out = ws.w;
   return JVP_OK;
+}
+
+int get_worklist(int dev, const jvp_mask_desc& m, int L, WorkList* out, int bm = kBM,
+                 int bn = kBN, int kind = 0) {
+  const WsKey key{dev, m.mode, m.tokens_per_frame, m.n_frames,
+                  m.chunk, L, bm, bn, kind};
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_ws.find(key);
+  if (it != g_ws.end()) {
+    *out = it->second.w;
+    return JVP_OK;
+  }
+  const Schedule s = kind == 0 ? build_schedule(m, L, bm, bn) : build_schedule_kv(m, L, bm, bn);
+  return upload_schedule(key, s, out);
+}
+
+int get_worklist_dense(int dev, int Lq, int Lk, int splits, WorkList* out) {
+  const WsKey key{dev, -1, splits, 0, Lq, Lk, 128, 128, 2};
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_ws.find(key);
+  if (it != g_ws.end()) {
+    *out = it->second.w;
+    return JVP_OK;
+  }
+  return upload_schedule(key, build_schedule_dense(Lq, Lk, 128, 128, splits), out);
+}
+
+// Partial-result workspace of at least `bytes` for (dev, st).
+int get_partials(int dev, cudaStream_t st, size_t bytes, void** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto& e = g_part[std::make_pair(dev, st)];
+  if (e.first && e.second >= bytes) {
+    *out = e.first;
+    return JVP_OK;
+  }
+  if (e.first) {
+    // Earlier launches on this stream may still read the old buffer.
+    if (cudaStreamSynchronize(st) != cudaSuccess || cudaFree(e.first) != cudaSuccess)
+      return JVP_ERR_LAUNCH_FAILED;
+    e.first = nullptr;
+    e.second = 0;
+  }
+  if (cudaMalloc(&e.first, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    e.first = nullptr;
+    return JVP_ERR_OUT_OF_MEMORY;
+  }
+  e.second = bytes;
+  *out = e.first;
+  return JVP_OK;
+}
+
+// Key splits for cache attention: `units` = B*H*query tiles; minimises
+// waves(S) * (tiles per split + 2), the +2 standing for a split's partial
+// write and combine; ties go to fewer splits.
+int choose_splits(long long units, int n_kt, int sms) {
+  int best = 1;
+  double best_cost = 1e300;
+  const int smax = n_kt < 64 ? n_kt : 64;
+  for (int sp = 1; sp <= smax; ++sp) {
+    const long long waves = (units * sp + sms - 1) / sms;
+    const double cost = double(waves) * (double(n_kt) / sp + (sp > 1 ? 2.0 : 0.0));
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = sp;
+    }
+  }
+  return best;
 }
 
 int get_counter(int dev, cudaStream_t st, unsigned** out) {
@@ -245,6 +310,87 @@ int64_t jvp_attn_bwd_scratch_len(int B, int H, int L) {
   return 2 * int64_t(B) * H * Lp;
 }
 
+int jvp_attn_cache_fwd(const void* q, const void* k_cache, const void* v_cache, void* o,
+                       float* lse, int B, int H, int Lq, int Lk, int Lcache, int d,
+                       jvp_dtype dtype, float softmax_scale, void* stream) {
+  if (!q || !k_cache || !v_cache || !o || !lse) return JVP_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || Lq <= 0 || Lk <= 0 || Lcache < Lk || d <= 0 || dtype != JVP_BF16)
+    return JVP_ERR_INVALID_ARG;
+  if (std::isnan(softmax_scale) || std::isinf(softmax_scale)) return JVP_ERR_INVALID_ARG;
+  if (d != 128) return JVP_ERR_UNSUPPORTED_HEAD_DIM;
+  if ((long long)B * H * Lq >= (1LL << 31) || (long long)B * H * Lcache >= (1LL << 31))
+    return JVP_ERR_TOO_LARGE;
+  const void* ptrs[] = {q, k_cache, v_cache, o, lse};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return JVP_ERR_MISALIGNED;
+  DevInfo* di = nullptr;
+  int rc = device_info(&di);
+  if (rc != JVP_OK) return rc;
+  if (di->major != 10 || di->minor != 0) return JVP_ERR_UNSUPPORTED_DEVICE;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  CacheArgs a;
+  a.q = q; a.k = k_cache; a.v = v_cache; a.o = o; a.lse = lse;
+  a.B = B; a.H = H; a.Lq = Lq; a.Lk = Lk; a.Lcache = Lcache;
+  a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(d));
+  a.stream = static_cast<cudaStream_t>(stream);
+  a.err = di->err;
+  a.wait_limit_ns = wait_limit_ns();
+  a.part = nullptr;
+  a.ml = nullptr;
+  const int n_qt = (Lq + 127) / 128, n_kt = (Lk + 127) / 128;
+  const int splits = choose_splits((long long)B * H * n_qt, n_kt, di->sms);
+  WorkList w;
+  rc = get_worklist_dense(dev, Lq, Lk, splits, &w);
+  if (rc != JVP_OK) return rc;
+  if (splits > 1) {
+    const size_t items = size_t(B) * H * n_qt * splits;
+    const size_t part_bytes = items * 128 * 128 * sizeof(float);
+    void* buf = nullptr;
+    rc = get_partials(dev, a.stream, part_bytes + items * 128 * 2 * sizeof(float), &buf);
+    if (rc != JVP_OK) return rc;
+    a.part = static_cast<float*>(buf);
+    a.ml = reinterpret_cast<float*>(static_cast<char*>(buf) + part_bytes);
+  }
+  rc = get_counter(dev, a.stream, &a.item_ctr);
+  if (rc != JVP_OK) return rc;
+  return launch_cache_sm100(a, w, splits, di->sms);
+}
+
+int jvp_attn_rope_copy(const void* src, void* dst, int B, int H, int src_rows, int dst_rows,
+                       int rows, int src_row0, int dst_row0, int d, jvp_dtype dtype,
+                       const float* rope_cos, const float* rope_sin, int rope_rows,
+                       int rope_row0, void* stream) {
+  if (!src || !dst || B <= 0 || H <= 0 || d <= 0 || rows < 0 || src_row0 < 0 || dst_row0 < 0)
+    return JVP_ERR_INVALID_ARG;
+  if (dtype != JVP_BF16 && dtype != JVP_FP32) return JVP_ERR_INVALID_ARG;
+  if (d % (dtype == JVP_BF16 ? 8 : 4) != 0) return JVP_ERR_INVALID_ARG;
+  if ((long long)src_row0 + rows > src_rows || (long long)dst_row0 + rows > dst_rows)
+    return JVP_ERR_INVALID_ARG;
+  if ((rope_cos == nullptr) != (rope_sin == nullptr)) return JVP_ERR_INVALID_ARG;
+  if (rope_cos && (rope_row0 < 0 || (long long)rope_row0 + rows > rope_rows))
+    return JVP_ERR_INVALID_ARG;
+  if ((long long)B * H * (src_rows > dst_rows ? src_rows : dst_rows) * d >= (1LL << 40))
+    return JVP_ERR_TOO_LARGE;
+  if (src == dst && src_row0 != dst_row0) return JVP_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(dst) || (rope_cos && (!aligned16(rope_cos) ||
+                                                          !aligned16(rope_sin))))
+    return JVP_ERR_MISALIGNED;
+  if (rows == 0) return JVP_OK;
+  DevInfo* di = nullptr;
+  int rc = device_info(&di);
+  if (rc != JVP_OK) return rc;
+  if (di->major != 10 || di->minor != 0) return JVP_ERR_UNSUPPORTED_DEVICE;
+  RopeArgs a;
+  a.src = src; a.dst = dst; a.B = B; a.H = H;
+  a.src_rows = src_rows; a.dst_rows = dst_rows; a.rows = rows;
+  a.src_row0 = src_row0; a.dst_row0 = dst_row0; a.d = d;
+  a.bf16 = dtype == JVP_BF16;
+  a.cos = rope_cos; a.sin = rope_sin; a.rope_row0 = rope_row0;
+  a.stream = static_cast<cudaStream_t>(stream);
+  return launch_rope_copy(a, di->sms);
+}
+
 int jvp_attn_schedule_kv(jvp_mask_desc mask, int L, int bq, int bk, int32_t* ktiles,
                          int ktile_cap, int32_t* segs, int seg_cap, int* n_ktiles, int* n_segs) {
   int rc = validate_mask(mask, L);
@@ -353,6 +499,13 @@ int jvp_attn_release(void) {
       rc = JVP_ERR_LAUNCH_FAILED;
   }
   g_ctr.clear();
+  for (auto& kv : g_part) {
+    if (!kv.second.first) continue;
+    if (cudaSetDevice(kv.first.first) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess ||
+        cudaFree(kv.second.first) != cudaSuccess)
+      rc = JVP_ERR_LAUNCH_FAILED;
+  }
+  g_part.clear();
   if (have_dev) cudaSetDevice(cur);
   return rc;
 }

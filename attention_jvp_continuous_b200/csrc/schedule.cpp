@@ -251,4 +251,41 @@ Schedule build_schedule_kv(const jvp_mask_desc& m, int L, int bq, int bk) {
   return s;
 }
 
+Schedule build_schedule_dense(int Lq, int Lk, int bq, int bk, int splits) {
+  Schedule s;
+  s.L = Lk;
+  s.bm = bq;
+  s.bn = bk;
+  s.n_qt = (Lq + bq - 1) / bq;
+  s.n_kt = (Lk + bk - 1) / bk;
+  const bool ragged = Lk % bk != 0;
+  for (int sp = 0; sp < splits; ++sp) {
+    const int k0 = int(int64_t(sp) * s.n_kt / splits);
+    const int k1 = int(int64_t(sp + 1) * s.n_kt / splits);
+    const int seg_begin = int(s.segs.size() / 2);
+    int nseg = 0;
+    const int full_end = (ragged && k1 == s.n_kt) ? k1 - 1 : k1;
+    if (full_end > k0) {
+      s.segs.push_back(k0);
+      s.segs.push_back((full_end - k0) << 1);
+      ++nseg;
+    }
+    if (full_end < k1) {
+      s.segs.push_back(full_end);
+      s.segs.push_back((1 << 1) | 1);
+      ++nseg;
+    }
+    s.max_ktiles = std::max<int64_t>(s.max_ktiles, k1 - k0);
+    for (int qt = 0; qt < s.n_qt; ++qt) {
+      s.qtiles.push_back(qt);
+      s.qtiles.push_back(seg_begin);
+      s.qtiles.push_back(nseg);
+      s.qtiles.push_back(k1 - k0);
+      s.n_full += full_end - k0;
+      s.n_partial += k1 - full_end;
+    }
+  }
+  return s;
+}
+
 }  // namespace jvp

@@ -48,6 +48,15 @@ Schedule build_schedule(const jvp_mask_desc& m, int L, int bm, int bn);
 // here, since the pass reads per-query LSE and D values).
 Schedule build_schedule_kv(const jvp_mask_desc& m, int L, int bq, int bk);
 
+// Dense rectangular work list for chunk attention over a key/value cache:
+// Lq query rows against the first Lk keys, all admitted. The key tiles of
+// bk keys are cut into `splits` contiguous ranges of near-equal length
+// (split s: tiles [s n_kt / splits, (s+1) n_kt / splits)); entry e = s *
+// n_qt + qt covers query tile qt of split s: {qt, seg_begin, seg_count,
+// n_ktiles}. The last key tile is PARTIAL when Lk is not a multiple of bk
+// (its own segment); all others are FULL. Requires 1 <= splits <= n_kt.
+Schedule build_schedule_dense(int Lq, int Lk, int bq, int bk, int splits);
+
 // The same work list as build_schedule (same entries, same order), written
 // into caller-provided arrays without any heap allocation: entries of 4
 // int32 to `qtiles`, segments of 2 int32 ({kt_begin, (count << 1) |

@@ -204,6 +204,58 @@ int jvp_attn_bwd(const void* q, const void* k, const void* v, const void* o,
  */
 int64_t jvp_attn_bwd_scratch_len(int B, int H, int L);
 
+/* ---- key/value cache: read-only chunk attention and appends ------------- */
+/*
+ * jvp_attn_cache_fwd: the read-only forward of causal rollout (Causal-rCM
+ * report, Sec. 3.2.1 "KV Cache"): the Lq query rows of the current chunk
+ * attend to the first Lk rows of a key/value cache, i.e. the committed
+ * prefix the chunk needs followed by the chunk's own keys, which the caller
+ * has written at their cache position (jvp_attn_rope_copy). With noisy
+ * context (Sec. 3.1.3) the committed rows are those of the last denoising
+ * forward; the operation is the same.
+ *
+ *   o = softmax(c q k[0:Lk]^T) v[0:Lk],  lse = log sum exp(c q k[0:Lk]^T)
+ *
+ * q        [B, H, Lq, d] bf16            o    [B, H, Lq, d] bf16 (output)
+ * k_cache, v_cache [B, H, Lcache, d] bf16 (rows Lk..Lcache-1 are not read;
+ *          the kernel's tensor maps stop at Lk)
+ * lse      [B, H, Lq] float32, natural log (output)
+ * softmax_scale <= 0 selects 1/sqrt(d). Requires 1 <= Lk <= Lcache, Lq >= 1,
+ * dtype JVP_BF16 (else JVP_ERR_INVALID_ARG) and d = 128 (else
+ * JVP_ERR_UNSUPPORTED_HEAD_DIM); all pointers 16-byte aligned. When the
+ * chunk has too few 128-row query tiles to fill the GPU the key range is
+ * split across CTAs and a second kernel combines the splits; the library
+ * keeps the partial-result workspace per (device, stream), grows it when a
+ * larger call needs it (JVP_ERR_OUT_OF_MEMORY on failure) and frees it in
+ * jvp_attn_release. Asynchronous on `stream`; errors as jvp_attn_fwd.
+ */
+int jvp_attn_cache_fwd(const void* q, const void* k_cache, const void* v_cache, void* o,
+                       float* lse, int B, int H, int Lq, int Lk, int Lcache, int d,
+                       jvp_dtype dtype, float softmax_scale, void* stream);
+
+/*
+ * jvp_attn_rope_copy: copies rows [src_row0, src_row0 + rows) of every
+ * (b, h) slice of src [B, H, src_rows, d] to rows [dst_row0, dst_row0 +
+ * rows) of dst [B, H, dst_rows, d] (same dtype), optionally rotating them
+ * with rotary position embedding (Sec. 3.2.1: post-RoPE caching rotates
+ * keys once when they are appended; pre-RoPE caching stores them unrotated
+ * and rotates the exposed prefix into a working buffer before a read).
+ * With rope_cos and rope_sin (both non-null, float32 [rope_rows, d/2]), row
+ * j of the range is rotated by table row rope_row0 + j: each pair
+ * (x_2i, x_2i+1) becomes (x_2i c - x_2i+1 s, x_2i s + x_2i+1 c), computed
+ * in fp32 and rounded once. Both null: a plain copy (values, or keys of a
+ * pre-RoPE cache). src and dst may be the same buffer only with identical
+ * row ranges (in place); otherwise the ranges must not overlap.
+ * Requires rows >= 0 (0: nothing to do), src_row0 + rows <= src_rows,
+ * dst_row0 + rows <= dst_rows, rope_row0 + rows <= rope_rows, d a multiple
+ * of 8 (bf16) or 4 (fp32), 16-byte aligned src/dst and tables (else
+ * JVP_ERR_INVALID_ARG / JVP_ERR_MISALIGNED). Asynchronous on `stream`.
+ */
+int jvp_attn_rope_copy(const void* src, void* dst, int B, int H, int src_rows, int dst_rows,
+                       int rows, int src_row0, int dst_row0, int d, jvp_dtype dtype,
+                       const float* rope_cos, const float* rope_sin, int rope_rows,
+                       int rope_row0, void* stream);
+
 /* ---- host-side mask / schedule queries (no GPU needed) ------------------- */
 /*
  * jvp_attn_mask_stats: for the mask on L tokens and a bm x bn tile grid

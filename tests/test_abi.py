@@ -98,3 +98,65 @@ def test_python_wrapper_rejects_cpu_tensors():
 def test_error_type_carries_code():
     e = _lib.JvpAttnError(_lib.JVP_ERR_SHAPE_MISMATCH, "where")
     assert e.code == -2 and "mask descriptor" in str(e)
+
+
+FAKE = 1 << 20  # 16-byte aligned dummy device address; never dereferenced on error paths
+
+
+def call_cache(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, H=2, Lq=100, Lk=500, Lcache=512,
+             d=128, dtype=_lib.JVP_BF16, scale=0.0)
+    a.update(kw)
+    fp = ctypes.POINTER(ctypes.c_float)
+    return _lib.lib().jvp_attn_cache_fwd(a["q"], a["k"], a["v"], a["o"],
+                                         ctypes.cast(a["lse"], fp), a["B"], a["H"], a["Lq"],
+                                         a["Lk"], a["Lcache"], a["d"], a["dtype"], a["scale"],
+                                         None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), _lib.JVP_ERR_INVALID_ARG),
+    (dict(Lk=0), _lib.JVP_ERR_INVALID_ARG),
+    (dict(Lk=513), _lib.JVP_ERR_INVALID_ARG),
+    (dict(Lq=0), _lib.JVP_ERR_INVALID_ARG),
+    (dict(dtype=_lib.JVP_FP32), _lib.JVP_ERR_INVALID_ARG),
+    (dict(d=64), _lib.JVP_ERR_UNSUPPORTED_HEAD_DIM),
+    (dict(scale=float("inf")), _lib.JVP_ERR_INVALID_ARG),
+    (dict(o=FAKE + 8), _lib.JVP_ERR_MISALIGNED),
+])
+def test_cache_fwd_argument_errors(kw, code):
+    assert call_cache(**kw) == code
+
+
+def call_rope(**kw):
+    a = dict(src=FAKE, dst=FAKE + (1 << 16), B=1, H=2, src_rows=64, dst_rows=128, rows=32,
+             src_row0=0, dst_row0=96, d=128, dtype=_lib.JVP_BF16, cos=FAKE, sin=FAKE,
+             rope_rows=40, rope_row0=8)
+    a.update(kw)
+    fp = ctypes.POINTER(ctypes.c_float)
+    cvt = lambda x: ctypes.cast(x, fp) if x else None  # noqa: E731
+    return _lib.lib().jvp_attn_rope_copy(a["src"], a["dst"], a["B"], a["H"], a["src_rows"],
+                                         a["dst_rows"], a["rows"], a["src_row0"],
+                                         a["dst_row0"], a["d"], a["dtype"], cvt(a["cos"]),
+                                         cvt(a["sin"]), a["rope_rows"], a["rope_row0"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dst_row0=97), _lib.JVP_ERR_INVALID_ARG),           # past the destination rows
+    (dict(src_row0=33), _lib.JVP_ERR_INVALID_ARG),           # past the source rows
+    (dict(rope_row0=9), _lib.JVP_ERR_INVALID_ARG),           # past the table
+    (dict(sin=0), _lib.JVP_ERR_INVALID_ARG),                 # one table only
+    (dict(d=100), _lib.JVP_ERR_INVALID_ARG),                 # bf16 rows of 16-byte vectors
+    (dict(rows=-1), _lib.JVP_ERR_INVALID_ARG),
+    (dict(dst=FAKE, dst_row0=90), _lib.JVP_ERR_INVALID_ARG),  # overlapping, not in place
+    (dict(src=FAKE + 4), _lib.JVP_ERR_MISALIGNED),
+    (dict(rows=0), _lib.JVP_OK),                              # nothing to do, no device touched
+])
+def test_rope_copy_argument_errors(kw, code):
+    assert call_rope(**kw) == code
+
+
+def test_bwd_scratch_len():
+    assert _lib.lib().jvp_attn_bwd_scratch_len(1, 12, 65520) == 2 * 12 * 65536
+    assert _lib.lib().jvp_attn_bwd_scratch_len(2, 3, 1) == 2 * 6 * 128
+    assert _lib.lib().jvp_attn_bwd_scratch_len(0, 1, 1) == -1
