@@ -11,16 +11,17 @@
 //   warp 1       TMEM owner and MMA issuer: S = Q K^T (N = 128) into a
 //                double buffer, O += P V (N = 128, P from TMEM)
 //   warps 4-11   softmax: two warpgroups, each 64 of a tile's 128 keys of
-//                every row, exchanging row maxima; lazy rescale of O (only
-//                when a row max grows by more than 2^8); epilogue
+//                every row with its own running max and its own O
+//                accumulator (lazy rescale only when its row max grows by
+//                more than 2^8); the epilogue merges the two halves
 // Work item = (batch*head, 128-query tile, key split). When the chunk has
 // too few query tiles to fill the GPU the key range is split and every
 // split writes an unnormalised fp32 partial (O, running max, sum) that a
 // second kernel combines; otherwise the epilogue writes O and LSE itself.
 //
-// TMEM: S buffer b at [128 b, 128 b + 128) with the bf16 P packed into its
-// first 64 columns; O at [256, 384). Every mbarrier wait is bounded as in
-// the JVP kernel.
+// TMEM: S buffer b at [128 b, 128 b + 128), the bf16 P of each key half
+// packed over the start of that half's S columns; O_a at [256, 384) and O_b
+// at [384, 512). Every mbarrier wait is bounded as in the JVP kernel.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -73,11 +74,10 @@ enum : uint32_t {
   B_PVD = 16,     // 2: PV MMAs of the buffer's latest tile complete
   B_AFREE = 18,   // O read by the epilogue
   B_DRAIN = 19,
-  B_XMAX = 20,    // 8: [lane quarter][tile parity]
-  B_XSUM = 28,    // 4: [lane quarter]
-  B_IFULL = 32,   // 4
-  B_IEMPTY = 36,  // 4
-  kNumBars = 40
+  B_XSUM = 20,    // 4: [lane quarter], end-of-item merge of the halves
+  B_IFULL = 24,   // 4
+  B_IEMPTY = 28,  // 4
+  kNumBars = 32
 };
 constexpr uint32_t SM_TMEM_SLOT = SM_BAR + 8 * kNumBars;
 constexpr uint32_t SM_ABORT = SM_TMEM_SLOT + 4;
@@ -85,7 +85,10 @@ constexpr uint32_t SM_RING = SM_ABORT + 4;
 static_assert(SM_RING + 16 <= SM_XCHG, "barrier area overflow");
 static_assert(kSmemBytes <= 232448, "shared memory over the per-block limit");
 
-constexpr uint32_t TM_O = 256;
+// Two O accumulators, one per key half of every tile (each softmax
+// warpgroup keeps its own running max for its half; the halves are merged
+// once per item in the epilogue).
+constexpr uint32_t TM_O = 256;  // O_a [256, 384) for keys [0, 64), O_b [384, 512) for [64, 128)
 constexpr uint32_t IDESC_S = ptx::idesc_bf16(BM, BN, false, false);  // 128 x 128, K-major B
 constexpr uint32_t IDESC_PV = ptx::idesc_bf16(BM, D, false, true);   // 128 x 128, MN-major B
 
@@ -136,7 +139,6 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     mbar_init(bar(B_AFREE), 2 * BM);
     mbar_init(bar(B_DRAIN), 1);
-    for (int i = 0; i < 8; ++i) mbar_init(bar(B_XMAX + i), 64);
     for (int i = 0; i < 4; ++i) mbar_init(bar(B_XSUM + i), 64);
     for (uint32_t i = 0; i < kRing; ++i) {
       mbar_init(bar(B_IFULL + i), 1);
@@ -241,11 +243,15 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         tc_fence_after();
         const uint64_t vb = v_desc + b * (kStage >> 4);
         const uint32_t first = c.j == 0 ? 0u : 1u;
-        // O += P V: 8 steps of 16 keys; P's 128 keys are packed in 64 columns.
+        // O_a += P[:, 0:64] V[0:64], O_b += P[:, 64:128] V[64:128]: 4 steps of
+        // 16 keys each. The bf16 P of keys [64 h, 64 h + 64) is packed into
+        // buffer columns [64 h, 64 h + 32), the start of the S columns that
+        // softmax warpgroup h itself read.
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts(tmem + TM_O, tmem + b * 128u + ks * 8u, vb + ((ks * 2048) >> 4), IDESC_PV,
-                 first | (ks > 0));
+          mma_ts(tmem + TM_O + (ks >> 2) * 128u,
+                 tmem + b * 128u + (ks >> 2) * 64u + (ks & 3) * 8u,
+                 vb + ((ks * 2048) >> 4), IDESC_PV, first | ((ks & 3) > 0));
         mma_commit(bar(B_VEMPTY + b));
         mma_commit(bar(B_PVD + b));
         return true;
@@ -276,15 +282,16 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   } else if (warp >= 4) {
     // ----------------------------------------------------------- softmax ----
     // Warps 4-7 take keys [0, 64) of every 128-key tile, warps 8-11 keys
-    // [64, 128); warps 4+q and 8+q hold the same rows (TMEM lane quarter q)
-    // and exchange partial row maxima every tile, so both apply one running
-    // max; their partial sums are added at the end.
+    // [64, 128) (one row per thread, TMEM lane quarter q for warps 4+q and
+    // 8+q). Each warpgroup keeps its own running max and sum for its half
+    // and accumulates into its own O (O_a or O_b), so the two never wait for
+    // each other inside an item; the epilogue merges the halves.
     const int hw = (warp - 4) >> 2;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t tl = tmem + (uint32_t(q4 * 32) << 16);
-    float* const xmax = reinterpret_cast<float*>(base_ptr + SM_XCHG);  // [2 parity][2][128]
-    float* const xsum = xmax + 4 * BM;                                 // [2][128]
+    const uint32_t my_o = TM_O + 128u * hw;
+    float* const xsum = reinterpret_cast<float*>(base_ptr + SM_XCHG);  // [2 (m, l)][2][128]
     Cursor c;
     c.start(p, ring, kConsumerWarp);
     float m_ref = -CUDART_INF_F, l = 0.f;
@@ -325,47 +332,40 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       for (int w2 = 4; w2 > 0; w2 >>= 1)
 #pragma unroll
         for (int i = 0; i < w2; ++i) m8[i] = fmaxf(m8[i], m8[i + w2]);
-      xmax[(b * 2u + hw) * BM + r] = m8[0];
-      // The exchange also orders TMEM: warpgroup 1 writes its P over S
-      // columns [32, 64) that warpgroup 0 has just read.
-      tc_fence_before();
-      mbar_arrive(bar(B_XMAX + q4 * 2 + b));
-      ok = wait_bar(bar(B_XMAX + q4 * 2 + b), (c.t >> 1) & 1u, p, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      const float mxs = fmaxf(m8[0], xmax[(b * 2u + (hw ^ 1)) * BM + r]) * p.c2;
+      const float mxs = m8[0] * p.c2;  // -inf while every key of this half is masked
       float alpha = 1.f;
       bool need = false;
       if (m_ref == -CUDART_INF_F) {
-        m_ref = mxs;  // first tile of the item: nothing accumulated yet
+        m_ref = mxs;  // first keys of this half: nothing accumulated yet (l = 0)
       } else if (mxs > m_ref + kTau) {
         alpha = ex2(m_ref - mxs);
         m_ref = mxs;
         need = true;
       }
+      // Each warp decides for its own rows and scales only its own O.
       if (__any_sync(0xffffffffu, need)) {
         l *= alpha;
-        // O holds PV(t-1); wait for it, then scale this warpgroup's half.
-        // (PV(t-3), the previous phase of that barrier, completed before
-        // S(t-1) was issued.)
+        // This O holds PV(t-1); wait for it. (PV(t-3), the previous phase of
+        // that barrier, completed before S(t-1) was issued.)
         ok = wait_bar(bar(B_PVD + ((c.t - 1) & 1u)), ((c.t - 1) >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
 #pragma unroll 1
-        for (int q = 0; q < 2; ++q) {
-          const uint32_t col = TM_O + 64u * hw + 32u * q;
+        for (int q = 0; q < 4; ++q) {
           uint32_t a[32];
-          tmem_ld32(tl + col, a);
+          tmem_ld32(tl + my_o + 32u * q, a);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) * alpha);
-          tmem_st32(tl + col, a);
+          tmem_st32(tl + my_o + 32u * q, a);
         }
         tmem_wait_st();
       }
-      // e = 2^(c2 s - m) in packed pairs; bf16 P into this warpgroup's 32
-      // columns of the buffer (keys 64 hw .. 64 hw + 63).
-      const uint64_t c2v = f2pack(p.c2, p.c2), mv = f2pack(-m_ref, -m_ref);
+      // e = 2^(c2 s - m) in packed pairs (m = 0 while the half is all
+      // masked, so that e = 0 there); bf16 P over the first 32 of the S
+      // columns this warp has just read (never the other warpgroup's).
+      const float mref_use = m_ref == -CUDART_INF_F ? 0.f : m_ref;
+      const uint64_t c2v = f2pack(p.c2, p.c2), mv = f2pack(-mref_use, -mref_use);
       uint64_t la = 0, lb = 0;
       uint32_t pp[32];
 #pragma unroll
@@ -382,7 +382,7 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         f2unpack(add2(la, lb), u0, u1);
         l += u0 + u1;
       }
-      tmem_st32(tl + b * 128u + 32u * hw, pp);
+      tmem_st32(tl + b * 128u + 64u * hw, pp);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_PFULL + b));
@@ -393,50 +393,62 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         // before S(t) was issued.
         ok = wait_bar(bar(B_PVD + (c.t & 1u)), (c.t >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
-        xsum[hw * BM + r] = l;
+        xsum[hw * BM + r] = m_ref;
+        xsum[(2 + hw) * BM + r] = l;
         mbar_arrive(bar(B_XSUM + q4));
         ok = wait_bar(bar(B_XSUM + q4), c.item_idx & 1, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
-        const float lt = l + xsum[(hw ^ 1) * BM + r];
+        // Merge the halves: M = max(m_a, m_b), w = 2^(m - M) (0 for an
+        // all-masked half), L = w_a l_a + w_b l_b.
+        const float m_a = hw == 0 ? m_ref : xsum[r], m_b = hw == 1 ? m_ref : xsum[BM + r];
+        const float l_a = hw == 0 ? l : xsum[2 * BM + r], l_b = hw == 1 ? l : xsum[3 * BM + r];
+        const float M = fmaxf(m_a, m_b);
+        const float w_a = m_a == -CUDART_INF_F ? 0.f : ex2(m_a - M);
+        const float w_b = m_b == -CUDART_INF_F ? 0.f : ex2(m_b - M);
+        const float lt = w_a * l_a + w_b * l_b;
         tc_fence_after();
         const bool row_ok = grow < p.Lq;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const float sa_ = p.split ? w_a : w_a * inv, sb_ = p.split ? w_b : w_b * inv;
+        // This warpgroup writes head-dim columns [64 hw, 64 hw + 64).
 #pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {
           const uint32_t col = 64u * hw + 32u * cc;
-          uint32_t a[32];
-          tmem_ld32(tl + TM_O + col, a);
+          uint32_t oa[32], ob[32];
+          tmem_ld32(tl + TM_O + col, oa);
+          tmem_ld32(tl + TM_O + 128u + col, ob);
           tmem_wait_ld();
-          if (!p.split) {
-            const float inv = lt > 0.f ? 1.f / lt : 0.f;
-            uint32_t po[16];
+          float v[32];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              po[i] = pack_bf16(__uint_as_float(a[2 * i]) * inv,
-                                __uint_as_float(a[2 * i + 1]) * inv);
+          for (int i = 0; i < 32; ++i)
+            v[i] = fmaf(__uint_as_float(oa[i]), sa_, __uint_as_float(ob[i]) * sb_);
+          if (!p.split) {
             if (row_ok) {
               uint4* go = reinterpret_cast<uint4*>(p.o + (size_t(c.bh) * p.Lq + grow) * D + col);
 #pragma unroll
               for (int i = 0; i < 4; ++i)
-                go[i] = make_uint4(po[4 * i], po[4 * i + 1], po[4 * i + 2], po[4 * i + 3]);
+                go[i] = make_uint4(pack_bf16(v[8 * i], v[8 * i + 1]),
+                                   pack_bf16(v[8 * i + 2], v[8 * i + 3]),
+                                   pack_bf16(v[8 * i + 4], v[8 * i + 5]),
+                                   pack_bf16(v[8 * i + 6], v[8 * i + 7]));
             }
           } else {
-            // Unnormalised partial of this key split, for every row of the
-            // tile (rows past Lq are never combined).
+            // Unnormalised partial of this key split relative to M, for every
+            // row of the tile (rows past Lq are never combined).
             float4* dst = reinterpret_cast<float4*>(p.part + (size_t(c.item) * BM + r) * D + col);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(a[4 * i]), __uint_as_float(a[4 * i + 1]),
-                                   __uint_as_float(a[4 * i + 2]), __uint_as_float(a[4 * i + 3]));
+              dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
           }
         }
         tc_fence_before();
         mbar_arrive(bar(B_AFREE));
         if (hw == 0) {
           if (p.split)
-            p.ml[size_t(c.item) * BM + r] = make_float2(m_ref, lt);
+            p.ml[size_t(c.item) * BM + r] = make_float2(M, lt);
           else if (row_ok)
             p.lse[size_t(c.bh) * p.Lq + grow] =
-                lt > 0.f ? (m_ref + log2f(lt)) * 0.69314718055994531f : -CUDART_INF_F;
+                lt > 0.f ? (M + log2f(lt)) * 0.69314718055994531f : -CUDART_INF_F;
         }
       }
       c.next(p, ring, kConsumerWarp);

@@ -19,6 +19,12 @@ reported. Rank 0 prints one JSON line.
 ``--impl reference`` times the float64 CPU oracle on this machine's host cores
 instead (rank 0 only), on a bounded sample of query rows per step.
 
+``--op cache`` measures the read-only forward of causal rollout instead:
+the last chunk of the workload's video (chunk * tokens_per_frame queries)
+attends to a key/value cache holding all n_frames frames; one step writes
+the chunk's keys (rotated by RoPE) and values into their cache slots and
+runs the cache attention; 4*d FLOPs per (query, key) pair.
+
 ``--op bwd`` measures the masked attention backward instead (gradients of
 <G, O> for the primal output, jvp_attn_bwd) on the same workload, counting
 10*d FLOPs per admitted pair: S recomputed (2d), dP = G V^T (2d), and the
@@ -40,6 +46,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "attention-JVP TFLOP/s (12*d per unmasked pair) and % of B200 bf16 tensor peak"
+METRIC_CACHE = ("KV-cache chunk attention TFLOP/s (4*d per query-key pair) and % of B200 "
+                "bf16 tensor peak")
 METRIC_BWD = ("masked attention backward TFLOP/s (10*d per unmasked pair) and % of B200 "
               "bf16 tensor peak")
 UNIT = "TFLOP/s"
@@ -198,6 +206,51 @@ def dist_setup():
 
 # ---------------------------------------------------------------- our arm --
 
+def device_timed(step, steps: int, world: int, local: int, stream, ja):
+    """Times ``steps`` calls of ``step`` with CUDA events on ``stream``,
+    bracketed by barriers and device synchronisation, with nvidia-smi clock
+    samples meanwhile. Returns (per-step ms, max-over-ranks total ms, clocks)."""
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    bus = ClockSampler.bus_id_of(torch.cuda.get_device_properties(local))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    with ClockSampler(bus) as clk:
+        ev[0].record(stream)
+        for i in range(steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ja.check_device_error()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    total = max_over_ranks(ev[0].elapsed_time(ev[-1]), world)
+    return per, total, clk.summary()
+
+
+def e2e_timed(e2e_step, steps: int, world: int, stream, ja) -> float:
+    """Max-over-ranks ms of ``steps`` end-to-end steps (one untimed first)."""
+    import torch
+    import torch.distributed as dist
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ja.check_device_error()
+    return max_over_ranks(e0.elapsed_time(e1), world)
+
+
 def run_ours(args, w):
     import datetime
 
@@ -250,23 +303,7 @@ def run_ours(args, w):
     ja.check_device_error()
 
     # ---- device-timed region (inputs resident in HBM) ----
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    bus = ClockSampler.bus_id_of(torch.cuda.get_device_properties(local))
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    with ClockSampler(bus) as clk:
-        ev[0].record(stream)
-        for i in range(args.steps):
-            step()
-            ev[i + 1].record(stream)
-        torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    ja.check_device_error()
-    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    total_ms = ev[0].elapsed_time(ev[-1])
-    total_ms_max = max_over_ranks(total_ms, world)
+    per, total_ms_max, clocks = device_timed(step, args.steps, world, local, stream, ja)
     value = flops * args.steps * world / (total_ms_max * 1e-3) / 1e12
     launch_ms = sum(per) / len(per)
 
@@ -289,23 +326,9 @@ def run_ours(args, w):
         for h, d in zip(host_out, dev_out):
             h.copy_(d, non_blocking=True)
 
-    e2e_step()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    ja.check_device_error()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_ms = e2e_timed(e2e_step, e2e_steps, world, stream, ja)
     e2e_value = flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
 
-    clocks = clk.summary()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -357,6 +380,126 @@ def run_ours(args, w):
         line["cpu_baseline"] = (cpu_baseline_bwd(w, step_in, rows_per_head=args.cpu_rows_bwd)
                                 if bwd else
                                 cpu_baseline(w, inputs, rows_per_head=args.cpu_rows))
+    return line
+
+
+def cache_shape(w):
+    """(Lq, Lk) of the rollout's last chunk: one chunk of queries against all
+    frames of the video (the committed prefix plus the chunk itself)."""
+    chunk = max(1, w.chunk)
+    return chunk * w.tokens_per_frame, w.n_frames * w.tokens_per_frame
+
+
+def run_ours_cache(args, w):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import attention_jvp_continuous_b200 as ja
+    from attention_jvp_continuous_b200.inputs import rope_table
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    ja._lib.lib()
+    Lq, Lk = cache_shape(w)
+    B, H, d = w.B, w.H, w.d
+    flops = 4.0 * d * Lq * Lk * B * H
+    gen = torch.Generator(device="cuda").manual_seed(rank_seed(w.seed, rank))
+
+    def draw(rows):
+        return torch.randn((B, H, rows, d), generator=gen, device="cuda").to(torch.bfloat16)
+
+    q, k_cur, v_cur = draw(Lq), draw(Lq), draw(Lq)
+    kc, vc = draw(Lk), draw(Lk)  # committed prefix (post-RoPE keys) and values
+    cos, sin = rope_table(Lk, d, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Lq), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    pos = Lk - Lq
+    attn_ev = []
+
+    def step(record=False):
+        ja.rope_copy(k_cur, kc, Lq, 0, pos, cos, sin, rope_row0=pos)
+        ja.rope_copy(v_cur, vc, Lq, 0, pos)
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            ja.cache_attn(q, kc, vc, Lk, o, lse)
+            e1.record(stream)
+            attn_ev.append((e0, e1))
+        else:
+            ja.cache_attn(q, kc, vc, Lk, o, lse)
+
+    for _ in range(args.warmup):
+        step()
+    ja.check_device_error()
+    per, total_ms_max, clocks = device_timed(lambda: step(True), args.steps, world, local,
+                                             stream, ja)
+    value = flops * args.steps * world / (total_ms_max * 1e-3) / 1e12
+    attn_ms = sum(a.elapsed_time(b) for a, b in attn_ev) / len(attn_ev)
+
+    # end to end: the chunk's q, k, v from pinned host memory, o and LSE back;
+    # the cache is rollout state and stays in HBM
+    host_in = [t.cpu().pin_memory() for t in (q, k_cur, v_cur)]
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, lse)]
+
+    def e2e_step():
+        for dv, hv in zip((q, k_cur, v_cur), host_in):
+            dv.copy_(hv, non_blocking=True)
+        step()
+        for hv, dv in zip(host_out, (o, lse)):
+            hv.copy_(dv, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_ms = e2e_timed(e2e_step, e2e_steps, world, stream, ja)
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC_CACHE, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms_max / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": f"{w.name} rollout, last chunk: {Lq} queries ({max(1, w.chunk)} "
+                        f"frame(s) x {w.tokens_per_frame} tokens) over a cache of {Lk} keys "
+                        f"({w.n_frames} frames), B={B} H={H} d={d}, post-RoPE keys",
+            "B": B, "H": H, "d": d, "Lq": Lq, "Lk": Lk, "flops_per_step": flops,
+            "step": "rope_copy(k chunk, rotated) + rope_copy(v chunk) + cache attention",
+            "l2": "cache %.0f MB read per step (above the 126 MB L2); no flush"
+                  % (2 * B * H * Lk * d * 2 / 1e6),
+            "parallelism": f"dp{world} (independent problems per rank, no data collective)",
+        },
+        "e2e": {"value": round(flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12, 2),
+                "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps,
+                "note": "chunk q, k, v in and o, lse out; the cache stays resident"},
+        "gpu_launches": args.steps * 4,
+        "roofline": {
+            "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": UNIT,
+            "frac": round(achieved / peak, 4), "traffic": None,
+            "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
+            "frac_of_sustained": round(achieved / float(peaks.get(
+                "bf16_tflops_sustained", peak)), 4),
+            "frac_of_nominal_2250": round(achieved / NOMINAL_BF16_TFLOPS, 4),
+            "kernel": "attn_cache_sm100_kernel + attn_cache_combine_kernel (one call)",
+            "launch_ms": round(attn_ms, 4),
+        },
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_cache(w, q, kc, vc, rows_per_head=args.cpu_rows_cache)
     return line
 
 
@@ -427,6 +570,30 @@ def cpu_baseline_bwd(w, step_in, rows_per_head: int):
                       f"float64 numpy)"}
 
 
+def oracle_sample_cache(w, q, kc, vc, rows_per_head: int, seed: int = 1234):
+    """Times the float64 cache-attention oracle on ``rows_per_head`` seeded
+    query rows of every head; returns (seconds, query-key pairs)."""
+    from attention_jvp_continuous_b200.inputs import sample_rows
+    from oracle import cache_attention_head
+
+    Lq, Lk = cache_shape(w)
+    rows = sample_rows(Lq, rows_per_head, seed=seed)
+    t0 = time.perf_counter()
+    for b in range(w.B):
+        for h in range(w.H):
+            cache_attention_head(q[b, h, rows], kc[b, h], vc[b, h], Lk)
+    return time.perf_counter() - t0, len(rows) * Lk * w.B * w.H
+
+
+def cpu_baseline_cache(w, q, kc, vc, rows_per_head: int):
+    q, kc, vc = q.cpu(), kc.cpu(), vc.cpu()
+    dt, pairs = oracle_sample_cache(w, q, kc, vc, rows_per_head)
+    return {"value": round(4.0 * w.d * pairs / dt / 1e12, 6), "unit": UNIT,
+            "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{rows_per_head} seeded query rows per head x {w.B * w.H} heads "
+                      f"over the full cache ({pairs} pairs, {dt:.1f} s, float64 numpy)"}
+
+
 def run_reference(args, w):
     world, rank, _ = dist_setup()
     if rank != 0:
@@ -436,7 +603,14 @@ def run_reference(args, w):
     from attention_jvp_continuous_b200.inputs import make_inputs
     inputs, _ = make_inputs(w, device="cpu")
     rows = args.ref_rows
-    if args.op == "bwd":
+    if args.op == "cache":
+        Lq, Lk = cache_shape(w)
+        gen = torch.Generator().manual_seed(w.seed)
+        qh = torch.randn((w.B, w.H, Lq, w.d), generator=gen).to(torch.bfloat16)
+        kh = torch.randn((w.B, w.H, Lk, w.d), generator=gen).to(torch.bfloat16)
+        vh = torch.randn((w.B, w.H, Lk, w.d), generator=gen).to(torch.bfloat16)
+        run_sample = lambda seed: oracle_sample_cache(w, qh, kh, vh, rows, seed=seed)  # noqa: E731
+    elif args.op == "bwd":
         # The oracle's gradient needs no primal output; a seeded cotangent.
         gen = torch.Generator().manual_seed(w.seed + 17)
         g = torch.randn(inputs[0].shape, generator=gen).to(inputs[0].dtype)
@@ -452,11 +626,12 @@ def run_reference(args, w):
         times.append(dt)
         pairs += sp
     total = sum(times)
-    value = flops_per_pair(w, args.op) * pairs / total / 1e12
+    value = (4.0 * w.d if args.op == "cache" else flops_per_pair(w, args.op)) * pairs / total / 1e12
     cores = blas_threads()
     sample = f"{rows} seeded query rows per head x {w.B * w.H} heads per step"
-    return {
-        "impl": "reference", "metric": METRIC_BWD if args.op == "bwd" else METRIC,
+    line = {
+        "impl": "reference",
+        "metric": {"bwd": METRIC_BWD, "cache": METRIC_CACHE}.get(args.op, METRIC),
         "value": round(value, 6), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * total / args.steps, 2), "higher_is_better": True,
@@ -470,6 +645,11 @@ def run_reference(args, w):
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
+    if args.op == "cache":
+        Lq, Lk = cache_shape(w)
+        line["config"].update({"workload": f"{w.name} rollout, last chunk (oracle on sampled "
+                                           f"rows)", "Lq": Lq, "Lk": Lk})
+    return line
 
 
 def main(argv=None):
@@ -487,8 +667,11 @@ def main(argv=None):
                     help="query rows per head per step of --impl reference")
     ap.add_argument("--cpu-rows-bwd", type=int, default=1024,
                     help="query rows per head in the --op bwd cpu_baseline sample")
-    ap.add_argument("--op", choices=["jvp", "bwd"], default="jvp",
-                    help="jvp: the attention JVP (default); bwd: the masked backward")
+    ap.add_argument("--cpu-rows-cache", type=int, default=512,
+                    help="query rows per head in the --op cache cpu_baseline sample")
+    ap.add_argument("--op", choices=["jvp", "bwd", "cache"], default="jvp",
+                    help="jvp: the attention JVP (default); bwd: the masked backward; "
+                         "cache: KV-cache chunk attention of the rollout's last chunk")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the workload's head count (small cases for ncu captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -505,7 +688,12 @@ def main(argv=None):
     world, rank, _ = dist_setup()
     if world != args.gpus and args.impl == "ours":
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
-    line = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
+    if args.impl == "reference":
+        line = run_reference(args, w)
+    elif args.op == "cache":
+        line = run_ours_cache(args, w)
+    else:
+        line = run_ours(args, w)
     if line is not None and rank == 0:
         print(json.dumps(line), flush=True)
 
