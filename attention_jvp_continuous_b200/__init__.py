@@ -20,7 +20,7 @@ CHUNK_CAUSAL = 2
 TEACHER_FORCING = 3
 
 __all__ = ["Mask", "jvp_attn", "jvp_attn_fwd", "attn_bwd", "jvp_attn_bwd", "bwd_scratch_len",
-           "cache_attn", "rope_copy", "mask_stats", "tile_classes",
+           "cache_attn", "rope_copy", "qkv_prologue", "mask_stats", "tile_classes",
            "schedule", "schedule_kv", "check_device_error", "set_wait_limit", "release",
            "JvpAttnError",
            "DENSE", "FRAME_CAUSAL", "CHUNK_CAUSAL", "TEACHER_FORCING"]
@@ -212,6 +212,48 @@ def rope_copy(src, dst, rows: int, src_row0: int = 0, dst_row0: int = 0, cos=Non
         int(dst_row0), d, _dtype_code(src), cp, sp, n_rope, int(rope_row0),
         ctypes.c_void_p(stream))
     _lib.check(rc, "jvp_attn_rope_copy")
+
+
+def qkv_prologue(qkv, d_qkv, H: int, norm_q=None, norm_k=None, norm_group: Optional[int] = None,
+                 eps: float = 1e-6, cos=None, sin=None, out=None, stream: Optional[int] = None):
+    """Attention-layer tangent prologue (jvp_attn_qkv_prologue): from the fused
+    projections qkv, d_qkv [B, L, 3*H*d] (bf16, CUDA) of x and its tangent,
+    QK-norm (weights norm_q / norm_k, float32 [norm_group]; norm_group H*d or
+    d) with its derivative, RoPE by token row (cos / sin float32 [>= L, d/2])
+    and the [B, H, L, d] layout. Returns (q, k, v, dq, dk, dv), into `out`
+    (six tensors) when given."""
+    import torch
+    for t in (qkv, d_qkv):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError("qkv and d_qkv must be contiguous bf16 CUDA tensors [B, L, 3 H d]")
+    if d_qkv.shape != qkv.shape or qkv.shape[2] % (3 * H):
+        raise ValueError("qkv and d_qkv must share one shape [B, L, 3 H d]")
+    B, L, C3 = qkv.shape
+    d = C3 // (3 * H)
+    if out is None:
+        out = [torch.empty((B, H, L, d), dtype=qkv.dtype, device=qkv.device) for _ in range(6)]
+    for t in out:
+        if t.shape != (B, H, L, d) or t.dtype != qkv.dtype or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError("outputs must be contiguous bf16 CUDA tensors [B, H, L, d]")
+    fp = ctypes.POINTER(ctypes.c_float)
+
+    def fptr(t):
+        if t is None:
+            return None
+        if not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError("norm weights and rotation tables must be contiguous float32 CUDA tensors")
+        return ctypes.cast(t.data_ptr(), fp)
+
+    n_rope = 0 if cos is None else cos.shape[0]
+    group = (H * d if norm_group is None else int(norm_group)) if norm_q is not None else 0
+    if stream is None:
+        stream = torch.cuda.current_stream(qkv.device).cuda_stream
+    rc = _lib.lib().jvp_attn_qkv_prologue(
+        qkv.data_ptr(), d_qkv.data_ptr(), *[t.data_ptr() for t in out], fptr(norm_q),
+        fptr(norm_k), group, float(eps), fptr(cos), fptr(sin), n_rope, B, L, H, d,
+        _lib.JVP_BF16, ctypes.c_void_p(stream))
+    _lib.check(rc, "jvp_attn_qkv_prologue")
+    return tuple(out)
 
 
 def mask_stats(mask: Mask, L: Optional[int] = None, bm: int = 128, bn: int = 64):

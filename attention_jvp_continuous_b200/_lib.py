@@ -33,7 +33,8 @@ TILE_EMPTY, TILE_FULL, TILE_PARTIAL = 0, 1, 2
 
 # Exported functions, as declared in include/jvp_attn.h.
 EXPORTS = ("jvp_attn_fwd", "jvp_attn_fwd_noalloc", "jvp_attn_bwd", "jvp_attn_bwd_scratch_len",
-           "jvp_attn_cache_fwd", "jvp_attn_rope_copy", "jvp_attn_mask_stats",
+           "jvp_attn_cache_fwd", "jvp_attn_rope_copy", "jvp_attn_qkv_prologue",
+           "jvp_attn_mask_stats",
            "jvp_attn_tile_classes", "jvp_attn_schedule", "jvp_attn_schedule_kv",
            "jvp_attn_check_device_error",
            "jvp_attn_set_wait_limit", "jvp_attn_release", "jvp_attn_strerror",
@@ -86,6 +87,9 @@ def lib() -> ctypes.CDLL:
         L.jvp_attn_cache_fwd.restype = i32
         L.jvp_attn_rope_copy.argtypes = [vp, vp] + [i32] * 9 + [fp, fp, i32, i32, vp]
         L.jvp_attn_rope_copy.restype = i32
+        L.jvp_attn_qkv_prologue.argtypes = [vp] * 8 + [fp, fp, i32, ctypes.c_float, fp, fp] + \
+            [i32] * 6 + [vp]
+        L.jvp_attn_qkv_prologue.restype = i32
         L.jvp_attn_mask_stats.argtypes = [MaskDesc, i32, i32, i32, i64p, i64p, i64p, i64p]
         L.jvp_attn_mask_stats.restype = i32
         L.jvp_attn_tile_classes.argtypes = [MaskDesc, i32, i32, i32,

@@ -91,6 +91,18 @@ struct RopeArgs {
 };
 int launch_rope_copy(const RopeArgs& a, int num_sms);
 
+// Attention-layer tangent prologue (jvp_attn_qkv_prologue): bf16.
+struct PrologueArgs {
+  const void *qkv, *dqkv;  // [B, L, 3 H d]
+  void* out[6];            // q, k, v, dq, dk, dv: [B, H, L, d]
+  const float *norm_q, *norm_k;  // [group] or null (no norm)
+  const float *cos, *sin;        // [>= L, d/2] or null (no rotation)
+  int B, L, H, d, group;
+  float eps;
+  cudaStream_t stream;
+};
+int launch_qkv_prologue(const PrologueArgs& a, int num_sms);
+
 // Per-wait limit for the tensor-core kernel (jvp_attn_set_wait_limit).
 unsigned long long wait_limit_ns();
 

@@ -391,6 +391,41 @@ int jvp_attn_rope_copy(const void* src, void* dst, int B, int H, int src_rows, i
   return launch_rope_copy(a, di->sms);
 }
 
+int jvp_attn_qkv_prologue(const void* qkv, const void* d_qkv, void* q, void* k, void* v,
+                          void* dq, void* dk, void* dv, const float* norm_q,
+                          const float* norm_k, int norm_group, float eps,
+                          const float* rope_cos, const float* rope_sin, int rope_rows, int B,
+                          int L, int H, int d, jvp_dtype dtype, void* stream) {
+  const void* ptrs[] = {qkv, d_qkv, q, k, v, dq, dk, dv};
+  for (const void* p : ptrs)
+    if (!p) return JVP_ERR_INVALID_ARG;
+  if (B <= 0 || L <= 0 || H <= 0 || d <= 0 || dtype != JVP_BF16) return JVP_ERR_INVALID_ARG;
+  if (d < 8 || d > 256 || (d & (d - 1)) != 0) return JVP_ERR_UNSUPPORTED_HEAD_DIM;
+  if ((H * d) % 256 != 0) return JVP_ERR_INVALID_ARG;
+  if ((norm_q == nullptr) != (norm_k == nullptr)) return JVP_ERR_INVALID_ARG;
+  if (norm_q && (norm_group != H * d && norm_group != d)) return JVP_ERR_INVALID_ARG;
+  if (norm_q && (!(eps >= 0.f) || std::isinf(eps))) return JVP_ERR_INVALID_ARG;
+  if ((rope_cos == nullptr) != (rope_sin == nullptr)) return JVP_ERR_INVALID_ARG;
+  if (rope_cos && rope_rows < L) return JVP_ERR_INVALID_ARG;
+  if ((long long)B * L * 3 * H * d >= (1LL << 40)) return JVP_ERR_TOO_LARGE;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return JVP_ERR_MISALIGNED;
+  const void* opt[] = {norm_q, norm_k, rope_cos, rope_sin};
+  for (const void* p : opt)
+    if (p && !aligned16(p)) return JVP_ERR_MISALIGNED;
+  DevInfo* di = nullptr;
+  int rc = device_info(&di);
+  if (rc != JVP_OK) return rc;
+  if (di->major != 10 || di->minor != 0) return JVP_ERR_UNSUPPORTED_DEVICE;
+  PrologueArgs a;
+  a.qkv = qkv; a.dqkv = d_qkv;
+  a.out[0] = q; a.out[1] = k; a.out[2] = v; a.out[3] = dq; a.out[4] = dk; a.out[5] = dv;
+  a.norm_q = norm_q; a.norm_k = norm_k; a.cos = rope_cos; a.sin = rope_sin;
+  a.B = B; a.L = L; a.H = H; a.d = d; a.group = norm_q ? norm_group : H * d; a.eps = eps;
+  a.stream = static_cast<cudaStream_t>(stream);
+  return launch_qkv_prologue(a, di->sms);
+}
+
 int jvp_attn_schedule_kv(jvp_mask_desc mask, int L, int bq, int bk, int32_t* ktiles,
                          int ktile_cap, int32_t* segs, int seg_cap, int* n_ktiles, int* n_segs) {
   int rc = validate_mask(mask, L);

@@ -256,6 +256,37 @@ int jvp_attn_rope_copy(const void* src, void* dst, int B, int H, int src_rows, i
                        const float* rope_cos, const float* rope_sin, int rope_rows,
                        int rope_row0, void* stream);
 
+/* ---- attention-layer tangent prologue ------------------------------------ */
+/*
+ * jvp_attn_qkv_prologue: the primal-tangent hand-off from an attention
+ * layer's fused QKV projection to jvp_attn_fwd (layer-level JVP, Causal-rCM
+ * report Sec. 3.2.2 "JVP FSDP2": each layer maps (x, dx) to (y, dy); with
+ * the weights at their stop-gradient values the projection tangent is
+ * dx W, computed by the caller's GEMM). For every token, q and k are RMS
+ * normalised over groups of norm_group channels with weights norm_q /
+ * norm_k, their tangents by the derivative of that normalisation
+ *   r = 1/sqrt(mean(a^2) + eps),  y = a r w,  dy = w r (da - a mean(a da) r^2),
+ * then both are rotated by rotary position embedding (row l of rope_cos /
+ * rope_sin [rope_rows >= L, d/2], float32, pairs (x_2i, x_2i+1) as in
+ * jvp_attn_rope_copy; the tangent rotates like the primal), and q, k, v and
+ * their tangents are written in the [B, H, L, d] layout of jvp_attn_fwd.
+ *
+ * qkv, d_qkv   [B, L, 3 H d] bf16: [q | k | v] of x and of dx, each block
+ *              H*d channels, channel h*d + j = head h, dimension j
+ * q .. dv      outputs [B, H, L, d] bf16
+ * norm_q, norm_k  float32 [norm_group], both NULL for no normalisation;
+ *              norm_group is H*d (one group per token) or d (per head)
+ * rope_cos, rope_sin  both NULL for no rotation
+ * Requires dtype JVP_BF16, d a power of two in [8, 256]
+ * (else JVP_ERR_UNSUPPORTED_HEAD_DIM), H*d a multiple of 256, 16-byte
+ * aligned pointers. Memory-bound; asynchronous on `stream`.
+ */
+int jvp_attn_qkv_prologue(const void* qkv, const void* d_qkv, void* q, void* k, void* v,
+                          void* dq, void* dk, void* dv, const float* norm_q,
+                          const float* norm_k, int norm_group, float eps,
+                          const float* rope_cos, const float* rope_sin, int rope_rows, int B,
+                          int L, int H, int d, jvp_dtype dtype, void* stream);
+
 /* ---- host-side mask / schedule queries (no GPU needed) ------------------- */
 /*
  * jvp_attn_mask_stats: for the mask on L tokens and a bm x bn tile grid

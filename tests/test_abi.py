@@ -160,3 +160,30 @@ def test_bwd_scratch_len():
     assert _lib.lib().jvp_attn_bwd_scratch_len(1, 12, 65520) == 2 * 12 * 65536
     assert _lib.lib().jvp_attn_bwd_scratch_len(2, 3, 1) == 2 * 6 * 128
     assert _lib.lib().jvp_attn_bwd_scratch_len(0, 1, 1) == -1
+
+
+def call_prologue(**kw):
+    a = dict(qkv=FAKE, dqkv=FAKE, outs=[FAKE] * 6, nq=FAKE, nk=FAKE, group=1536, eps=1e-6,
+             cos=FAKE, sin=FAKE, rope_rows=100, B=1, L=100, H=12, d=128, dtype=_lib.JVP_BF16)
+    a.update(kw)
+    fp = ctypes.POINTER(ctypes.c_float)
+    cvt = lambda x: ctypes.cast(x, fp) if x else None  # noqa: E731
+    return _lib.lib().jvp_attn_qkv_prologue(a["qkv"], a["dqkv"], *a["outs"], cvt(a["nq"]),
+                                            cvt(a["nk"]), a["group"], a["eps"], cvt(a["cos"]),
+                                            cvt(a["sin"]), a["rope_rows"], a["B"], a["L"],
+                                            a["H"], a["d"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(qkv=0), _lib.JVP_ERR_INVALID_ARG),
+    (dict(nk=0), _lib.JVP_ERR_INVALID_ARG),                   # one norm weight only
+    (dict(group=64), _lib.JVP_ERR_INVALID_ARG),               # neither H*d nor d
+    (dict(rope_rows=99), _lib.JVP_ERR_INVALID_ARG),           # table shorter than L
+    (dict(H=3, d=32), _lib.JVP_ERR_INVALID_ARG),              # H*d not a multiple of 256
+    (dict(d=96, H=8), _lib.JVP_ERR_UNSUPPORTED_HEAD_DIM),
+    (dict(dtype=_lib.JVP_FP32), _lib.JVP_ERR_INVALID_ARG),
+    (dict(eps=float("nan")), _lib.JVP_ERR_INVALID_ARG),
+    (dict(outs=[FAKE] * 5 + [FAKE + 8]), _lib.JVP_ERR_MISALIGNED),
+])
+def test_prologue_argument_errors(kw, code):
+    assert call_prologue(**kw) == code
