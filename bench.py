@@ -25,6 +25,12 @@ attends to a key/value cache holding all n_frames frames; one step writes
 the chunk's keys (rotated by RoPE) and values into their cache slots and
 runs the cache attention; 4*d FLOPs per (query, key) pair.
 
+``--op prologue`` measures the attention layer's tangent prologue on the
+workload's tokens: from the fused QKV projections of x and dx ([B, L, 3 H d]
+each), QK-norm over all H*d channels with its tangent, RoPE, and the
+[B, H, L, d] layout of the JVP kernel; memory-bound, reported as
+algorithmic GB/s (inputs read once, outputs written once).
+
 ``--op bwd`` measures the masked attention backward instead (gradients of
 <G, O> for the primal output, jvp_attn_bwd) on the same workload, counting
 10*d FLOPs per admitted pair: S recomputed (2d), dP = G V^T (2d), and the
@@ -48,6 +54,8 @@ if ROOT not in sys.path:
 METRIC = "attention-JVP TFLOP/s (12*d per unmasked pair) and % of B200 bf16 tensor peak"
 METRIC_CACHE = ("KV-cache chunk attention TFLOP/s (4*d per query-key pair) and % of B200 "
                 "bf16 tensor peak")
+METRIC_PROLOGUE = ("attention-layer tangent prologue GB/s (QK-norm JVP + RoPE + layout; "
+                   "algorithmic bytes) and % of measured HBM bandwidth")
 METRIC_BWD = ("masked attention backward TFLOP/s (10*d per unmasked pair) and % of B200 "
               "bf16 tensor peak")
 UNIT = "TFLOP/s"
@@ -503,6 +511,115 @@ def run_ours_cache(args, w):
     return line
 
 
+def run_ours_prologue(args, w):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import attention_jvp_continuous_b200 as ja
+    from attention_jvp_continuous_b200.inputs import rope_table
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    ja._lib.lib()
+    B, L, H, d = w.B, w.L, w.H, w.d
+    C = H * d
+    gen = torch.Generator(device="cuda").manual_seed(rank_seed(w.seed, rank))
+    P = torch.randn((B, L, 3 * C), generator=gen, device="cuda").to(torch.bfloat16)
+    dP = (torch.randn((B, L, 3 * C), generator=gen, device="cuda") * w.tangent_std).to(
+        torch.bfloat16)
+    wq = 1.0 + 0.1 * torch.randn((C,), generator=gen, device="cuda")
+    wk = 1.0 + 0.1 * torch.randn((C,), generator=gen, device="cuda")
+    # teacher forcing: clean token i and noisy token F*T + i share position i
+    half = L // 2 if w.mode == 3 else L
+    cos, sin = rope_table(half, d, device="cuda")
+    if w.mode == 3:
+        cos, sin = torch.cat([cos, cos]).contiguous(), torch.cat([sin, sin]).contiguous()
+    out = [torch.empty((B, H, L, d), dtype=torch.bfloat16, device="cuda") for _ in range(6)]
+    stream = torch.cuda.current_stream()
+    nbytes = 2 * P.numel() * 2 + 6 * B * H * L * d * 2
+
+    def step():
+        ja.qkv_prologue(P, dP, H, wq, wk, C, 1e-6, cos, sin, out=out)
+
+    for _ in range(args.warmup):
+        step()
+    ja.check_device_error()
+    per, total_ms_max, clocks = device_timed(step, args.steps, world, local, stream, ja)
+    value = nbytes * args.steps * world / (total_ms_max * 1e-3) / 1e9
+    launch_ms = sum(per) / len(per)
+    host_in = [t.cpu().pin_memory() for t in (P, dP)]
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in out]
+
+    def e2e_step():
+        for dv, hv in zip((P, dP), host_in):
+            dv.copy_(hv, non_blocking=True)
+        step()
+        for hv, dv in zip(host_out, out):
+            hv.copy_(dv, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_ms = e2e_timed(e2e_step, e2e_steps, world, stream, ja)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["hbm_gbs"])
+    achieved = nbytes / (launch_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC_PROLOGUE, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms_max / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": f"{w.name} tokens: B={B} L={L} H={H} d={d}, projections [B, L, 3*{C}] "
+                        f"of x and dx, QK-norm over {C} channels, RoPE",
+            "B": B, "L": L, "H": H, "d": d, "bytes_per_step": nbytes,
+            "l2": "%.2f GB moved per step (above the 126 MB L2); no flush" % (nbytes / 1e9),
+            "parallelism": f"dp{world} (independent problems per rank, no data collective)",
+        },
+        "e2e": {"value": round(nbytes * e2e_steps * world / (e2e_ms * 1e-3) / 1e9, 1),
+                "unit": "GB/s", "h2d_bytes_per_step": sum(t.numel() * t.element_size()
+                                                          for t in host_in),
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in host_out),
+                "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "roofline": {
+            "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": None,
+            "peak_source": f"{peak_src} HBM copy bandwidth",
+            "kernel": "qkv_prologue_kernel", "launch_ms": round(launch_ms, 4),
+        },
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_prologue(w, P, dP, wq, wk, cos, sin,
+                                                     tokens=args.cpu_tokens_prologue)
+    return line
+
+
+def cpu_baseline_prologue(w, P, dP, wq, wk, cos, sin, tokens: int):
+    """The float64 prologue oracle on the first `tokens` tokens of each batch
+    row, in algorithmic GB/s of the same bf16 layout."""
+    from oracle.layer_prologue import qkv_prologue
+    n = min(tokens, w.L)
+    Ph, dPh = P[:, :n].cpu(), dP[:, :n].cpu()
+    t0 = time.perf_counter()
+    qkv_prologue(Ph, dPh, w.H, w.d, wq.cpu(), wk.cpu(), w.H * w.d, 1e-6, cos[:n].cpu(),
+                 sin[:n].cpu())
+    dt = time.perf_counter() - t0
+    nbytes = (2 * Ph.numel() * 2 + 6 * w.B * w.H * n * w.d * 2)
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"first {n} tokens x {w.B} batch rows ({dt:.1f} s, float64 numpy)"}
+
+
 # ---------------------------------------------------- oracle on the host --
 
 def oracle_sample(w, host_inputs, rows_per_head: int, seed: int = 1234):
@@ -594,10 +711,49 @@ def cpu_baseline_cache(w, q, kc, vc, rows_per_head: int):
                       f"over the full cache ({pairs} pairs, {dt:.1f} s, float64 numpy)"}
 
 
+def reference_prologue(args, w, world: int):
+    """--impl reference --op prologue: the float64 prologue oracle on
+    16 * ref_rows tokens per step, in algorithmic GB/s."""
+    import torch
+
+    from attention_jvp_continuous_b200.inputs import rope_table
+    from oracle.layer_prologue import qkv_prologue
+    C, n = w.H * w.d, min(16 * args.ref_rows, w.L)
+    gen = torch.Generator().manual_seed(w.seed)
+    P = torch.randn((w.B, n, 3 * C), generator=gen).to(torch.bfloat16)
+    dP = torch.randn((w.B, n, 3 * C), generator=gen).to(torch.bfloat16)
+    wq, wk = torch.ones(C), torch.ones(C)
+    cos, sin = rope_table(n, w.d)
+    nbytes = 2 * P.numel() * 2 + 6 * w.B * w.H * n * w.d * 2
+    for _ in range(args.warmup):
+        qkv_prologue(P, dP, w.H, w.d, wq, wk, C, 1e-6, cos, sin)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        qkv_prologue(P, dP, w.H, w.d, wq, wk, C, 1e-6, cos, sin)
+    total = time.perf_counter() - t0
+    value = nbytes * args.steps / total / 1e9
+    sample = f"{n} tokens x {w.B} batch rows per step"
+    return {
+        "impl": "reference", "metric": METRIC_PROLOGUE, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / args.steps, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name} tokens (oracle on a token sample)", "B": w.B,
+                   "H": w.H, "L": w.L, "d": w.d, "parallelism": "host cores, rank 0 only"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
 def run_reference(args, w):
     world, rank, _ = dist_setup()
     if rank != 0:
         return None
+    if args.op == "prologue":
+        return reference_prologue(args, w, world)
     import torch
 
     from attention_jvp_continuous_b200.inputs import make_inputs
@@ -669,7 +825,9 @@ def main(argv=None):
                     help="query rows per head in the --op bwd cpu_baseline sample")
     ap.add_argument("--cpu-rows-cache", type=int, default=512,
                     help="query rows per head in the --op cache cpu_baseline sample")
-    ap.add_argument("--op", choices=["jvp", "bwd", "cache"], default="jvp",
+    ap.add_argument("--cpu-tokens-prologue", type=int, default=16384,
+                    help="tokens in the --op prologue cpu_baseline sample")
+    ap.add_argument("--op", choices=["jvp", "bwd", "cache", "prologue"], default="jvp",
                     help="jvp: the attention JVP (default); bwd: the masked backward; "
                          "cache: KV-cache chunk attention of the rollout's last chunk")
     ap.add_argument("--heads", type=int, default=None,
@@ -692,6 +850,8 @@ def main(argv=None):
         line = run_reference(args, w)
     elif args.op == "cache":
         line = run_ours_cache(args, w)
+    elif args.op == "prologue":
+        line = run_ours_prologue(args, w)
     else:
         line = run_ours(args, w)
     if line is not None and rank == 0:
