@@ -74,20 +74,18 @@ constexpr uint32_t kSmemBytes = SM_BAR + 512 + 4096 + 1024;  // + barriers, exch
 enum : uint32_t {
   B_QFULL = 0,
   B_QEMPTY = 1,
-  B_KFULL = 2,   // 2 slots
-  B_KSPARE = 4,  // 2 (unused: S-ready releases the K stage)
-  B_VFULL = 6,   // 2
-  B_VEMPTY = 8,  // 2
-  B_SFULL = 10,  // 2
-  B_PFULL = 12,  // 2
-  B_PVDONE = 14,
-  B_AFREE = 15,
-  B_DRAIN = 16,
-  B_XMAX = 17,    // 8 slots: [lane quarter][tile parity], softmax halves' max exchange
-  B_XSUM = 25,    // 4 slots: [lane quarter], end-of-item l/g exchange
-  B_IFULL = 29,   // 4 slots: work-item ring, published
-  B_IEMPTY = 33,  // 4 slots: work-item ring, released
-  kNumBars = 37
+  B_KFULL = 2,    // 2 slots (S(t) complete releases K stage t&1: B_SFULL)
+  B_VFULL = 4,    // 2
+  B_PVD = 6,      // 2: PV(t) of buffer t&1 complete; also releases V stage t&1
+  B_SFULL = 8,    // 2
+  B_PFULL = 10,   // 2
+  B_AFREE = 12,
+  B_DRAIN = 13,
+  B_XMAX = 14,    // 8 slots: [lane quarter][tile parity], softmax halves' max exchange
+  B_XSUM = 22,    // 4 slots: [lane quarter], end-of-item l/g exchange
+  B_IFULL = 26,   // 4 slots: work-item ring, published
+  B_IEMPTY = 30,  // 4 slots: work-item ring, released
+  kNumBars = 34
 };
 constexpr uint32_t SM_TMEM_SLOT = SM_BAR + 8 * kNumBars;  // u32: TMEM base
 constexpr uint32_t SM_ABORT = SM_TMEM_SLOT + 4;           // u32: abort flag
@@ -155,11 +153,10 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(B_KFULL + s), 1);
       mbar_init(bar(B_VFULL + s), 1);
-      mbar_init(bar(B_VEMPTY + s), 1);
+      mbar_init(bar(B_PVD + s), 1);
       mbar_init(bar(B_SFULL + s), 1);
       mbar_init(bar(B_PFULL + s), 2 * BM);
     }
-    mbar_init(bar(B_PVDONE), 1);
     mbar_init(bar(B_AFREE), 2 * BM);
     mbar_init(bar(B_DRAIN), 1);
     for (int i = 0; i < 8; ++i) mbar_init(bar(B_XMAX + i), 64);
@@ -227,7 +224,7 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         tma_load_3d(ks + kKHalf, &tm_dk, bar(B_KFULL + s), 0, y, c.bh);
         tma_load_3d(ks + 2 * kKHalf, &tm_k, bar(B_KFULL + s), 64, y, c.bh);
         tma_load_3d(ks + 3 * kKHalf, &tm_dk, bar(B_KFULL + s), 64, y, c.bh);
-        if (c.t >= 2) ok = wait_bar(bar(B_VEMPTY + s), (u - 1) & 1u, p, abort_flag);
+        if (c.t >= 2) ok = wait_bar(bar(B_PVD + s), (u - 1) & 1u, p, abort_flag);
         if (!ok) break;
         mbar_expect_tx(bar(B_VFULL + s), kStageBytes);
         ++v_issued;
@@ -306,8 +303,7 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
           mma_ts(tmem + TM_A23, a_pd + ks * 8, vb + ((ks * 2048) >> 4), IDESC_PV, 1u);
-        mma_commit(bar(B_VEMPTY + b));
-        mma_commit(bar(B_PVDONE));
+        mma_commit(bar(B_PVD + b));  // PV(t) done: V stage b free, A1/A23 current
         return true;
       };
       Cursor cs, cp;
@@ -413,7 +409,9 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         g *= alpha;
         // A1/A23 hold PV(t-1); wait for it, then scale this quarter's rows:
         // the first warpgroup scales A1, the second A23.
-        ok = wait_bar(bar(B_PVDONE), (c.t - 1) & 1u, p, abort_flag);
+        // (PV(t-3), the previous phase of that barrier, completed before
+        // S(t-1) was issued.)
+        ok = wait_bar(bar(B_PVD + ((c.t - 1) & 1u)), ((c.t - 1) >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
 #pragma unroll 1
@@ -471,11 +469,9 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
       if (c.j == c.n - 1) {
         // ------------------------------------------------------ epilogue --
-        // PV(t-1) may still be running here, i.e. the barrier may be two
-        // phases short of PV(t); a parity wait is only unambiguous one phase
-        // ahead, so wait for PV(t-1) first, then for PV(t).
-        ok = c.t == 0 || wait_bar(bar(B_PVDONE), (c.t - 1) & 1u, p, abort_flag);
-        ok = ok && wait_bar(bar(B_PVDONE), c.t & 1u, p, abort_flag);
+        // PV(t) done; PV(t-2), the previous phase of this barrier, completed
+        // before S(t) was issued, so the parity wait is unambiguous.
+        ok = wait_bar(bar(B_PVD + (c.t & 1u)), (c.t >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         // Row totals of l and g from both halves.
         xsum[hw * BM + r] = l;
