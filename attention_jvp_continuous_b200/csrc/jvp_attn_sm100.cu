@@ -257,68 +257,106 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint64_t dq_desc = sdesc_sw128(base + SM_DQ, 16, 1024);
       const uint64_t k_desc = sdesc_sw128(base + SM_K, 16, 1024);       // stage 0
       const uint64_t v_desc = sdesc_sw128(base + SM_V, kKHalf, 1024);   // stage 0
-      auto issue_s = [&](const Cursor& c) -> bool {
-        const uint32_t b = c.t & 1u;
+      // The tensor pipe takes a tile's 24 MMAs back to back in ~1.65k cycles,
+      // but holds only a few queued MMAs: scalar work done between batches
+      // (barrier checks, commits, cursor steps) lets it run dry. So each
+      // batch is issued in two halves, and the waits for the next batch and
+      // the cursor step go between them, while the first half executes.
+      auto wait_s = [&](const Cursor& c) -> bool {  // S(t): Q (new item), K|dK stage
         if (c.j == 0 && !wait_bar(bar(B_QFULL), c.item_idx & 1, p, abort_flag)) return false;
-        if (!wait_bar(bar(B_KFULL + b), (c.t >> 1) & 1u, p, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t d_s = tmem + b * 128u, d_ds = d_s + 64u;
-        const uint64_t kb = k_desc + b * (kStageBytes >> 4);
-        // [S | Q dK^T] = Q [K ; dK]^T: one N=128 MMA per 16-wide k-step.
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t oq = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
-          const uint32_t ob = ((kk >> 2) * (2 * kKHalf) + (kk & 3) * 32) >> 4;
-          mma_ss(d_s, q_desc + oq, kb + ob, IDESC_SK, kk > 0);
-        }
-        // dS = Q dK^T + dQ K^T: N=64 MMAs accumulate dQ K^T onto it.
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t oq = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
-          const uint32_t ob = ((kk >> 2) * (2 * kKHalf) + (kk & 3) * 32) >> 4;
-          mma_ss(d_ds, dq_desc + oq, kb + ob, IDESC_S, 1u);
-        }
-        mma_commit(bar(B_SFULL + b));  // also releases K stage b to the producer
-        if (c.j == c.n - 1) mma_commit(bar(B_QEMPTY));
-        return true;
+        return wait_bar(bar(B_KFULL + (c.t & 1u)), (c.t >> 1) & 1u, p, abort_flag);
       };
-      auto issue_pv = [&](const Cursor& c) -> bool {
+      auto wait_pv = [&](const Cursor& c) -> bool {  // PV(t): accumulators, P, V|dV stage
         const uint32_t b = c.t & 1u;
         if (c.j == 0 && c.item_idx > 0 &&
             !wait_bar(bar(B_AFREE), (c.item_idx - 1) & 1, p, abort_flag))
           return false;
         if (!wait_bar(bar(B_PFULL + b), (c.t >> 1) & 1u, p, abort_flag)) return false;
-        if (!wait_bar(bar(B_VFULL + b), (c.t >> 1) & 1u, p, abort_flag)) return false;
-        tc_fence_after();
-        const uint64_t vb = v_desc + b * (kStageBytes >> 4);
-        const uint32_t a_p = tmem + b * 128u, a_pd = a_p + 64u;
-        const uint32_t first = c.j == 0 ? 0u : 1u;
-        // [A1 | A23] += P [V | dV]: one N=256 MMA per 16-key step (A1 and A23
-        // are adjacent in TMEM; V h0, V h1, dV h0, dV h1 are 8 KB apart).
-#pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts(tmem + TM_A1, a_p + ks * 8, vb + ((ks * 2048) >> 4), IDESC_PVV,
-                 first | (ks > 0));
-        // A23 += (scale e dS) V
-#pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts(tmem + TM_A23, a_pd + ks * 8, vb + ((ks * 2048) >> 4), IDESC_PV, 1u);
-        mma_commit(bar(B_PVD + b));  // PV(t) done: V stage b free, A1/A23 current
-        return true;
+        return wait_bar(bar(B_VFULL + b), (c.t >> 1) & 1u, p, abort_flag);
       };
+      // [S | Q dK^T] = Q [K ; dK]^T: one N=128 MMA per 16-wide k-step.
+      auto issue_s_a = [&](const Cursor& c) {
+        const uint32_t b = c.t & 1u;
+        const uint64_t kb = k_desc + b * (kStageBytes >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t oq = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
+          const uint32_t ob = ((kk >> 2) * (2 * kKHalf) + (kk & 3) * 32) >> 4;
+          mma_ss(tmem + b * 128u, q_desc + oq, kb + ob, IDESC_SK, kk > 0);
+        }
+      };
+      // dS = Q dK^T + dQ K^T: N=64 MMAs accumulate dQ K^T onto it.
+      auto issue_s_b = [&](uint32_t b) {
+        const uint64_t kb = k_desc + b * (kStageBytes >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t oq = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
+          const uint32_t ob = ((kk >> 2) * (2 * kKHalf) + (kk & 3) * 32) >> 4;
+          mma_ss(tmem + b * 128u + 64u, dq_desc + oq, kb + ob, IDESC_S, 1u);
+        }
+      };
+      // [A1 | A23] += P [V | dV]: one N=256 MMA per 16-key step (A1 and A23
+      // are adjacent in TMEM; V h0, V h1, dV h0, dV h1 are 8 KB apart).
+      auto issue_pv_a = [&](const Cursor& c) {
+        const uint32_t b = c.t & 1u;
+        const uint64_t vb = v_desc + b * (kStageBytes >> 4);
+        const uint32_t first = c.j == 0 ? 0u : 1u;
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks)
+          mma_ts(tmem + TM_A1, tmem + b * 128u + ks * 8, vb + ((ks * 2048) >> 4), IDESC_PVV,
+                 first | (ks > 0));
+      };
+      // A23 += (scale e dS) V
+      auto issue_pv_b = [&](uint32_t b) {
+        const uint64_t vb = v_desc + b * (kStageBytes >> 4);
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks)
+          mma_ts(tmem + TM_A23, tmem + b * 128u + 64u + ks * 8, vb + ((ks * 2048) >> 4),
+                 IDESC_PV, 1u);
+      };
+      // Order S(0) S(1) PV(0) S(2) PV(1) ...: S(t+2) overwrites the buffer
+      // whose P PV(t) reads, and one thread's MMAs run in issue order.
       Cursor cs, cp;
       cs.start(p, ring, kConsumerThread);
       cp.start(p, ring, kConsumerThread);
       for (int pre = 0; pre < 2 && cs.valid && ok; ++pre) {
-        ok = issue_s(cs);
+        ok = wait_s(cs);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t b = cs.t & 1u;
+        const bool last = cs.j == cs.n - 1;
+        issue_s_a(cs);
+        issue_s_b(b);
+        mma_commit(bar(B_SFULL + b));  // also releases K stage b to the producer
+        if (last) mma_commit(bar(B_QEMPTY));
         cs.next(p, ring, kConsumerThread);
       }
-      while (cp.valid && ok) {
-        ok = issue_pv(cp);
+      if (ok && cp.valid) ok = wait_pv(cp);
+      while (ok && cp.valid) {
+        tc_fence_after();
+        const uint32_t bp = cp.t & 1u;
+        issue_pv_a(cp);
+        // while PV(t)'s first half runs: the waits for S(t+2)
+        const bool have_s = cs.valid;
+        if (have_s) ok = wait_s(cs);
+        tc_fence_after();
+        issue_pv_b(bp);
+        mma_commit(bar(B_PVD + bp));  // PV(t) done: V stage free, A1/A23 current
         cp.next(p, ring, kConsumerThread);
-        if (ok && cs.valid) {
-          ok = issue_s(cs);
+        if (!ok) break;
+        if (have_s) {
+          const uint32_t bs = cs.t & 1u;
+          const bool last = cs.j == cs.n - 1;
+          issue_s_a(cs);
+          // while S(t+2)'s first half runs: the cursor step and the waits
+          // for PV(t+1)
           cs.next(p, ring, kConsumerThread);
+          if (cp.valid) ok = wait_pv(cp);
+          issue_s_b(bs);
+          mma_commit(bar(B_SFULL + bs));
+          if (last) mma_commit(bar(B_QEMPTY));
+        } else if (cp.valid) {
+          ok = wait_pv(cp);
         }
       }
       if (!ok || *abort_flag) {
