@@ -262,17 +262,28 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       // (barrier checks, commits, cursor steps) lets it run dry. So each
       // batch is issued in two halves, and the waits for the next batch and
       // the cursor step go between them, while the first half executes.
+      // Each wait first tests all of its barriers back to back (one latency
+      // instead of one per barrier; they are normally complete already) and
+      // falls back to the bounded waits one by one.
       auto wait_s = [&](const Cursor& c) -> bool {  // S(t): Q (new item), K|dK stage
-        if (c.j == 0 && !wait_bar(bar(B_QFULL), c.item_idx & 1, p, abort_flag)) return false;
-        return wait_bar(bar(B_KFULL + (c.t & 1u)), (c.t >> 1) & 1u, p, abort_flag);
+        const uint32_t bk = bar(B_KFULL + (c.t & 1u)), pk = (c.t >> 1) & 1u;
+        const bool need_q = c.j == 0;
+        const bool rk = mbar_test(bk, pk);
+        const bool rq = !need_q || mbar_test(bar(B_QFULL), c.item_idx & 1);
+        if (rk && rq) return true;
+        if (need_q && !wait_bar(bar(B_QFULL), c.item_idx & 1, p, abort_flag)) return false;
+        return wait_bar(bk, pk, p, abort_flag);
       };
       auto wait_pv = [&](const Cursor& c) -> bool {  // PV(t): accumulators, P, V|dV stage
-        const uint32_t b = c.t & 1u;
-        if (c.j == 0 && c.item_idx > 0 &&
-            !wait_bar(bar(B_AFREE), (c.item_idx - 1) & 1, p, abort_flag))
-          return false;
-        if (!wait_bar(bar(B_PFULL + b), (c.t >> 1) & 1u, p, abort_flag)) return false;
-        return wait_bar(bar(B_VFULL + b), (c.t >> 1) & 1u, p, abort_flag);
+        const uint32_t b = c.t & 1u, par = (c.t >> 1) & 1u;
+        const bool need_a = c.j == 0 && c.item_idx > 0;
+        const bool rp = mbar_test(bar(B_PFULL + b), par);
+        const bool rv = mbar_test(bar(B_VFULL + b), par);
+        const bool ra = !need_a || mbar_test(bar(B_AFREE), (c.item_idx - 1) & 1);
+        if (rp && rv && ra) return true;
+        if (need_a && !wait_bar(bar(B_AFREE), (c.item_idx - 1) & 1, p, abort_flag)) return false;
+        if (!wait_bar(bar(B_PFULL + b), par, p, abort_flag)) return false;
+        return wait_bar(bar(B_VFULL + b), par, p, abort_flag);
       };
       // [S | Q dK^T] = Q [K ; dK]^T: one N=128 MMA per 16-wide k-step.
       auto issue_s_a = [&](const Cursor& c) {
