@@ -187,3 +187,15 @@ def call_prologue(**kw):
 ])
 def test_prologue_argument_errors(kw, code):
     assert call_prologue(**kw) == code
+
+
+def test_size_limits():
+    # index ranges of the kernels: rejected before any device work
+    assert call_cache(B=70000, H=70000, Lq=1, Lk=1, Lcache=1) == _lib.JVP_ERR_TOO_LARGE
+    fp = ctypes.POINTER(ctypes.c_float)
+    rc = _lib.lib().jvp_attn_bwd(*[FAKE] * 5, ctypes.cast(FAKE, fp), *[FAKE] * 3,
+                                 ctypes.cast(FAKE, fp), 1 << 40, 70000, 70000, 64, 128,
+                                 _lib.JVP_BF16, _lib.MaskDesc(ja.TEACHER_FORCING, 8, 4, 1), 0.0,
+                                 None)
+    assert rc == _lib.JVP_ERR_TOO_LARGE
+    assert call_prologue(B=1 << 20, L=1 << 15, rope_rows=1 << 15) == _lib.JVP_ERR_TOO_LARGE

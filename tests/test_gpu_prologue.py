@@ -84,3 +84,24 @@ def test_prologue_then_attention_jvp():
                           sin.cpu())
     for name, got, ref in zip(("q", "k", "v", "dq", "dk", "dv"), (q, k, v, dq, dk, dv), ref_in):
         close_bf16(got, ref, name)
+
+
+@pytest.mark.slow
+def test_prologue_full_size_sampled_tokens():
+    # The bench's shape: 65,520 tokens, 12 heads of 128, norm over all 1,536
+    # channels, RoPE; sampled tokens against the oracle.
+    from attention_jvp_continuous_b200.inputs import sample_rows
+    B, L, H, d = 1, 65520, 12, 128
+    C = H * d
+    P = randn(20, (B, L, 3 * C), std=2.0)
+    dP = randn(21, (B, L, 3 * C), std=0.1)
+    wq = randn(22, (C,), torch.float32) * 0.2 + 1.0
+    wk = randn(23, (C,), torch.float32) * 0.2 + 1.0
+    cos, sin = rope_table(L, d, device="cuda")
+    out = ja.qkv_prologue(P, dP, H, wq, wk, C, 1e-6, cos, sin)
+    torch.cuda.synchronize()
+    rows = torch.from_numpy(sample_rows(L, 48, seed=3))
+    ref = qkv_prologue(P[:, rows].cpu(), dP[:, rows].cpu(), H, d, wq.cpu(), wk.cpu(), C, 1e-6,
+                       cos[rows.cuda()].cpu(), sin[rows.cuda()].cpu())
+    for name, o, r in zip(("q", "k", "v", "dq", "dk", "dv"), out, ref):
+        close_bf16(o[:, :, rows.cuda()], r, name)
