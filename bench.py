@@ -239,19 +239,59 @@ def device_timed(step, steps: int, world: int, local: int, stream, ja):
     return per, total, clk.summary()
 
 
-def e2e_timed(e2e_step, steps: int, world: int, stream, ja) -> float:
-    """Max-over-ranks ms of ``steps`` end-to-end steps (one untimed first)."""
+def e2e_pipelined(host_in, out_like, compute, steps: int, world: int, ja) -> float:
+    """End-to-end throughput of a stream of batches held in pinned host
+    memory: every step copies its inputs host->device, runs ``compute``
+    (dev_in, dev_out) through the library and copies its outputs back.
+    Double-buffered on three streams (copy in, compute, copy out) ordered by
+    events, so that step i+1's inputs and step i-1's outputs cross the host
+    link while step i computes. Returns the max-over-ranks ms of ``steps``
+    steps, from before the first copy in to after the last copy out."""
     import torch
     import torch.distributed as dist
-    e2e_step()
+    cs = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    dev_in = [[torch.empty(h.shape, dtype=h.dtype, device="cuda") for h in host_in]
+              for _ in range(2)]
+    dev_out = [[torch.empty_like(t) for t in out_like] for _ in range(2)]
+    host_out = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in out_like]
+                for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def run(n, start_ev=None):
+        if start_ev is not None:
+            s_in.wait_event(start_ev)
+        for i in range(n):
+            k = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_done[k])  # buffer k's last compute finished
+                for d, h in zip(dev_in[k], host_in):
+                    d.copy_(h, non_blocking=True)
+                ev_in[k].record(s_in)
+            cs.wait_event(ev_in[k])
+            if i >= 2:
+                cs.wait_event(ev_out[k])  # buffer k's last outputs copied out
+            compute(dev_in[k], dev_out[k])
+            ev_done[k].record(cs)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[k])
+                for h, d in zip(host_out[k], dev_out[k]):
+                    h.copy_(d, non_blocking=True)
+                ev_out[k].record(s_out)
+        cs.wait_stream(s_in)
+        cs.wait_stream(s_out)
+
+    run(2)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(cs)
+    run(steps, e0)
+    e1.record(cs)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -317,24 +357,18 @@ def run_ours(args, w):
 
     # ---- end to end through the C ABI: pinned host in, host out ----
     host_in = [t.cpu().pin_memory() for t in step_in]
-    dev_in = [torch.empty_like(t) for t in step_in]
-    dev_out = grads if bwd else [o, d_o, lse]
-    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in dev_out]
+    out_like = grads if bwd else [o, d_o, lse]
     h2d = sum(t.numel() * t.element_size() for t in host_in)
-    d2h = sum(t.numel() * t.element_size() for t in host_out)
-    e2e_steps = max(1, min(args.steps, 5))
+    d2h = sum(t.numel() * t.element_size() for t in out_like)
+    e2e_steps = max(2, min(args.steps, 10))
 
-    def e2e_step():
-        for d, h in zip(dev_in, host_in):
-            d.copy_(h, non_blocking=True)
+    def compute(dev_in, dev_out):
         if bwd:
-            ja.jvp_attn_bwd(*dev_in, *grads, scratch, mask)
+            ja.jvp_attn_bwd(*dev_in, *dev_out, scratch, mask)
         else:
-            ja.jvp_attn_fwd(*dev_in, o, d_o, lse, mask)
-        for h, d in zip(host_out, dev_out):
-            h.copy_(d, non_blocking=True)
+            ja.jvp_attn_fwd(*dev_in, *dev_out, mask)
 
-    e2e_ms = e2e_timed(e2e_step, e2e_steps, world, stream, ja)
+    e2e_ms = e2e_pipelined(host_in, out_like, compute, e2e_steps, world, ja)
     e2e_value = flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
 
     if world > 1:
@@ -368,7 +402,10 @@ def run_ours(args, w):
             "parallelism": f"dp{world} (independent problems per rank, no data collective)",
         },
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "note": "pinned host batches; copies in, compute and copies out on three "
+                        "streams, double-buffered (step i+1's inputs and step i-1's outputs "
+                        "move while step i computes)"},
         "gpu_launches": args.steps * (2 if bwd else 1),
         "roofline": {
             "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": UNIT,
@@ -453,19 +490,16 @@ def run_ours_cache(args, w):
     # end to end: the chunk's q, k, v from pinned host memory, o and LSE back;
     # the cache is rollout state and stays in HBM
     host_in = [t.cpu().pin_memory() for t in (q, k_cur, v_cur)]
-    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, lse)]
 
-    def e2e_step():
-        for dv, hv in zip((q, k_cur, v_cur), host_in):
-            dv.copy_(hv, non_blocking=True)
-        step()
-        for hv, dv in zip(host_out, (o, lse)):
-            hv.copy_(dv, non_blocking=True)
+    def compute(dev_in, dev_out):
+        ja.rope_copy(dev_in[1], kc, Lq, 0, pos, cos, sin, rope_row0=pos)
+        ja.rope_copy(dev_in[2], vc, Lq, 0, pos)
+        ja.cache_attn(dev_in[0], kc, vc, Lk, dev_out[0], dev_out[1])
 
-    e2e_steps = max(1, min(args.steps, 5))
-    e2e_ms = e2e_timed(e2e_step, e2e_steps, world, stream, ja)
+    e2e_steps = max(2, min(args.steps, 10))
+    e2e_ms = e2e_pipelined(host_in, [o, lse], compute, e2e_steps, world, ja)
     h2d = sum(t.numel() * t.element_size() for t in host_in)
-    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    d2h = sum(t.numel() * t.element_size() for t in (o, lse))
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -492,7 +526,8 @@ def run_ours_cache(args, w):
         "e2e": {"value": round(flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12, 2),
                 "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps,
-                "note": "chunk q, k, v in and o, lse out; the cache stays resident"},
+                "note": "chunk q, k, v in and o, lse out (pipelined as in the jvp op); "
+                        "the cache stays resident"},
         "gpu_launches": args.steps * 4,
         "roofline": {
             "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": UNIT,
@@ -553,17 +588,12 @@ def run_ours_prologue(args, w):
     value = nbytes * args.steps * world / (total_ms_max * 1e-3) / 1e9
     launch_ms = sum(per) / len(per)
     host_in = [t.cpu().pin_memory() for t in (P, dP)]
-    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in out]
 
-    def e2e_step():
-        for dv, hv in zip((P, dP), host_in):
-            dv.copy_(hv, non_blocking=True)
-        step()
-        for hv, dv in zip(host_out, out):
-            hv.copy_(dv, non_blocking=True)
+    def compute(dev_in, dev_out):
+        ja.qkv_prologue(dev_in[0], dev_in[1], H, wq, wk, C, 1e-6, cos, sin, out=dev_out)
 
-    e2e_steps = max(1, min(args.steps, 5))
-    e2e_ms = e2e_timed(e2e_step, e2e_steps, world, stream, ja)
+    e2e_steps = max(2, min(args.steps, 10))
+    e2e_ms = e2e_pipelined(host_in, out, compute, e2e_steps, world, ja)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -587,8 +617,8 @@ def run_ours_prologue(args, w):
         "e2e": {"value": round(nbytes * e2e_steps * world / (e2e_ms * 1e-3) / 1e9, 1),
                 "unit": "GB/s", "h2d_bytes_per_step": sum(t.numel() * t.element_size()
                                                           for t in host_in),
-                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in host_out),
-                "steps": e2e_steps},
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in out),
+                "steps": e2e_steps, "note": "pipelined as in the jvp op"},
         "gpu_launches": args.steps,
         "roofline": {
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
