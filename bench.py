@@ -849,7 +849,7 @@ def main(argv=None):
                     choices=["tf", "frame_causal", "chunk_tf", "tf_long"])
     ap.add_argument("--cpu-rows", type=int, default=3072,
                     help="query rows per head in the cpu_baseline sample")
-    ap.add_argument("--ref-rows", type=int, default=32,
+    ap.add_argument("--ref-rows", type=int, default=256,
                     help="query rows per head per step of --impl reference")
     ap.add_argument("--cpu-rows-bwd", type=int, default=1024,
                     help="query rows per head in the --op bwd cpu_baseline sample")
