@@ -1,5 +1,5 @@
 """Failure detection on the GPU without faulting it: every wait inside the
-tensor-core kernel is bounded. With a 1 ns limit the first wait that cannot
+tensor-core kernels (attention JVP, backward, cache attention) is bounded. With a 1 ns limit the first wait that cannot
 be satisfied at once gives up; the kernel records a timeout in the device
 error word, drains its own copies and MMAs, frees its tensor memory and
 exits. The host reads the error, and the same context then computes correct
@@ -45,3 +45,47 @@ def test_wait_timeout_is_reported_and_context_recovers():
     for got, want in ((o, ref[0]), (do, ref[1])):
         g = got.float().cpu().numpy().astype(np.float64)
         assert np.linalg.norm(g - want) <= 5e-3 * np.linalg.norm(want)
+
+
+def _timeout_then_recover(run, check):
+    ja.check_device_error()
+    try:
+        ja.set_wait_limit(1)
+        run()
+        with pytest.raises(ja.JvpAttnError) as e:
+            ja.check_device_error()
+        assert e.value.code == _lib.JVP_ERR_DEVICE_TIMEOUT
+    finally:
+        ja.set_wait_limit(0)
+    ja.check_device_error()
+    check(run())
+    ja.check_device_error()
+
+
+def test_backward_and_cache_waits_are_bounded_too():
+    from oracle import cache_attention
+    from oracle.attention_backward import attention_backward
+    w = Workload("fault_bwd", 1, 2, 128, ja.TEACHER_FORCING, 100, 3, 1, "bf16", 1.0)
+    spec = MaskSpec(w.mode, w.tokens_per_frame, w.n_frames, w.chunk)
+    mask = ja.Mask(w.mode, w.tokens_per_frame, w.n_frames, w.chunk)
+    (q, k, v, g, *_), _ = make_inputs(w, device="cpu")
+    dq, dk, dv, dg = (t.cuda() for t in (q, k, v, g))
+    o, _, lse = ja.jvp_attn(dq, dk, dv, *(torch.zeros_like(t) for t in (dq, dk, dv)), mask)
+    ja.check_device_error()
+    ref = attention_backward(q, k, v, g, spec)
+
+    def check_bwd(grads):
+        for got, want in zip(grads, ref):
+            gg = got.float().cpu().numpy().astype(np.float64)
+            assert np.linalg.norm(gg - want) <= 1e-2 * np.linalg.norm(want)
+
+    _timeout_then_recover(lambda: ja.attn_bwd(dq, dk, dv, o, dg, lse, mask), check_bwd)
+
+    Lk = 500
+    ref_o, _ = cache_attention(q, k, v, Lk)
+
+    def check_cache(res):
+        gg = res[0].float().cpu().numpy().astype(np.float64)
+        assert np.linalg.norm(gg - ref_o) <= 5e-3 * np.linalg.norm(ref_o)
+
+    _timeout_then_recover(lambda: ja.cache_attn(dq, dk, dv, Lk), check_cache)
