@@ -17,7 +17,8 @@
 //
 // Warp roles (384 threads, one CTA per SM, persistent over the work list):
 //   warp 0       TMA producer: Q/dQ per query tile, K|dK and V|dV rings of 2
-//   warp 1       TMEM owner and MMA issuer (one thread)
+//   warp 1       TMEM owner and MMA issuer (the whole warp runs the loop;
+//                one elected lane issues)
 //   warps 4..11  softmax/JVP state, P write-back to TMEM, epilogue: two
 //                warpgroups, each taking 32 of a tile's 64 key columns of
 //                every row (one row per thread), exchanging row maxima
@@ -248,7 +249,11 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA ----
-    if (lane == 0) {
+    // The whole warp runs the issue loop (uniform control flow keeps the
+    // descriptors in the uniform datapath); one elected lane issues each MMA
+    // and commit. This issues faster than a lone lane 0 when the softmax
+    // warps share the scheduler.
+    {
       bool ok = true;
       // Descriptors of the fixed shared-memory operands; an MMA's operand
       // is the base plus a compile-time byte offset >> 4 (the start-address
@@ -270,9 +275,10 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const bool need_q = c.j == 0;
         const bool rk = mbar_test(bk, pk);
         const bool rq = !need_q || mbar_test(bar(B_QFULL), c.item_idx & 1);
-        if (rk && rq) return true;
-        if (need_q && !wait_bar(bar(B_QFULL), c.item_idx & 1, p, abort_flag)) return false;
-        return wait_bar(bk, pk, p, abort_flag);
+        if (__all_sync(0xffffffffu, rk && rq)) return true;
+        bool w = !need_q || wait_bar(bar(B_QFULL), c.item_idx & 1, p, abort_flag);
+        w = w && wait_bar(bk, pk, p, abort_flag);
+        return __all_sync(0xffffffffu, w);
       };
       auto wait_pv = [&](const Cursor& c) -> bool {  // PV(t): accumulators, P, V|dV stage
         const uint32_t b = c.t & 1u, par = (c.t >> 1) & 1u;
@@ -280,10 +286,11 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const bool rp = mbar_test(bar(B_PFULL + b), par);
         const bool rv = mbar_test(bar(B_VFULL + b), par);
         const bool ra = !need_a || mbar_test(bar(B_AFREE), (c.item_idx - 1) & 1);
-        if (rp && rv && ra) return true;
-        if (need_a && !wait_bar(bar(B_AFREE), (c.item_idx - 1) & 1, p, abort_flag)) return false;
-        if (!wait_bar(bar(B_PFULL + b), par, p, abort_flag)) return false;
-        return wait_bar(bar(B_VFULL + b), par, p, abort_flag);
+        if (__all_sync(0xffffffffu, rp && rv && ra)) return true;
+        bool w = !need_a || wait_bar(bar(B_AFREE), (c.item_idx - 1) & 1, p, abort_flag);
+        w = w && wait_bar(bar(B_PFULL + b), par, p, abort_flag);
+        w = w && wait_bar(bar(B_VFULL + b), par, p, abort_flag);
+        return __all_sync(0xffffffffu, w);
       };
       // [S | Q dK^T] = Q [K ; dK]^T: one N=128 MMA per 16-wide k-step.
       auto issue_s_a = [&](const Cursor& c) {
@@ -293,7 +300,7 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t oq = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
           const uint32_t ob = ((kk >> 2) * (2 * kKHalf) + (kk & 3) * 32) >> 4;
-          mma_ss(tmem + b * 128u, q_desc + oq, kb + ob, IDESC_SK, kk > 0);
+          mma_ss_elect(tmem + b * 128u, q_desc + oq, kb + ob, IDESC_SK, kk > 0);
         }
       };
       // dS = Q dK^T + dQ K^T: N=64 MMAs accumulate dQ K^T onto it.
@@ -303,7 +310,7 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t oq = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
           const uint32_t ob = ((kk >> 2) * (2 * kKHalf) + (kk & 3) * 32) >> 4;
-          mma_ss(tmem + b * 128u + 64u, dq_desc + oq, kb + ob, IDESC_S, 1u);
+          mma_ss_elect(tmem + b * 128u + 64u, dq_desc + oq, kb + ob, IDESC_S, 1u);
         }
       };
       // [A1 | A23] += P [V | dV]: one N=256 MMA per 16-key step (A1 and A23
@@ -314,7 +321,7 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t first = c.j == 0 ? 0u : 1u;
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts(tmem + TM_A1, tmem + b * 128u + ks * 8, vb + ((ks * 2048) >> 4), IDESC_PVV,
+          mma_ts_elect(tmem + TM_A1, tmem + b * 128u + ks * 8, vb + ((ks * 2048) >> 4), IDESC_PVV,
                  first | (ks > 0));
       };
       // A23 += (scale e dS) V
@@ -322,14 +329,15 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint64_t vb = v_desc + b * (kStageBytes >> 4);
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts(tmem + TM_A23, tmem + b * 128u + 64u + ks * 8, vb + ((ks * 2048) >> 4),
+          mma_ts_elect(tmem + TM_A23, tmem + b * 128u + 64u + ks * 8, vb + ((ks * 2048) >> 4),
                  IDESC_PV, 1u);
       };
       // Order S(0) S(1) PV(0) S(2) PV(1) ...: S(t+2) overwrites the buffer
-      // whose P PV(t) reads, and one thread's MMAs run in issue order.
+      // whose P PV(t) reads, and the MMAs of one issuing lane run in issue
+      // order (elect.sync picks the same lane while the warp is converged).
       Cursor cs, cp;
-      cs.start(p, ring, kConsumerThread);
-      cp.start(p, ring, kConsumerThread);
+      cs.start(p, ring, kConsumerWarp);
+      cp.start(p, ring, kConsumerWarp);
       for (int pre = 0; pre < 2 && cs.valid && ok; ++pre) {
         ok = wait_s(cs);
         if (!ok) break;
@@ -338,9 +346,9 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const bool last = cs.j == cs.n - 1;
         issue_s_a(cs);
         issue_s_b(b);
-        mma_commit(bar(B_SFULL + b));  // also releases K stage b to the producer
-        if (last) mma_commit(bar(B_QEMPTY));
-        cs.next(p, ring, kConsumerThread);
+        mma_commit_elect(bar(B_SFULL + b));  // also releases K stage b to the producer
+        if (last) mma_commit_elect(bar(B_QEMPTY));
+        cs.next(p, ring, kConsumerWarp);
       }
       if (ok && cp.valid) ok = wait_pv(cp);
       while (ok && cp.valid) {
@@ -352,8 +360,8 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (have_s) ok = wait_s(cs);
         tc_fence_after();
         issue_pv_b(bp);
-        mma_commit(bar(B_PVD + bp));  // PV(t) done: V stage free, A1/A23 current
-        cp.next(p, ring, kConsumerThread);
+        mma_commit_elect(bar(B_PVD + bp));  // PV(t) done: V stage free, A1/A23 current
+        cp.next(p, ring, kConsumerWarp);
         if (!ok) break;
         if (have_s) {
           const uint32_t bs = cs.t & 1u;
@@ -361,18 +369,18 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           issue_s_a(cs);
           // while S(t+2)'s first half runs: the cursor step and the waits
           // for PV(t+1)
-          cs.next(p, ring, kConsumerThread);
+          cs.next(p, ring, kConsumerWarp);
           if (cp.valid) ok = wait_pv(cp);
           issue_s_b(bs);
-          mma_commit(bar(B_SFULL + bs));
-          if (last) mma_commit(bar(B_QEMPTY));
+          mma_commit_elect(bar(B_SFULL + bs));
+          if (last) mma_commit_elect(bar(B_QEMPTY));
         } else if (cp.valid) {
           ok = wait_pv(cp);
         }
       }
       if (!ok || *abort_flag) {
-        // Wait for every MMA this thread issued before TMEM is freed.
-        mma_commit(bar(B_DRAIN));
+        // Wait for every MMA this warp issued before TMEM is freed.
+        mma_commit_elect(bar(B_DRAIN));
         drain_wait(bar(B_DRAIN), 0);
       }
     }
