@@ -21,7 +21,7 @@ TEACHER_FORCING = 3
 
 __all__ = ["Mask", "jvp_attn", "jvp_attn_fwd", "attn_bwd", "jvp_attn_bwd", "bwd_scratch_len",
            "cache_attn", "rope_copy", "qkv_prologue", "mask_stats", "tile_classes",
-           "schedule", "schedule_kv", "check_device_error", "set_wait_limit", "release",
+           "schedule", "schedule_kv", "check_device_error", "set_wait_limit", "set_stall_test", "release",
            "JvpAttnError",
            "DENSE", "FRAME_CAUSAL", "CHUNK_CAUSAL", "TEACHER_FORCING"]
 
@@ -324,8 +324,14 @@ def check_device_error(stream: Optional[int] = None) -> None:
 
 
 def set_wait_limit(ns: int) -> None:
-    """Per-wait limit of the tensor-core kernel in ns (0 = default, 2 s)."""
+    """Per-wait limit of the tensor-core kernels in ns (0 = default, 2 s)."""
     _lib.check(_lib.lib().jvp_attn_set_wait_limit(int(ns)), "jvp_attn_set_wait_limit")
+
+
+def set_stall_test(enable: bool) -> None:
+    """Failure-detection test switch: while on, every tensor-core launch ends
+    through its bounded-wait timeout path (JVP_ERR_DEVICE_TIMEOUT)."""
+    _lib.check(_lib.lib().jvp_attn_set_stall_test(1 if enable else 0), "jvp_attn_set_stall_test")
 
 
 def release() -> None:

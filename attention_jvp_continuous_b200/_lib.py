@@ -37,7 +37,7 @@ EXPORTS = ("jvp_attn_fwd", "jvp_attn_fwd_noalloc", "jvp_attn_bwd", "jvp_attn_bwd
            "jvp_attn_mask_stats",
            "jvp_attn_tile_classes", "jvp_attn_schedule", "jvp_attn_schedule_kv",
            "jvp_attn_check_device_error",
-           "jvp_attn_set_wait_limit", "jvp_attn_release", "jvp_attn_strerror",
+           "jvp_attn_set_wait_limit", "jvp_attn_set_stall_test", "jvp_attn_release", "jvp_attn_strerror",
            "jvp_attn_version")
 
 
@@ -105,6 +105,8 @@ def lib() -> ctypes.CDLL:
         L.jvp_attn_check_device_error.restype = i32
         L.jvp_attn_set_wait_limit.argtypes = [ctypes.c_uint64]
         L.jvp_attn_set_wait_limit.restype = i32
+        L.jvp_attn_set_stall_test.argtypes = [i32]
+        L.jvp_attn_set_stall_test.restype = i32
         L.jvp_attn_release.argtypes = []
         L.jvp_attn_release.restype = i32
         L.jvp_attn_strerror.argtypes = [i32]

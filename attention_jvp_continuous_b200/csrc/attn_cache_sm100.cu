@@ -39,7 +39,6 @@ namespace cache {
 using namespace jvp::ptx;
 using pipe::drain_wait;
 using pipe::ItemRing;
-using pipe::kConsumerThread;
 using pipe::kConsumerWarp;
 using pipe::kProducer;
 using pipe::kRing;
@@ -106,6 +105,7 @@ struct Params {
   unsigned* err;
   unsigned* item_ctr;
   unsigned long long wait_limit_ns;
+  int stall_test;  // the MMA warp first waits on a phase that nothing completes
 };
 using Cursor = pipe::Cursor<Params>;
 
@@ -212,34 +212,39 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA ----
-    if (lane == 0) {
+    // The whole warp runs the loop in uniform control flow; one elected lane
+    // issues each MMA and commit.
+    {
       bool ok = true;
+      auto wait_w = [&](uint32_t b_, uint32_t par_) -> bool {
+        return __all_sync(0xffffffffu, wait_bar(b_, par_, p, abort_flag));
+      };
       const uint64_t q_desc = sdesc_sw128(base + SM_Q, 16, 1024);
       const uint64_t k_desc = sdesc_sw128(base + SM_K, 16, 1024);     // K-major, stage 0
       const uint64_t v_desc = sdesc_sw128(base + SM_V, kHalf, 1024);  // MN-major, stage 0
       auto issue_s = [&](const Cursor& c) -> bool {
         const uint32_t b = c.t & 1u, sk = c.t % NK;
-        if (c.j == 0 && !wait_bar(bar(B_QFULL), c.item_idx & 1, p, abort_flag)) return false;
-        if (!wait_bar(bar(B_KFULL + sk), (c.t / NK) & 1u, p, abort_flag)) return false;
+        if (c.j == 0 && !wait_w(bar(B_QFULL), c.item_idx & 1)) return false;
+        if (!wait_w(bar(B_KFULL + sk), (c.t / NK) & 1u)) return false;
         tc_fence_after();
         const uint64_t kb = k_desc + sk * (kStage >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
-          mma_ss(tmem + b * 128u, q_desc + off, kb + off, IDESC_S, kk > 0);
+          mma_ss_elect(tmem + b * 128u, q_desc + off, kb + off, IDESC_S, kk > 0);
         }
-        mma_commit(bar(B_SFULL + b));
-        mma_commit(bar(B_KEMPTY + sk));
-        if (c.j == c.n - 1) mma_commit(bar(B_QEMPTY));
+        mma_commit_elect(bar(B_SFULL + b));
+        mma_commit_elect(bar(B_KEMPTY + sk));
+        if (c.j == c.n - 1) mma_commit_elect(bar(B_QEMPTY));
         return true;
       };
       auto issue_pv = [&](const Cursor& c) -> bool {
         const uint32_t b = c.t & 1u;
         if (c.j == 0 && c.item_idx > 0 &&
-            !wait_bar(bar(B_AFREE), (c.item_idx - 1) & 1, p, abort_flag))
+            !wait_w(bar(B_AFREE), (c.item_idx - 1) & 1))
           return false;
-        if (!wait_bar(bar(B_PFULL + b), (c.t >> 1) & 1u, p, abort_flag)) return false;
-        if (!wait_bar(bar(B_VFULL + b), (c.t >> 1) & 1u, p, abort_flag)) return false;
+        if (!wait_w(bar(B_PFULL + b), (c.t >> 1) & 1u)) return false;
+        if (!wait_w(bar(B_VFULL + b), (c.t >> 1) & 1u)) return false;
         tc_fence_after();
         const uint64_t vb = v_desc + b * (kStage >> 4);
         const uint32_t first = c.j == 0 ? 0u : 1u;
@@ -249,32 +254,36 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         // softmax warpgroup h itself read.
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts(tmem + TM_O + (ks >> 2) * 128u,
+          mma_ts_elect(tmem + TM_O + (ks >> 2) * 128u,
                  tmem + b * 128u + (ks >> 2) * 64u + (ks & 3) * 8u,
                  vb + ((ks * 2048) >> 4), IDESC_PV, first | ((ks & 3) > 0));
-        mma_commit(bar(B_VEMPTY + b));
-        mma_commit(bar(B_PVD + b));
+        mma_commit_elect(bar(B_VEMPTY + b));
+        mma_commit_elect(bar(B_PVD + b));
         return true;
       };
       // Order S(0) S(1) PV(0) S(2) PV(1) ...: S(t+2) overwrites the buffer
-      // whose P PV(t) reads, and one thread's MMAs run in issue order.
+      // whose P PV(t) reads, and the MMAs of one issuing lane run in issue order.
       Cursor cs, cp;
-      cs.start(p, ring, kConsumerThread);
-      cp.start(p, ring, kConsumerThread);
+      cs.start(p, ring, kConsumerWarp);
+      cp.start(p, ring, kConsumerWarp);
+      // Failure-detection test: wait on the drain barrier's first phase,
+      // which nothing completes before this warp's own drain commit, so the
+      // bounded wait runs out and the abort path below is taken.
+      if (p.stall_test) ok = __all_sync(0xffffffffu, wait_bar(bar(B_DRAIN), 0u, p, abort_flag));
       for (int pre = 0; pre < 2 && cs.valid && ok; ++pre) {
         ok = issue_s(cs);
-        cs.next(p, ring, kConsumerThread);
+        cs.next(p, ring, kConsumerWarp);
       }
       while (cp.valid && ok) {
         ok = issue_pv(cp);
-        cp.next(p, ring, kConsumerThread);
+        cp.next(p, ring, kConsumerWarp);
         if (ok && cs.valid) {
           ok = issue_s(cs);
-          cs.next(p, ring, kConsumerThread);
+          cs.next(p, ring, kConsumerWarp);
         }
       }
-      if (!ok || *abort_flag) {
-        mma_commit(bar(B_DRAIN));
+      if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
+        mma_commit_elect(bar(B_DRAIN));
         drain_wait(bar(B_DRAIN), 0);
       }
     }
@@ -568,6 +577,7 @@ int launch_cache_sm100(const CacheArgs& a, const WorkList& w, int splits, int nu
   p.err = a.err;
   p.item_ctr = a.item_ctr;
   p.wait_limit_ns = a.wait_limit_ns;
+  p.stall_test = a.stall_test ? 1 : 0;
   if (p.split && (!p.part || !p.ml)) return JVP_ERR_LAUNCH_FAILED;
   static std::mutex attr_mu;
   static bool attr_done[64] = {};

@@ -34,6 +34,7 @@ struct LaunchArgs {
   // the launch). Launches that share a counter must be stream-ordered.
   unsigned* item_ctr = nullptr;
   unsigned long long wait_limit_ns;
+  bool stall_test = false;  // jvp_attn_set_stall_test
 };
 
 // CUDA-core kernel (fp32 arithmetic) for fp32 or bf16 inputs, d in {32,64,96,128}.
@@ -55,6 +56,7 @@ struct BwdArgs {
   unsigned* err;
   unsigned* item_ctr;  // two u32 words: one per pass
   unsigned long long wait_limit_ns;
+  bool stall_test = false;  // jvp_attn_set_stall_test
 };
 
 // Backward passes (dQ, then dK/dV): bf16, d = 128, sm_100a. wq: query-tile
@@ -72,6 +74,7 @@ struct CacheArgs {
   unsigned* err;
   unsigned* item_ctr;
   unsigned long long wait_limit_ns;
+  bool stall_test = false;  // jvp_attn_set_stall_test
   float* part;  // split > 1: [items, 128, 128] fp32 partial outputs
   float* ml;    // split > 1: [items, 128] {max, sum} pairs
 };
@@ -103,8 +106,10 @@ struct PrologueArgs {
 };
 int launch_qkv_prologue(const PrologueArgs& a, int num_sms);
 
-// Per-wait limit for the tensor-core kernel (jvp_attn_set_wait_limit).
+// Per-wait limit for the tensor-core kernels (jvp_attn_set_wait_limit).
 unsigned long long wait_limit_ns();
+// Failure-detection test switch of the tensor-core kernels (jvp_attn_set_stall_test).
+bool stall_test();
 
 // Current device's SM count and error word; JVP_ERR_UNSUPPORTED_DEVICE
 // unless it is an sm_100 device. Allocates nothing.

@@ -26,6 +26,7 @@ namespace {
 constexpr int kBM = 128, kBN = 64;            // tensor-core tile shape
 constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;  // 2 s per wait
 std::atomic<unsigned long long> g_wait_limit{kDefaultWaitLimitNs};
+std::atomic<bool> g_stall_test{false};
 constexpr int kMaxDevices = 64;
 
 struct DevInfo {
@@ -202,6 +203,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 }  // namespace
 
 unsigned long long wait_limit_ns() { return g_wait_limit.load(); }
+bool stall_test() { return g_stall_test.load(); }
 
 int current_device_state(int* sms, unsigned** err) {
   DevInfo* di = nullptr;
@@ -250,6 +252,7 @@ int jvp_attn_fwd(const void* q, const void* k, const void* v, const void* dq, co
   a.stream = static_cast<cudaStream_t>(stream);
   a.err = di->err;
   a.wait_limit_ns = wait_limit_ns();
+  a.stall_test = stall_test();
   if (!tensor_core) return launch_simt(a, dtype == JVP_BF16);
 
   int dev = 0;
@@ -294,6 +297,7 @@ int jvp_attn_bwd(const void* q, const void* k, const void* v, const void* o, con
   a.stream = static_cast<cudaStream_t>(stream);
   a.err = di->err;
   a.wait_limit_ns = wait_limit_ns();
+  a.stall_test = stall_test();
   WorkList wq, wkv;
   rc = get_worklist(dev, mask, L, &wq, 128, 64, 0);
   if (rc != JVP_OK) return rc;
@@ -336,6 +340,7 @@ int jvp_attn_cache_fwd(const void* q, const void* k_cache, const void* v_cache, 
   a.stream = static_cast<cudaStream_t>(stream);
   a.err = di->err;
   a.wait_limit_ns = wait_limit_ns();
+  a.stall_test = stall_test();
   a.part = nullptr;
   a.ml = nullptr;
   const int n_qt = (Lq + 127) / 128, n_kt = (Lk + 127) / 128;
@@ -514,6 +519,11 @@ int jvp_attn_check_device_error(void* stream) {
 
 int jvp_attn_set_wait_limit(uint64_t ns) {
   g_wait_limit.store(ns == 0 ? kDefaultWaitLimitNs : (unsigned long long)ns);
+  return JVP_OK;
+}
+
+int jvp_attn_set_stall_test(int enable) {
+  g_stall_test.store(enable != 0);
   return JVP_OK;
 }
 

@@ -38,7 +38,6 @@ namespace bwd {
 using namespace jvp::ptx;
 using pipe::drain_wait;
 using pipe::ItemRing;
-using pipe::kConsumerThread;
 using pipe::kConsumerWarp;
 using pipe::kProducer;
 using pipe::kRing;
@@ -126,6 +125,7 @@ struct Params {
   unsigned* err;
   unsigned* item_ctr;
   unsigned long long wait_limit_ns;
+  int stall_test;  // the MMA warp first waits on a phase that nothing completes
 };
 using Cursor = pipe::Cursor<Params>;
 
@@ -253,8 +253,14 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
     __syncwarp();
   } else if (warp == 1 || warp == 2) {
     // ---------------------------------------------------- MMA issuers ----
-    if (lane == 0) {
+    // Each issuer is a whole warp in uniform control flow; one elected lane
+    // issues its MMAs and commits (faster issue than a lone lane while the
+    // softmax warps share the scheduler).
+    {
       const bool issuer_a = warp == 1;
+      auto wait_w = [&](uint32_t b_, uint32_t par_) -> bool {
+        return __all_sync(0xffffffffu, wait_bar(b_, par_, p, abort_flag));
+      };
       const uint64_t a0_desc = sdesc_sw128(base + LY::A0, 16, 1024);
       const uint64_t a1_desc = sdesc_sw128(base + LY::A1, 16, 1024);
       const uint64_t xk_desc = sdesc_sw128(base + LY::X, 16, 1024);       // K-major view
@@ -264,19 +270,19 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       // First MMAs of tile t: S = A0 X^T (issuer A) or dP = A1 Y^T (issuer B).
       auto issue_first = [&](const Cursor& c, bool s_mma) -> bool {
         const uint32_t b = c.t & 1u;
-        if (c.j == 0 && !wait_bar(bar(B_AF), c.item_idx & 1, p, abort_flag)) return false;
+        if (c.j == 0 && !wait_w(bar(B_AF), c.item_idx & 1)) return false;
         uint32_t stage;
         uint64_t bdesc;
         if (s_mma) {
           // Buffer b last held tile t-2, whose operands acc(t-2) reads.
-          if (c.t >= 2 && !wait_bar(bar(B_MD + b), ((c.t >> 1) - 1) & 1u, p, abort_flag))
+          if (c.t >= 2 && !wait_w(bar(B_MD + b), ((c.t >> 1) - 1) & 1u))
             return false;
           stage = c.t % NX;
-          if (!wait_bar(bar(B_XF + stage), (c.t / NX) & 1u, p, abort_flag)) return false;
+          if (!wait_w(bar(B_XF + stage), (c.t / NX) & 1u)) return false;
           bdesc = xk_desc + stage * (kTile >> 4);
         } else {
           stage = c.t % NY;
-          if (!wait_bar(bar(B_YF + stage), (c.t / NY) & 1u, p, abort_flag)) return false;
+          if (!wait_w(bar(B_YF + stage), (c.t / NY) & 1u)) return false;
           bdesc = yk_desc + stage * (kTile >> 4);
         }
         tc_fence_after();
@@ -285,15 +291,15 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ob = ((kk >> 2) * kTHalf + (kk & 3) * 32) >> 4;
           if (!kKV) {
-            mma_ts(d, tmem + (s_mma ? TM_QA : TM_GA) + 8u * kk, bdesc + ob, IDESC_N64, kk > 0);
+            mma_ts_elect(d, tmem + (s_mma ? TM_QA : TM_GA) + 8u * kk, bdesc + ob, IDESC_N64, kk > 0);
           } else {
             const uint32_t oa = ((kk >> 2) * kRHalf + (kk & 3) * 32) >> 4;
-            mma_ss(d, (s_mma ? a0_desc : a1_desc) + oa, bdesc + ob, IDESC_N64, kk > 0);
+            mma_ss_elect(d, (s_mma ? a0_desc : a1_desc) + oa, bdesc + ob, IDESC_N64, kk > 0);
           }
         }
-        mma_commit(bar(B_SF + b));
-        if (!s_mma && !kKV) mma_commit(bar(B_YE + stage));  // dQ pass: V feeds dP only
-        if (kKV && c.j == c.n - 1) mma_commit(bar(B_AE));   // done with A0 (A) / A1 (B)
+        mma_commit_elect(bar(B_SF + b));
+        if (!s_mma && !kKV) mma_commit_elect(bar(B_YE + stage));  // dQ pass: V feeds dP only
+        if (kKV && c.j == c.n - 1) mma_commit_elect(bar(B_AE));   // done with A0 (A) / A1 (B)
         return true;
       };
       // Accumulating MMAs (issuer B). The bf16 operands of a tile sit in
@@ -302,9 +308,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       auto issue_acc = [&](const Cursor& c) -> bool {
         const uint32_t b = c.t & 1u, sx = c.t % NX, sy = c.t % NY;
         if (c.j == 0 && c.item_idx > 0 &&
-            !wait_bar(bar(B_CF), (c.item_idx - 1) & 1, p, abort_flag))
+            !wait_w(bar(B_CF), (c.item_idx - 1) & 1))
           return false;
-        if (!wait_bar(bar(B_PF + b), (c.t >> 1) & 1u, p, abort_flag)) return false;
+        if (!wait_w(bar(B_PF + b), (c.t >> 1) & 1u)) return false;
         tc_fence_after();
         const uint32_t first = c.j == 0 ? 0u : 1u;
         const uint32_t a_p = tmem + b * 128u;  // dQ pass: dS; dK/dV pass: P^T
@@ -313,52 +319,56 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
           const uint32_t col = (ks >> 1) * 32u + (ks & 1) * 8u;
           if (!kKV) {
             // gQ += dS K
-            mma_ts(tmem + TM_C0, a_p + col, xm_desc + sx * (kTile >> 4) + ((ks * 2048) >> 4),
+            mma_ts_elect(tmem + TM_C0, a_p + col, xm_desc + sx * (kTile >> 4) + ((ks * 2048) >> 4),
                    IDESC_MN, first | (ks > 0));
           } else {
             // gV += P^T G ; gK += dS^T Q
-            mma_ts(tmem + TM_C0, a_p + col, ym_desc + sy * (kTile >> 4) + ((ks * 2048) >> 4),
+            mma_ts_elect(tmem + TM_C0, a_p + col, ym_desc + sy * (kTile >> 4) + ((ks * 2048) >> 4),
                    IDESC_MN, first | (ks > 0));
-            mma_ts(tmem + TM_C1, a_p + 64u + col,
+            mma_ts_elect(tmem + TM_C1, a_p + 64u + col,
                    xm_desc + sx * (kTile >> 4) + ((ks * 2048) >> 4), IDESC_MN,
                    first | (ks > 0));
           }
         }
         // X(t) was also read by S(t), which completed before the softmax
         // warps released tile t.
-        mma_commit(bar(B_XE + sx));
-        if (kKV) mma_commit(bar(B_YE + sy));
-        mma_commit(bar(B_MD + b));
+        mma_commit_elect(bar(B_XE + sx));
+        if (kKV) mma_commit_elect(bar(B_YE + sy));
+        mma_commit_elect(bar(B_MD + b));
         return true;
       };
       bool ok = true;
       if (issuer_a) {
         Cursor cs;
-        cs.start(p, ring, kConsumerThread);
+        cs.start(p, ring, kConsumerWarp);
+        // Failure-detection test: wait on the drain barrier's first phase,
+        // which nothing completes before this warp's own drain commit, so the
+        // bounded wait runs out and the abort path below is taken.
+        if (p.stall_test) ok = __all_sync(0xffffffffu, wait_bar(bar(B_DRAIN + 0), 0u, p, abort_flag));
         while (cs.valid && ok) {
           ok = issue_first(cs, true);
-          cs.next(p, ring, kConsumerThread);
+          cs.next(p, ring, kConsumerWarp);
         }
       } else {
         // dP runs up to two tiles ahead of acc, but not into the next item:
         // that item's stationary operands (dQ pass) are stored only after
         // the epilogue of this one, which waits for this item's last acc.
         Cursor cd, ca;
-        cd.start(p, ring, kConsumerThread);
-        ca.start(p, ring, kConsumerThread);
+        cd.start(p, ring, kConsumerWarp);
+        ca.start(p, ring, kConsumerWarp);
         while (ca.valid && ok) {
           while (ok && cd.valid && cd.t < ca.t + 2 && cd.item_idx == ca.item_idx) {
             ok = issue_first(cd, false);
-            cd.next(p, ring, kConsumerThread);
+            cd.next(p, ring, kConsumerWarp);
           }
           if (!ok) break;
           ok = issue_acc(ca);
-          ca.next(p, ring, kConsumerThread);
+          ca.next(p, ring, kConsumerWarp);
         }
       }
-      if (!ok || *abort_flag) {
+      if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
         const uint32_t db = bar(B_DRAIN + (issuer_a ? 0 : 1));
-        mma_commit(db);
+        mma_commit_elect(db);
         drain_wait(db, 0);
       }
     }
@@ -617,6 +627,7 @@ static int launch_pass(const BwdArgs& a, const WorkList& w, int num_sms, unsigne
   p.err = a.err;
   p.item_ctr = ctr;
   p.wait_limit_ns = a.wait_limit_ns;
+  p.stall_test = a.stall_test ? 1 : 0;
   static std::mutex attr_mu;
   static bool attr_done[64] = {};
   int dev = 0;

@@ -138,5 +138,6 @@ extern "C" int jvp_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   a.err = err;
   a.item_ctr = counter;
   a.wait_limit_ns = wait_limit_ns();
+  a.stall_test = stall_test();
   return launch_sm100(a, w, sms);
 }

@@ -116,6 +116,7 @@ struct Params {
   unsigned* err;
   unsigned* item_ctr;  // zero at launch; CTAs take work items from it in list order
   unsigned long long wait_limit_ns;
+  int stall_test;  // the MMA warp first waits on a phase that nothing completes
 };
 
 using pipe::wait_bar;
@@ -123,7 +124,6 @@ using pipe::drain_wait;
 using pipe::ItemRing;
 using pipe::Role;
 using pipe::kProducer;
-using pipe::kConsumerThread;
 using pipe::kConsumerWarp;
 using pipe::kRing;
 using pipe::kRingReaders;
@@ -338,6 +338,10 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       Cursor cs, cp;
       cs.start(p, ring, kConsumerWarp);
       cp.start(p, ring, kConsumerWarp);
+      // Failure-detection test: wait on the drain barrier's first phase,
+      // which nothing completes before this warp's own drain commit, so the
+      // bounded wait runs out and the abort path below is taken.
+      if (p.stall_test) ok = __all_sync(0xffffffffu, wait_bar(bar(B_DRAIN), 0u, p, abort_flag));
       for (int pre = 0; pre < 2 && cs.valid && ok; ++pre) {
         ok = wait_s(cs);
         if (!ok) break;
@@ -378,7 +382,7 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           ok = wait_pv(cp);
         }
       }
-      if (!ok || *abort_flag) {
+      if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
         // Wait for every MMA this warp issued before TMEM is freed.
         mma_commit_elect(bar(B_DRAIN));
         drain_wait(bar(B_DRAIN), 0);
@@ -649,6 +653,7 @@ int launch_sm100(const LaunchArgs& a, const WorkList& w, int num_sms) {
   p.err = a.err;
   p.item_ctr = a.item_ctr;
   p.wait_limit_ns = a.wait_limit_ns;
+  p.stall_test = a.stall_test ? 1 : 0;
   // The dynamic shared-memory opt-in is a per-device function attribute.
   static std::mutex attr_mu;
   static bool attr_done[64] = {};

@@ -356,6 +356,19 @@ int jvp_attn_check_device_error(void* stream);
  */
 int jvp_attn_set_wait_limit(uint64_t ns);
 
+/*
+ * jvp_attn_set_stall_test: failure-detection test switch. While enabled
+ * (enable != 0), the MMA warp of every tensor-core kernel launched
+ * (attention JVP, both backward passes, cache attention) first waits on a
+ * barrier phase that nothing completes, so the wait runs out after the limit
+ * set by jvp_attn_set_wait_limit and the launch ends through its timeout
+ * path: JVP_ERR_DEVICE_TIMEOUT in the device error word, outputs undefined,
+ * context usable. No memory is touched out of bounds and nothing traps.
+ * Process-wide; applies to launches made after the call; 0 turns it off.
+ * Always returns JVP_OK.
+ */
+int jvp_attn_set_stall_test(int enable);
+
 /* Frees every cached workspace on every device. Synchronises the device(s)
  * first. Safe to call at any time outside stream capture. */
 int jvp_attn_release(void);
