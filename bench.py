@@ -61,10 +61,17 @@ METRIC_BWD = ("masked attention backward TFLOP/s (10*d per unmasked pair) and % 
 UNIT = "TFLOP/s"
 NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
-KERNEL_SOURCES = ["attention_jvp_continuous_b200/csrc/jvp_attn_sm100.cu",
-                  "attention_jvp_continuous_b200/csrc/sm100_pipeline.cuh",
-                  "attention_jvp_continuous_b200/csrc/sm100_ptx.cuh",
-                  "attention_jvp_continuous_b200/csrc/mask_rows.cuh"]
+_CSRC = "attention_jvp_continuous_b200/csrc/"
+# Sources of each op's kernels: a stored DRAM-traffic figure is used only
+# while these files are unchanged since its capture.
+KERNEL_SOURCES = {
+    "jvp": [_CSRC + f for f in ("jvp_attn_sm100.cu", "sm100_pipeline.cuh", "sm100_ptx.cuh",
+                                "mask_rows.cuh")],
+    "bwd": [_CSRC + f for f in ("jvp_attn_bwd_sm100.cu", "sm100_pipeline.cuh", "sm100_ptx.cuh",
+                                "mask_rows.cuh")],
+    "cache": [_CSRC + f for f in ("attn_cache_sm100.cu", "sm100_pipeline.cuh", "sm100_ptx.cuh")],
+    "prologue": [_CSRC + "qkv_prologue.cu"],
+}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -79,23 +86,26 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_hash() -> str:
+def kernel_hash(op: str = "jvp") -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[op]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def stored_traffic(workload: str):
-    """DRAM bytes per launch from a committed ncu capture, if it was taken
-    on the current kernel source; else None."""
+def stored_traffic(key: str, op: str = "jvp", **shape):
+    """DRAM bytes per launch (per call, for ops of several kernels) from a
+    committed ncu capture, if it was taken on the current kernel source and
+    the entry's recorded shape (e.g. H) matches; else None."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
         d = json.load(f)
-    e = d.get(workload)
-    if not e or e.get("kernel_hash") != kernel_hash():
+    e = d.get(key)
+    if not e or e.get("kernel_hash") != kernel_hash(op):
+        return None
+    if any(k in e and e[k] != v for k, v in shape.items()):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -380,7 +390,8 @@ def run_ours(args, w):
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
     achieved = flops / (launch_ms * 1e-3) / 1e12
-    traffic = None if bwd else stored_traffic(w.name)
+    traffic = (stored_traffic(w.name + "_bwd", "bwd", H=w.H) if bwd
+               else stored_traffic(w.name, H=w.H))
     kernel = ("bwd_kernel<false> + bwd_kernel<true> (query pass, key/value pass)" if bwd
               else "jvp_attn_sm100_kernel")
     line = {
@@ -622,7 +633,8 @@ def run_ours_prologue(args, w):
         "gpu_launches": args.steps,
         "roofline": {
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "traffic": None,
+            "frac": round(achieved / peak, 4),
+            "traffic": stored_traffic(w.name + "_prologue", "prologue", H=H, L=L),
             "peak_source": f"{peak_src} HBM copy bandwidth",
             "kernel": "qkv_prologue_kernel", "launch_ms": round(launch_ms, 4),
         },
