@@ -22,13 +22,15 @@
 //   warps 4..11  softmax/JVP state, P write-back to TMEM, epilogue: two
 //                warpgroups, each taking 32 of a tile's 64 key columns of
 //                every row (one row per thread), exchanging row maxima
-// MMAs per 64-key tile: [S | Q dK^T] = Q [K ; dK]^T (N = 128), then
-// dS += dQ K^T (N = 64), then [A1 | A23] += P [V | dV] (N = 256, P from
-// TMEM), then A23 += (scale e dS) V (N = 128).
+// MMAs per 64-key tile: [S | Q dK^T] = Q [K ; dK]^T (N = 128), committed on
+// its own so the softmax can start on S, then dS += dQ K^T (N = 64), then
+// [A1 | A23] += P [V | dV] (N = 256, P from TMEM), then
+// A23 += (scale e dS) V (N = 128).
 // TMEM (512 columns): S/dS double buffer at [0,256): buffer b holds S in
-// columns [128b, 128b+64) and dS in [128b+64, 128b+128); the bf16 operands
-// e and scale*e*dS overwrite the first 32 columns of S and dS of their
-// buffer. A1 at [256,384), A23 at [384,512). MMA order per CTA is
+// columns [128b, 128b+64) and dS in [128b+64, 128b+128); each softmax half
+// writes its bf16 operands e and scale*e*dS over the first 16 of the 32 S
+// and dS columns it read (columns {0-15, 32-47} of S and of dS). A1 at
+// [256,384), A23 at [384,512). MMA order per CTA is
 // S(0) S(1) PV(0) S(2) PV(1) S(3) ..., so the softmax of tile t overlaps
 // PV(t-1) and S(t+1) on the tensor pipe.
 //
@@ -78,7 +80,7 @@ enum : uint32_t {
   B_KFULL = 2,    // 2 slots (S(t) complete releases K stage t&1: B_SFULL)
   B_VFULL = 4,    // 2
   B_PVD = 6,      // 2: PV(t) of buffer t&1 complete; also releases V stage t&1
-  B_SFULL = 8,    // 2
+  B_SFULL = 8,    // 2: S(t) complete, dS included; also releases K stage t&1
   B_PFULL = 10,   // 2
   B_AFREE = 12,
   B_DRAIN = 13,
@@ -86,7 +88,8 @@ enum : uint32_t {
   B_XSUM = 22,    // 4 slots: [lane quarter], end-of-item l/g exchange
   B_IFULL = 26,   // 4 slots: work-item ring, published
   B_IEMPTY = 30,  // 4 slots: work-item ring, released
-  kNumBars = 34
+  B_SAFULL = 34,  // 2: S and Q dK^T of buffer t&1 complete (dQ K^T may still run)
+  kNumBars = 36
 };
 constexpr uint32_t SM_TMEM_SLOT = SM_BAR + 8 * kNumBars;  // u32: TMEM base
 constexpr uint32_t SM_ABORT = SM_TMEM_SLOT + 4;           // u32: abort flag
@@ -156,6 +159,7 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar(B_VFULL + s), 1);
       mbar_init(bar(B_PVD + s), 1);
       mbar_init(bar(B_SFULL + s), 1);
+      mbar_init(bar(B_SAFULL + s), 1);
       mbar_init(bar(B_PFULL + s), 2 * BM);
     }
     mbar_init(bar(B_AFREE), 2 * BM);
@@ -321,16 +325,16 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t first = c.j == 0 ? 0u : 1u;
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts_elect(tmem + TM_A1, tmem + b * 128u + ks * 8, vb + ((ks * 2048) >> 4), IDESC_PVV,
-                 first | (ks > 0));
+          mma_ts_elect(tmem + TM_A1, tmem + b * 128u + (ks >> 1) * 32u + (ks & 1) * 8u,
+                       vb + ((ks * 2048) >> 4), IDESC_PVV, first | (ks > 0));
       };
       // A23 += (scale e dS) V
       auto issue_pv_b = [&](uint32_t b) {
         const uint64_t vb = v_desc + b * (kStageBytes >> 4);
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts_elect(tmem + TM_A23, tmem + b * 128u + 64u + ks * 8, vb + ((ks * 2048) >> 4),
-                 IDESC_PV, 1u);
+          mma_ts_elect(tmem + TM_A23, tmem + b * 128u + 64u + (ks >> 1) * 32u + (ks & 1) * 8u,
+                       vb + ((ks * 2048) >> 4), IDESC_PV, 1u);
       };
       // Order S(0) S(1) PV(0) S(2) PV(1) ...: S(t+2) overwrites the buffer
       // whose P PV(t) reads, and the MMAs of one issuing lane run in issue
@@ -349,6 +353,7 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t b = cs.t & 1u;
         const bool last = cs.j == cs.n - 1;
         issue_s_a(cs);
+        mma_commit_elect(bar(B_SAFULL + b));  // S ready: the softmax starts on it
         issue_s_b(b);
         mma_commit_elect(bar(B_SFULL + b));  // also releases K stage b to the producer
         if (last) mma_commit_elect(bar(B_QEMPTY));
@@ -371,6 +376,7 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           const uint32_t bs = cs.t & 1u;
           const bool last = cs.j == cs.n - 1;
           issue_s_a(cs);
+          mma_commit_elect(bar(B_SAFULL + bs));  // S ready: the softmax starts on it
           // while S(t+2)'s first half runs: the cursor step and the waits
           // for PV(t+1)
           cs.next(p, ring, kConsumerWarp);
@@ -418,12 +424,13 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         g = 0.f;
       }
       const uint32_t b = c.t & 1u;
-      ok = wait_bar(bar(B_SFULL + b), (c.t >> 1) & 1u, p, abort_flag);
+      // S lands first (its own commit); dS = Q dK^T + dQ K^T completes while
+      // the row max is taken and exchanged.
+      ok = wait_bar(bar(B_SAFULL + b), (c.t >> 1) & 1u, p, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       uint32_t sr[32], dr[32];
       tmem_ld32(tl + b * 128u + 32u * hw, sr);
-      tmem_ld32(tl + b * 128u + 64u + 32u * hw, dr);
       tmem_wait_ld();
       float s[32];
 #pragma unroll
@@ -446,14 +453,16 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int i = 0; i < w2; ++i) m8[i] = fmaxf(m8[i], m8[i + w2]);
       const uint32_t xp = b * 2u;  // exchange slot parity = tile parity
       xmax[(xp + hw) * BM + r] = m8[0];
-      // The exchange also orders TMEM: the partner overwrites half of the S
-      // and dS columns this warp has just read (its P operands), so both
-      // sides fence around it.
-      tc_fence_before();
+      // Each half writes its P and scale e dS back over the S and dS
+      // columns it read itself, so the exchange orders no TMEM accesses.
       mbar_arrive(bar(B_XMAX + q4 * 2 + b));
-      ok = wait_bar(bar(B_XMAX + q4 * 2 + b), (c.t >> 1) & 1u, p, abort_flag);
+      ok = wait_bar(bar(B_SFULL + b), (c.t >> 1) & 1u, p, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
+      tmem_ld32(tl + b * 128u + 64u + 32u * hw, dr);  // in flight across the exchange
+      ok = wait_bar(bar(B_XMAX + q4 * 2 + b), (c.t >> 1) & 1u, p, abort_flag);
+      tmem_wait_ld();
+      if (!__all_sync(0xffffffffu, ok)) break;
       const float mxs = fmaxf(m8[0], xmax[(xp + (hw ^ 1)) * BM + r]) * p.c2;
       float alpha = 1.f;
       bool need = false;
@@ -521,9 +530,11 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         f2unpack(add2(ga, gb), u0, u1);
         g += u0 + u1;
       }
-      // bf16 e into S columns [16 hw, 16 hw + 16), scale*e*dS into the dS ones.
-      tmem_st16(tl + b * 128u + 16u * hw, pp);
-      tmem_st16(tl + b * 128u + 64u + 16u * hw, pd);
+      // bf16 e into S columns [32 hw, 32 hw + 16), scale*e*dS into the dS
+      // ones: a 16-key MMA step takes its A operand from columns
+      // {0, 8, 32, 40} (+64 for scale e dS).
+      tmem_st16(tl + b * 128u + 32u * hw, pp);
+      tmem_st16(tl + b * 128u + 64u + 32u * hw, pd);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_PFULL + b));
