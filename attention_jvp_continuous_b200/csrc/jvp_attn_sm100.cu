@@ -17,20 +17,18 @@
 //
 // Warp roles (384 threads, one CTA per SM, persistent over the work list):
 //   warp 0       TMA producer: Q/dQ per query tile, K|dK and V|dV rings of 2
-//   warp 1       TMEM owner and MMA issuer (the whole warp runs the loop;
-//                one elected lane issues)
+//   warp 1       TMEM owner; issues S(t) (whole warp, one elected lane)
+//   warp 2       issues PV(t) (whole warp, one elected lane)
 //   warps 4..11  softmax/JVP state, P write-back to TMEM, epilogue: two
 //                warpgroups, each taking 32 of a tile's 64 key columns of
 //                every row (one row per thread), exchanging row maxima
-// MMAs per 64-key tile: [S | Q dK^T] = Q [K ; dK]^T (N = 128), committed on
-// its own so the softmax can start on S, then dS += dQ K^T (N = 64), then
-// [A1 | A23] += P [V | dV] (N = 256, P from TMEM), then
-// A23 += (scale e dS) V (N = 128).
+// MMAs per 64-key tile: [S | Q dK^T] = Q [K ; dK]^T (N = 128), then
+// dS += dQ K^T (N = 64), then [A1 | A23] += P [V | dV] (N = 256, P from
+// TMEM), then A23 += (scale e dS) V (N = 128).
 // TMEM (512 columns): S/dS double buffer at [0,256): buffer b holds S in
-// columns [128b, 128b+64) and dS in [128b+64, 128b+128); each softmax half
-// writes its bf16 operands e and scale*e*dS over the first 16 of the 32 S
-// and dS columns it read (columns {0-15, 32-47} of S and of dS). A1 at
-// [256,384), A23 at [384,512). MMA order per CTA is
+// columns [128b, 128b+64) and dS in [128b+64, 128b+128); the bf16 operands
+// e and scale*e*dS overwrite the first 32 columns of S and dS of their
+// buffer. A1 at [256,384), A23 at [384,512). MMA order per CTA is
 // S(0) S(1) PV(0) S(2) PV(1) S(3) ..., so the softmax of tile t overlaps
 // PV(t-1) and S(t+1) on the tensor pipe.
 //
@@ -80,7 +78,7 @@ enum : uint32_t {
   B_KFULL = 2,    // 2 slots (S(t) complete releases K stage t&1: B_SFULL)
   B_VFULL = 4,    // 2
   B_PVD = 6,      // 2: PV(t) of buffer t&1 complete; also releases V stage t&1
-  B_SFULL = 8,    // 2: S(t) complete, dS included; also releases K stage t&1
+  B_SFULL = 8,    // 2
   B_PFULL = 10,   // 2
   B_AFREE = 12,
   B_DRAIN = 13,
@@ -88,8 +86,10 @@ enum : uint32_t {
   B_XSUM = 22,    // 4 slots: [lane quarter], end-of-item l/g exchange
   B_IFULL = 26,   // 4 slots: work-item ring, published
   B_IEMPTY = 30,  // 4 slots: work-item ring, released
-  B_SAFULL = 34,  // 2: S and Q dK^T of buffer t&1 complete (dQ K^T may still run)
-  kNumBars = 36
+  B_DRAIN2 = 34,  // drain barrier of the second MMA warp
+  B_SAFULL = 35,  // 2: S and Q dK^T of buffer t&1 complete (dQ K^T may still run)
+  B_PVI = 37,     // 2: PV(t) of buffer t&1 issued (not complete)
+  kNumBars = 39
 };
 constexpr uint32_t SM_TMEM_SLOT = SM_BAR + 8 * kNumBars;  // u32: TMEM base
 constexpr uint32_t SM_ABORT = SM_TMEM_SLOT + 4;           // u32: abort flag
@@ -160,10 +160,12 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar(B_PVD + s), 1);
       mbar_init(bar(B_SFULL + s), 1);
       mbar_init(bar(B_SAFULL + s), 1);
+      mbar_init(bar(B_PVI + s), 1);
       mbar_init(bar(B_PFULL + s), 2 * BM);
     }
     mbar_init(bar(B_AFREE), 2 * BM);
     mbar_init(bar(B_DRAIN), 1);
+    mbar_init(bar(B_DRAIN2), 1);
     for (int i = 0; i < 8; ++i) mbar_init(bar(B_XMAX + i), 64);
     for (int i = 0; i < 4; ++i) mbar_init(bar(B_XSUM + i), 64);
     for (int i = 0; i < int(kRing); ++i) {
@@ -251,13 +253,19 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA ----
-    // The whole warp runs the issue loop (uniform control flow keeps the
-    // descriptors in the uniform datapath); one elected lane issues each MMA
-    // and commit. This issues faster than a lone lane 0 when the softmax
-    // warps share the scheduler.
+  } else if (warp == 1 || warp == 2) {
+    // ----------------------------------------------------------- MMA ----
+    // Issue is split over two warps: warp 1 issues S(t) (Q [K ; dK]^T and
+    // dQ K^T), warp 2 PV(t) ([A1 | A23] += P [V | dV], A23 += Pds V). Each
+    // runs its loop as a whole warp in uniform control flow and one elected
+    // lane issues its MMAs and commits. S(t) overwrites the TMEM buffer whose
+    // P PV(t-2) reads, so warp 1 issues it only after warp 2 has issued
+    // PV(t-2) (an mbarrier arrive behind tcgen05.fence::before_thread_sync,
+    // and tcgen05.fence::after_thread_sync on the waiting side): the CTA's
+    // MMAs run in the order they enter the tensor pipe. Otherwise the two
+    // streams are independent.
     {
+      const bool s_warp = warp == 1;
       bool ok = true;
       // Descriptors of the fixed shared-memory operands; an MMA's operand
       // is the base plus a compile-time byte offset >> 4 (the start-address
@@ -266,132 +274,94 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint64_t dq_desc = sdesc_sw128(base + SM_DQ, 16, 1024);
       const uint64_t k_desc = sdesc_sw128(base + SM_K, 16, 1024);       // stage 0
       const uint64_t v_desc = sdesc_sw128(base + SM_V, kKHalf, 1024);   // stage 0
-      // The tensor pipe takes a tile's 24 MMAs back to back in ~1.65k cycles,
-      // but holds only a few queued MMAs: scalar work done between batches
-      // (barrier checks, commits, cursor steps) lets it run dry. So each
-      // batch is issued in two halves, and the waits for the next batch and
-      // the cursor step go between them, while the first half executes.
-      // Each wait first tests all of its barriers back to back (one latency
-      // instead of one per barrier; they are normally complete already) and
-      // falls back to the bounded waits one by one.
-      auto wait_s = [&](const Cursor& c) -> bool {  // S(t): Q (new item), K|dK stage
-        const uint32_t bk = bar(B_KFULL + (c.t & 1u)), pk = (c.t >> 1) & 1u;
-        const bool need_q = c.j == 0;
-        const bool rk = mbar_test(bk, pk);
-        const bool rq = !need_q || mbar_test(bar(B_QFULL), c.item_idx & 1);
-        if (__all_sync(0xffffffffu, rk && rq)) return true;
-        bool w = !need_q || wait_bar(bar(B_QFULL), c.item_idx & 1, p, abort_flag);
-        w = w && wait_bar(bk, pk, p, abort_flag);
-        return __all_sync(0xffffffffu, w);
-      };
-      auto wait_pv = [&](const Cursor& c) -> bool {  // PV(t): accumulators, P, V|dV stage
-        const uint32_t b = c.t & 1u, par = (c.t >> 1) & 1u;
-        const bool need_a = c.j == 0 && c.item_idx > 0;
-        const bool rp = mbar_test(bar(B_PFULL + b), par);
-        const bool rv = mbar_test(bar(B_VFULL + b), par);
-        const bool ra = !need_a || mbar_test(bar(B_AFREE), (c.item_idx - 1) & 1);
-        if (__all_sync(0xffffffffu, rp && rv && ra)) return true;
-        bool w = !need_a || wait_bar(bar(B_AFREE), (c.item_idx - 1) & 1, p, abort_flag);
-        w = w && wait_bar(bar(B_PFULL + b), par, p, abort_flag);
-        w = w && wait_bar(bar(B_VFULL + b), par, p, abort_flag);
-        return __all_sync(0xffffffffu, w);
-      };
-      // [S | Q dK^T] = Q [K ; dK]^T: one N=128 MMA per 16-wide k-step.
-      auto issue_s_a = [&](const Cursor& c) {
-        const uint32_t b = c.t & 1u;
-        const uint64_t kb = k_desc + b * (kStageBytes >> 4);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t oq = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
-          const uint32_t ob = ((kk >> 2) * (2 * kKHalf) + (kk & 3) * 32) >> 4;
-          mma_ss_elect(tmem + b * 128u, q_desc + oq, kb + ob, IDESC_SK, kk > 0);
-        }
-      };
-      // dS = Q dK^T + dQ K^T: N=64 MMAs accumulate dQ K^T onto it.
-      auto issue_s_b = [&](uint32_t b) {
-        const uint64_t kb = k_desc + b * (kStageBytes >> 4);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t oq = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
-          const uint32_t ob = ((kk >> 2) * (2 * kKHalf) + (kk & 3) * 32) >> 4;
-          mma_ss_elect(tmem + b * 128u + 64u, dq_desc + oq, kb + ob, IDESC_S, 1u);
-        }
-      };
-      // [A1 | A23] += P [V | dV]: one N=256 MMA per 16-key step (A1 and A23
-      // are adjacent in TMEM; V h0, V h1, dV h0, dV h1 are 8 KB apart).
-      auto issue_pv_a = [&](const Cursor& c) {
-        const uint32_t b = c.t & 1u;
-        const uint64_t vb = v_desc + b * (kStageBytes >> 4);
-        const uint32_t first = c.j == 0 ? 0u : 1u;
-#pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts_elect(tmem + TM_A1, tmem + b * 128u + (ks >> 1) * 32u + (ks & 1) * 8u,
-                       vb + ((ks * 2048) >> 4), IDESC_PVV, first | (ks > 0));
-      };
-      // A23 += (scale e dS) V
-      auto issue_pv_b = [&](uint32_t b) {
-        const uint64_t vb = v_desc + b * (kStageBytes >> 4);
-#pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts_elect(tmem + TM_A23, tmem + b * 128u + 64u + (ks >> 1) * 32u + (ks & 1) * 8u,
-                       vb + ((ks * 2048) >> 4), IDESC_PV, 1u);
-      };
-      // Order S(0) S(1) PV(0) S(2) PV(1) ...: S(t+2) overwrites the buffer
-      // whose P PV(t) reads, and the MMAs of one issuing lane run in issue
-      // order (elect.sync picks the same lane while the warp is converged).
-      Cursor cs, cp;
-      cs.start(p, ring, kConsumerWarp);
-      cp.start(p, ring, kConsumerWarp);
+      Cursor c;
+      c.start(p, ring, kConsumerWarp);
       // Failure-detection test: wait on the drain barrier's first phase,
       // which nothing completes before this warp's own drain commit, so the
       // bounded wait runs out and the abort path below is taken.
-      if (p.stall_test) ok = __all_sync(0xffffffffu, wait_bar(bar(B_DRAIN), 0u, p, abort_flag));
-      for (int pre = 0; pre < 2 && cs.valid && ok; ++pre) {
-        ok = wait_s(cs);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t b = cs.t & 1u;
-        const bool last = cs.j == cs.n - 1;
-        issue_s_a(cs);
-        mma_commit_elect(bar(B_SAFULL + b));  // S ready: the softmax starts on it
-        issue_s_b(b);
-        mma_commit_elect(bar(B_SFULL + b));  // also releases K stage b to the producer
-        if (last) mma_commit_elect(bar(B_QEMPTY));
-        cs.next(p, ring, kConsumerWarp);
-      }
-      if (ok && cp.valid) ok = wait_pv(cp);
-      while (ok && cp.valid) {
-        tc_fence_after();
-        const uint32_t bp = cp.t & 1u;
-        issue_pv_a(cp);
-        // while PV(t)'s first half runs: the waits for S(t+2)
-        const bool have_s = cs.valid;
-        if (have_s) ok = wait_s(cs);
-        tc_fence_after();
-        issue_pv_b(bp);
-        mma_commit_elect(bar(B_PVD + bp));  // PV(t) done: V stage free, A1/A23 current
-        cp.next(p, ring, kConsumerWarp);
-        if (!ok) break;
-        if (have_s) {
-          const uint32_t bs = cs.t & 1u;
-          const bool last = cs.j == cs.n - 1;
-          issue_s_a(cs);
-          mma_commit_elect(bar(B_SAFULL + bs));  // S ready: the softmax starts on it
-          // while S(t+2)'s first half runs: the cursor step and the waits
-          // for PV(t+1)
-          cs.next(p, ring, kConsumerWarp);
-          if (cp.valid) ok = wait_pv(cp);
-          issue_s_b(bs);
-          mma_commit_elect(bar(B_SFULL + bs));
+      if (p.stall_test && s_warp)
+        ok = __all_sync(0xffffffffu, wait_bar(bar(B_DRAIN), 0u, p, abort_flag));
+      if (s_warp) {
+        while (ok && c.valid) {
+          const uint32_t b = c.t & 1u, par = (c.t >> 1) & 1u;
+          const bool need_q = c.j == 0, need_pv = c.t >= 2;
+          // All of the tile's barriers are tested back to back (they are
+          // normally complete already), then waited for one by one.
+          bool r = mbar_test(bar(B_KFULL + b), par);
+          r = r && (!need_q || mbar_test(bar(B_QFULL), c.item_idx & 1));
+          r = r && (!need_pv || mbar_test(bar(B_PVI + b), par ^ 1u));
+          if (!__all_sync(0xffffffffu, r)) {
+            bool w = !need_pv || wait_bar(bar(B_PVI + b), par ^ 1u, p, abort_flag);
+            w = w && (!need_q || wait_bar(bar(B_QFULL), c.item_idx & 1, p, abort_flag));
+            w = w && wait_bar(bar(B_KFULL + b), par, p, abort_flag);
+            ok = __all_sync(0xffffffffu, w);
+            if (!ok) break;
+          }
+          tc_fence_after();
+          const bool last = c.j == c.n - 1;
+          const uint64_t kb = k_desc + b * (kStageBytes >> 4);
+          // [S | Q dK^T] = Q [K ; dK]^T: one N=128 MMA per 16-wide k-step.
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t oq = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
+            const uint32_t ob = ((kk >> 2) * (2 * kKHalf) + (kk & 3) * 32) >> 4;
+            mma_ss_elect(tmem + b * 128u, q_desc + oq, kb + ob, IDESC_SK, kk > 0);
+          }
+          mma_commit_elect(bar(B_SAFULL + b));  // S ready: the softmax starts on it
+          // dS = Q dK^T + dQ K^T: N=64 MMAs accumulate dQ K^T onto it.
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t oq = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
+            const uint32_t ob = ((kk >> 2) * (2 * kKHalf) + (kk & 3) * 32) >> 4;
+            mma_ss_elect(tmem + b * 128u + 64u, dq_desc + oq, kb + ob, IDESC_S, 1u);
+          }
+          mma_commit_elect(bar(B_SFULL + b));  // also releases K stage b to the producer
           if (last) mma_commit_elect(bar(B_QEMPTY));
-        } else if (cp.valid) {
-          ok = wait_pv(cp);
+          c.next(p, ring, kConsumerWarp);
+        }
+      } else {
+        while (ok && c.valid) {
+          const uint32_t b = c.t & 1u, par = (c.t >> 1) & 1u;
+          const bool need_a = c.j == 0 && c.item_idx > 0;
+          const uint32_t pa = (c.item_idx - 1) & 1;
+          bool r = mbar_test(bar(B_PFULL + b), par);
+          r = r && mbar_test(bar(B_VFULL + b), par);
+          r = r && (!need_a || mbar_test(bar(B_AFREE), pa));
+          if (!__all_sync(0xffffffffu, r)) {
+            bool w = !need_a || wait_bar(bar(B_AFREE), pa, p, abort_flag);
+            w = w && wait_bar(bar(B_PFULL + b), par, p, abort_flag);
+            w = w && wait_bar(bar(B_VFULL + b), par, p, abort_flag);
+            ok = __all_sync(0xffffffffu, w);
+            if (!ok) break;
+          }
+          tc_fence_after();
+          const uint64_t vb = v_desc + b * (kStageBytes >> 4);
+          const uint32_t first = c.j == 0 ? 0u : 1u;
+          // [A1 | A23] += P [V | dV]: one N=256 MMA per 16-key step (A1 and
+          // A23 are adjacent in TMEM; V h0, V h1, dV h0, dV h1 are 8 KB apart).
+#pragma unroll
+          for (int ks = 0; ks < BN / 16; ++ks)
+            mma_ts_elect(tmem + TM_A1, tmem + b * 128u + (ks >> 1) * 32u + (ks & 1) * 8u,
+                         vb + ((ks * 2048) >> 4), IDESC_PVV, first | (ks > 0));
+          // A23 += (scale e dS) V
+#pragma unroll
+          for (int ks = 0; ks < BN / 16; ++ks)
+            mma_ts_elect(tmem + TM_A23, tmem + b * 128u + 64u + (ks >> 1) * 32u + (ks & 1) * 8u,
+                         vb + ((ks * 2048) >> 4), IDESC_PV, 1u);
+          mma_commit_elect(bar(B_PVD + b));  // PV(t) done: V stage free, A1/A23 current
+          // PV(t) is in the tensor pipe's queue: S(t+2) may follow it (the
+          // pipe runs the CTA's MMAs in the order they enter the queue).
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(B_PVI + b));
+          c.next(p, ring, kConsumerWarp);
         }
       }
       if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
         // Wait for every MMA this warp issued before TMEM is freed.
-        mma_commit_elect(bar(B_DRAIN));
-        drain_wait(bar(B_DRAIN), 0);
+        const uint32_t db = bar(s_warp ? B_DRAIN : B_DRAIN2);
+        mma_commit_elect(db);
+        drain_wait(db, 0);
       }
     }
     __syncwarp();
