@@ -69,7 +69,7 @@ struct Layout {
   static constexpr uint32_t X = kKV ? 4 * kRHalf : 0;
   static constexpr uint32_t Y = X + NX * kTile;
   static constexpr uint32_t BAR = Y + NY * kTile;  // 144 KB (dQ) / 224 KB (dK/dV)
-  static constexpr uint32_t TMEM_SLOT = BAR + 8 * 40;
+  static constexpr uint32_t TMEM_SLOT = BAR + 8 * 44;
   static constexpr uint32_t ABORT = TMEM_SLOT + 4;
   static constexpr uint32_t RING = ABORT + 4;
   static constexpr uint32_t kBytes = BAR + 512 + 1024;  // + alignment slack
@@ -90,9 +90,10 @@ enum : uint32_t {
   B_DRAIN = 29,  // 2: one per issuer
   B_IF = 31,     // 4: work-item ring
   B_IE = 35,     // 4
-  kNumBars = 39
+  B_AI = 39,     // 2: accumulating MMAs of the buffer's last tile issued
+  kNumBars = 41
 };
-static_assert(kNumBars <= 40, "barrier slots");
+static_assert(kNumBars <= 44, "barrier slots");
 static_assert(Layout<false>::RING + 16 <= Layout<false>::BAR + 512, "barrier area overflow");
 
 // TMEM columns: S/dP double buffer [0, 256) (buffer b at 128 b: S or S^T at
@@ -172,6 +173,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       mbar_init(bar(B_SF + b), 2);
       mbar_init(bar(B_PF + b), 2 * BR);
       mbar_init(bar(B_MD + b), 1);
+      mbar_init(bar(B_AI + b), 1);
       mbar_init(bar(B_DRAIN + b), 1);
     }
     mbar_init(bar(B_CF), 2 * BR);
@@ -274,8 +276,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         uint32_t stage;
         uint64_t bdesc;
         if (s_mma) {
-          // Buffer b last held tile t-2, whose operands acc(t-2) reads.
-          if (c.t >= 2 && !wait_w(bar(B_MD + b), ((c.t >> 1) - 1) & 1u))
+          // Buffer b last held tile t-2, whose operands acc(t-2) reads: S(t)
+          // is issued once acc(t-2) has entered the tensor pipe (issuer B
+          // arrives behind tcgen05.fence::before_thread_sync; the
+          // tc_fence_after below completes the pair), and the pipe runs the
+          // CTA's MMAs in the order they enter it.
+          if (c.t >= 2 && !wait_w(bar(B_AI + b), ((c.t >> 1) - 1) & 1u))
             return false;
           stage = c.t % NX;
           if (!wait_w(bar(B_XF + stage), (c.t / NX) & 1u)) return false;
@@ -335,6 +341,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         mma_commit_elect(bar(B_XE + sx));
         if (kKV) mma_commit_elect(bar(B_YE + sy));
         mma_commit_elect(bar(B_MD + b));
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_AI + b));  // acc(t) issued: S(t+2) may follow
         return true;
       };
       bool ok = true;
@@ -516,7 +525,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
 
       if (c.j == c.n - 1) {
         // ------------------------------------------------------ epilogue --
-        // acc(t-2) on the same barrier has completed: S(t) waited for it.
+        // acc(t-2), the previous phase of this barrier, has completed:
+        // issuer B issued it before dP(t), whose S-ready commit (covering
+        // all of issuer B's earlier MMAs) this warp has seen land.
         ok = wait_bar(bar(B_MD + (c.t & 1u)), (c.t >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();

@@ -231,6 +231,9 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         tma_load_3d(ks + kKHalf, &tm_dk, bar(B_KFULL + s), 0, y, c.bh);
         tma_load_3d(ks + 2 * kKHalf, &tm_k, bar(B_KFULL + s), 64, y, c.bh);
         tma_load_3d(ks + 3 * kKHalf, &tm_dk, bar(B_KFULL + s), 64, y, c.bh);
+        // V stage s is free once PV(t - 2) is done. PV(t - 4), the previous
+        // phase of that barrier, ran on the tensor pipe before S(t - 2),
+        // which was waited for just above, so the parity wait is unambiguous.
         if (c.t >= 2) ok = wait_bar(bar(B_PVD + s), (u - 1) & 1u, p, abort_flag);
         if (!ok) break;
         mbar_expect_tx(bar(B_VFULL + s), kStageBytes);
@@ -449,8 +452,9 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         g *= alpha;
         // A1/A23 hold PV(t-1); wait for it, then scale this quarter's rows:
         // the first warpgroup scales A1, the second A23.
-        // (PV(t-3), the previous phase of that barrier, completed before
-        // S(t-1) was issued.)
+        // (PV(t-3), the previous phase of that barrier, entered the tensor
+        // pipe before S(t-1), whose completion this warp has seen, and the
+        // pipe runs the CTA's MMAs in order.)
         ok = wait_bar(bar(B_PVD + ((c.t - 1) & 1u)), ((c.t - 1) >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
@@ -511,8 +515,9 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
       if (c.j == c.n - 1) {
         // ------------------------------------------------------ epilogue --
-        // PV(t) done; PV(t-2), the previous phase of this barrier, completed
-        // before S(t) was issued, so the parity wait is unambiguous.
+        // PV(t) done. PV(t-2), the previous phase of this barrier, entered
+        // the tensor pipe before S(t), whose completion this warp has seen,
+        // so it has completed and the parity wait is unambiguous.
         ok = wait_bar(bar(B_PVD + (c.t & 1u)), (c.t >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         // Row totals of l and g from both halves.
