@@ -8,8 +8,10 @@
 //   warp 0       TMA: Q once per item, K (3 stages) and V (2 stages) of 128
 //                keys; the cache is read through tensor maps whose row
 //                extent is Lk, so rows past the exposed prefix are zero-filled
-//   warp 1       TMEM owner and MMA issuer: S = Q K^T (N = 128) into a
-//                double buffer, O += P V (N = 128, P from TMEM)
+//   warp 1       TMEM owner; issues S = Q K^T (N = 128) into a double
+//                buffer
+//   warp 2       issues O += P V (N = 128, P from TMEM); S(t+2) is issued
+//                only once PV(t) is in the tensor pipe's queue
 //   warps 4-11   softmax: two warpgroups, each 64 of a tile's 128 keys of
 //                every row with its own running max and its own O
 //                accumulator (lazy rescale only when its row max grows by
@@ -76,7 +78,9 @@ enum : uint32_t {
   B_XSUM = 20,    // 4: [lane quarter], end-of-item merge of the halves
   B_IFULL = 24,   // 4
   B_IEMPTY = 28,  // 4
-  kNumBars = 32
+  B_PVI = 32,     // 2: PV MMAs of the buffer's latest tile issued (not complete)
+  B_DRAIN2 = 34,  // drain barrier of the PV-issuing warp
+  kNumBars = 35
 };
 constexpr uint32_t SM_TMEM_SLOT = SM_BAR + 8 * kNumBars;
 constexpr uint32_t SM_ABORT = SM_TMEM_SLOT + 4;
@@ -136,9 +140,11 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar(B_SFULL + s), 1);
       mbar_init(bar(B_PFULL + s), 2 * BM);
       mbar_init(bar(B_PVD + s), 1);
+      mbar_init(bar(B_PVI + s), 1);
     }
     mbar_init(bar(B_AFREE), 2 * BM);
     mbar_init(bar(B_DRAIN), 1);
+    mbar_init(bar(B_DRAIN2), 1);
     for (int i = 0; i < 4; ++i) mbar_init(bar(B_XSUM + i), 64);
     for (uint32_t i = 0; i < kRing; ++i) {
       mbar_init(bar(B_IFULL + i), 1);
@@ -210,9 +216,9 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------------ MMA ----
-    // The whole warp runs the loop in uniform control flow; one elected lane
+    // Each MMA warp runs its loop in uniform control flow; one elected lane
     // issues each MMA and commit.
     {
       bool ok = true;
@@ -225,6 +231,10 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       auto issue_s = [&](const Cursor& c) -> bool {
         const uint32_t b = c.t & 1u, sk = c.t % NK;
         if (c.j == 0 && !wait_w(bar(B_QFULL), c.item_idx & 1)) return false;
+        // Buffer b last held tile t-2, whose P PV(t-2) reads: issue S(t) once
+        // PV(t-2) is in the tensor pipe's queue (the pipe runs the CTA's MMAs
+        // in the order they enter it).
+        if (c.t >= 2 && !wait_w(bar(B_PVI + b), ((c.t >> 1) - 1) & 1u)) return false;
         if (!wait_w(bar(B_KFULL + sk), (c.t / NK) & 1u)) return false;
         tc_fence_after();
         const uint64_t kb = k_desc + sk * (kStage >> 4);
@@ -259,32 +269,28 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                  vb + ((ks * 2048) >> 4), IDESC_PV, first | ((ks & 3) > 0));
         mma_commit_elect(bar(B_VEMPTY + b));
         mma_commit_elect(bar(B_PVD + b));
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_PVI + b));  // PV(t) issued: S(t+2) may follow
         return true;
       };
-      // Order S(0) S(1) PV(0) S(2) PV(1) ...: S(t+2) overwrites the buffer
-      // whose P PV(t) reads, and the MMAs of one issuing lane run in issue order.
-      Cursor cs, cp;
-      cs.start(p, ring, kConsumerWarp);
-      cp.start(p, ring, kConsumerWarp);
+      // Warp 1 issues S(t), warp 2 PV(t); S(t+2) follows PV(t) in the pipe.
+      const bool s_warp = warp == 1;
+      Cursor c;
+      c.start(p, ring, kConsumerWarp);
       // Failure-detection test: wait on the drain barrier's first phase,
       // which nothing completes before this warp's own drain commit, so the
       // bounded wait runs out and the abort path below is taken.
-      if (p.stall_test) ok = __all_sync(0xffffffffu, wait_bar(bar(B_DRAIN), 0u, p, abort_flag));
-      for (int pre = 0; pre < 2 && cs.valid && ok; ++pre) {
-        ok = issue_s(cs);
-        cs.next(p, ring, kConsumerWarp);
-      }
-      while (cp.valid && ok) {
-        ok = issue_pv(cp);
-        cp.next(p, ring, kConsumerWarp);
-        if (ok && cs.valid) {
-          ok = issue_s(cs);
-          cs.next(p, ring, kConsumerWarp);
-        }
+      if (p.stall_test && s_warp)
+        ok = __all_sync(0xffffffffu, wait_bar(bar(B_DRAIN), 0u, p, abort_flag));
+      while (c.valid && ok) {
+        ok = s_warp ? issue_s(c) : issue_pv(c);
+        c.next(p, ring, kConsumerWarp);
       }
       if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
-        mma_commit_elect(bar(B_DRAIN));
-        drain_wait(bar(B_DRAIN), 0);
+        const uint32_t db = bar(s_warp ? B_DRAIN : B_DRAIN2);
+        mma_commit_elect(db);
+        drain_wait(db, 0);
       }
     }
     __syncwarp();
@@ -355,7 +361,8 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (__any_sync(0xffffffffu, need)) {
         l *= alpha;
         // This O holds PV(t-1); wait for it. (PV(t-3), the previous phase of
-        // that barrier, completed before S(t-1) was issued.)
+        // that barrier, entered the tensor pipe before S(t-1), whose
+        // completion this warp has seen.)
         ok = wait_bar(bar(B_PVD + ((c.t - 1) & 1u)), ((c.t - 1) >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
@@ -398,8 +405,8 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
       if (c.j == c.n - 1) {
         // ------------------------------------------------------ epilogue --
-        // PV(t) done; PV(t-2), the previous phase of this barrier, completed
-        // before S(t) was issued.
+        // PV(t) done; PV(t-2), the previous phase of this barrier, entered
+        // the tensor pipe before S(t), whose completion this warp has seen.
         ok = wait_bar(bar(B_PVD + (c.t & 1u)), (c.t >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         xsum[hw * BM + r] = m_ref;
