@@ -89,7 +89,8 @@ enum : uint32_t {
   B_DRAIN2 = 34,  // drain barrier of the second MMA warp
   B_SAFULL = 35,  // 2: S and Q dK^T of buffer t&1 complete (dQ K^T may still run)
   B_PVI = 37,     // 2: PV(t) of buffer t&1 issued (not complete)
-  kNumBars = 39
+  B_PDFULL = 39,  // 2: scale e dS of buffer t&1 written (B_PFULL: e written)
+  kNumBars = 41
 };
 constexpr uint32_t SM_TMEM_SLOT = SM_BAR + 8 * kNumBars;  // u32: TMEM base
 constexpr uint32_t SM_ABORT = SM_TMEM_SLOT + 4;           // u32: abort flag
@@ -162,6 +163,7 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar(B_SAFULL + s), 1);
       mbar_init(bar(B_PVI + s), 1);
       mbar_init(bar(B_PFULL + s), 2 * BM);
+      mbar_init(bar(B_PDFULL + s), 2 * BM);
     }
     mbar_init(bar(B_AFREE), 2 * BM);
     mbar_init(bar(B_DRAIN), 1);
@@ -346,6 +348,13 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int ks = 0; ks < BN / 16; ++ks)
             mma_ts_elect(tmem + TM_A1, tmem + b * 128u + (ks >> 1) * 32u + (ks & 1) * 8u,
                          vb + ((ks * 2048) >> 4), IDESC_PVV, first | (ks > 0));
+          // scale e dS is written after dS lands, once the softmax is done
+          // with the exponentials.
+          if (!__all_sync(0xffffffffu, mbar_test(bar(B_PDFULL + b), par))) {
+            ok = __all_sync(0xffffffffu, wait_bar(bar(B_PDFULL + b), par, p, abort_flag));
+            if (!ok) break;
+          }
+          tc_fence_after();
           // A23 += (scale e dS) V
 #pragma unroll
           for (int ks = 0; ks < BN / 16; ++ks)
@@ -429,12 +438,7 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       // Each half writes its P and scale e dS back over the S and dS
       // columns it read itself, so the exchange orders no TMEM accesses.
       mbar_arrive(bar(B_XMAX + q4 * 2 + b));
-      ok = wait_bar(bar(B_SFULL + b), (c.t >> 1) & 1u, p, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      tmem_ld32(tl + b * 128u + 64u + 32u * hw, dr);  // in flight across the exchange
       ok = wait_bar(bar(B_XMAX + q4 * 2 + b), (c.t >> 1) & 1u, p, abort_flag);
-      tmem_wait_ld();
       if (!__all_sync(0xffffffffu, ok)) break;
       const float mxs = fmaxf(m8[0], xmax[(xp + (hw ^ 1)) * BM + r]) * p.c2;
       float alpha = 1.f;
@@ -471,47 +475,68 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         tmem_wait_st();
       }
       const float mref_use = m_ref == -CUDART_INF_F ? 0.f : m_ref;
-      // Pairs of columns in packed fp32 (f32x2) arithmetic: 2^(c2 s - m),
-      // e dS, the partial sums and scale e dS take one instruction per pair.
+      // First what needs only S: e = 2^(c2 s - m), l and the bf16 e that
+      // P [V | dV] reads; then, once dS has landed (its N = 64 MMAs run
+      // while the exponentials are computed), e dS, g and scale e dS for
+      // A23 += (scale e dS) V. Pairs of columns in packed fp32 (f32x2)
+      // arithmetic take one instruction per pair.
       const uint64_t c2v = f2pack(p.c2, p.c2), mv = f2pack(-mref_use, -mref_use);
-      const uint64_t scv = f2pack(p.scale, p.scale);
-      uint64_t la = 0, lb = 0, ga = 0, gb = 0;  // 0 = two +0.0f
-      uint32_t pp[16], pd[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float x0, x1;
-        f2unpack(fma2(f2pack(s[2 * i], s[2 * i + 1]), c2v, mv), x0, x1);
-        const float e0 = ex2(x0), e1 = ex2(x1);
-        const uint64_t ev = f2pack(e0, e1);
-        const uint64_t edv =
-            mul2(ev, f2pack(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1])));
-        if (i & 1) {
-          lb = add2(lb, ev);
-          gb = add2(gb, edv);
-        } else {
-          la = add2(la, ev);
-          ga = add2(ga, edv);
-        }
-        pp[i] = pack_bf16(e0, e1);
-        float q0, q1;
-        f2unpack(mul2(edv, scv), q0, q1);
-        pd[i] = pack_bf16(q0, q1);
-      }
+      uint64_t ev[16];
       {
+        uint64_t la = 0, lb = 0;  // 0 = two +0.0f
+        uint32_t pp[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float x0, x1;
+          f2unpack(fma2(f2pack(s[2 * i], s[2 * i + 1]), c2v, mv), x0, x1);
+          const float e0 = ex2(x0), e1 = ex2(x1);
+          ev[i] = f2pack(e0, e1);
+          if (i & 1)
+            lb = add2(lb, ev[i]);
+          else
+            la = add2(la, ev[i]);
+          pp[i] = pack_bf16(e0, e1);
+        }
         float u0, u1;
         f2unpack(add2(la, lb), u0, u1);
         l += u0 + u1;
+        // bf16 e into S columns [32 hw, 32 hw + 16): a 16-key MMA step takes
+        // its A operand from columns {0, 8, 32, 40}.
+        tmem_st16(tl + b * 128u + 32u * hw, pp);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_PFULL + b));
+      }
+      ok = wait_bar(bar(B_SFULL + b), (c.t >> 1) & 1u, p, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      tmem_ld32(tl + b * 128u + 64u + 32u * hw, dr);
+      tmem_wait_ld();
+      {
+        const uint64_t scv = f2pack(p.scale, p.scale);
+        uint64_t ga = 0, gb = 0;
+        uint32_t pd[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint64_t edv =
+              mul2(ev[i], f2pack(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1])));
+          if (i & 1)
+            gb = add2(gb, edv);
+          else
+            ga = add2(ga, edv);
+          float q0, q1;
+          f2unpack(mul2(edv, scv), q0, q1);
+          pd[i] = pack_bf16(q0, q1);
+        }
+        float u0, u1;
         f2unpack(add2(ga, gb), u0, u1);
         g += u0 + u1;
+        // scale e dS into dS columns [64 + 32 hw, 64 + 32 hw + 16).
+        tmem_st16(tl + b * 128u + 64u + 32u * hw, pd);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_PDFULL + b));
       }
-      // bf16 e into S columns [32 hw, 32 hw + 16), scale*e*dS into the dS
-      // ones: a 16-key MMA step takes its A operand from columns
-      // {0, 8, 32, 40} (+64 for scale e dS).
-      tmem_st16(tl + b * 128u + 32u * hw, pp);
-      tmem_st16(tl + b * 128u + 64u + 32u * hw, pd);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(B_PFULL + b));
 
       if (c.j == c.n - 1) {
         // ------------------------------------------------------ epilogue --
