@@ -51,8 +51,8 @@ constexpr int kThreads = 384;
 constexpr uint32_t kRHalf = BR * 128;  // 16 KB: 128 rows x 64 head-dim columns
 constexpr uint32_t kTHalf = BT * 128;  //  8 KB: 64 rows x 64 columns
 constexpr uint32_t kTile = 2 * kTHalf; // 16 KB: one streamed 64-row operand
-// Readers of the work-item ring: issuer A, issuer B's two cursors, 8 softmax warps.
-constexpr uint32_t kReaders = 3 + 8;
+// Readers of the work-item ring: issuers A and B, 8 softmax warps.
+constexpr uint32_t kReaders = 2 + 8;
 
 // Shared memory: the dK/dV pass's two stationary operands (A0, A1; the dQ
 // pass keeps its stationary Q and G in TMEM), then the streamed operands in
@@ -130,15 +130,16 @@ struct Params {
 };
 using Cursor = pipe::Cursor<Params>;
 
-// MMA issue is split over two threads, since one thread issues at most about
-// one tcgen05.mma per ~47 cycles while a 128 x 64 x 16 MMA takes 32:
-//   issuer A (warp 1): S(t) = A0 X(t)^T into buffer t&1, once the
-//                      accumulating MMAs of tile t-2 (same buffer) are done;
-//   issuer B (warp 2): dP(t) = A1 Y(t)^T, and acc(t) once the softmax warps
-//                      have written tile t's bf16 operands. B issues dP(t)
-//                      after acc(t-2), so its own order protects the buffer.
-// The pipe executes each thread's MMAs in issue order; every hand-over
-// between the two threads and the other roles goes through an mbarrier.
+// MMA issue is split over two warps (one elected lane of each issues), since
+// one lane issues at most about one tcgen05.mma per ~47 cycles while a
+// 128 x 64 x 16 MMA takes 32:
+//   issuer A (warp 1): S(t) = A0 X(t)^T and dP(t) = A1 Y(t)^T into buffer
+//                      t&1, once the accumulating MMAs of tile t-2 (same
+//                      buffer) have entered the tensor pipe;
+//   issuer B (warp 2): acc(t) once the softmax warps have written tile t's
+//                      bf16 operands.
+// The pipe executes the CTA's MMAs in the order they enter it; every
+// hand-over between the issuers and the other roles goes through an mbarrier.
 template <bool kKV>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
@@ -269,7 +270,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       const uint64_t xm_desc = sdesc_sw128(base + LY::X, kTHalf, 1024);   // MN-major view
       const uint64_t yk_desc = sdesc_sw128(base + LY::Y, 16, 1024);
       const uint64_t ym_desc = sdesc_sw128(base + LY::Y, kTHalf, 1024);
-      // First MMAs of tile t: S = A0 X^T (issuer A) or dP = A1 Y^T (issuer B).
+      // First MMAs of tile t (issuer A): S = A0 X^T or dP = A1 Y^T.
       auto issue_first = [&](const Cursor& c, bool s_mma) -> bool {
         const uint32_t b = c.t & 1u;
         if (c.j == 0 && !wait_w(bar(B_AF), c.item_idx & 1)) return false;
@@ -347,32 +348,23 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         return true;
       };
       bool ok = true;
+      Cursor c;
+      c.start(p, ring, kConsumerWarp);
       if (issuer_a) {
-        Cursor cs;
-        cs.start(p, ring, kConsumerWarp);
         // Failure-detection test: wait on the drain barrier's first phase,
         // which nothing completes before this warp's own drain commit, so the
         // bounded wait runs out and the abort path below is taken.
         if (p.stall_test) ok = __all_sync(0xffffffffu, wait_bar(bar(B_DRAIN + 0), 0u, p, abort_flag));
-        while (cs.valid && ok) {
-          ok = issue_first(cs, true);
-          cs.next(p, ring, kConsumerWarp);
+        // S(t), then dP(t): both overwrite buffer t&1 and follow acc(t-2).
+        while (c.valid && ok) {
+          ok = issue_first(c, true) && issue_first(c, false);
+          c.next(p, ring, kConsumerWarp);
         }
       } else {
-        // dP runs up to two tiles ahead of acc, but not into the next item:
-        // that item's stationary operands (dQ pass) are stored only after
-        // the epilogue of this one, which waits for this item's last acc.
-        Cursor cd, ca;
-        cd.start(p, ring, kConsumerWarp);
-        ca.start(p, ring, kConsumerWarp);
-        while (ca.valid && ok) {
-          while (ok && cd.valid && cd.t < ca.t + 2 && cd.item_idx == ca.item_idx) {
-            ok = issue_first(cd, false);
-            cd.next(p, ring, kConsumerWarp);
-          }
-          if (!ok) break;
-          ok = issue_acc(ca);
-          ca.next(p, ring, kConsumerWarp);
+        // Issuer B only accumulates, so it takes P(t) as soon as it lands.
+        while (c.valid && ok) {
+          ok = issue_acc(c);
+          c.next(p, ring, kConsumerWarp);
         }
       }
       if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
@@ -525,9 +517,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
 
       if (c.j == c.n - 1) {
         // ------------------------------------------------------ epilogue --
-        // acc(t-2), the previous phase of this barrier, has completed:
-        // issuer B issued it before dP(t), whose S-ready commit (covering
-        // all of issuer B's earlier MMAs) this warp has seen land.
+        // acc(t-2), the previous phase of this barrier, has completed: it
+        // entered the tensor pipe before S(t) and dP(t), whose completion
+        // this warp has seen, and the pipe runs the CTA's MMAs in order.
         ok = wait_bar(bar(B_MD + (c.t & 1u)), (c.t >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
