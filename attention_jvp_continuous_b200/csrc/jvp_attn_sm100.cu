@@ -17,8 +17,9 @@
 //
 // Warp roles (384 threads, one CTA per SM, persistent over the work list):
 //   warp 0       TMA producer: Q/dQ per query tile, K|dK and V|dV rings of 2
-//   warp 1       TMEM owner; issues S(t) (whole warp, one elected lane)
-//   warp 2       issues PV(t) (whole warp, one elected lane)
+//   warp 1       TMEM owner; issues PV(t) and then S(t+2) (whole warp, one
+//                elected lane)
+//   warp 2       issues dS += dQ K^T(t) once S(t) has completed
 //   warps 4..11  softmax/JVP state, P write-back to TMEM, epilogue: two
 //                warpgroups, each taking 32 of a tile's 64 key columns of
 //                every row (one row per thread), exchanging row maxima
@@ -88,7 +89,6 @@ enum : uint32_t {
   B_IEMPTY = 30,  // 4 slots: work-item ring, released
   B_DRAIN2 = 34,  // drain barrier of the second MMA warp
   B_SAFULL = 35,  // 2: S and Q dK^T of buffer t&1 complete (dQ K^T may still run)
-  B_PVI = 37,     // 2: PV(t) of buffer t&1 issued (not complete)
   B_PDFULL = 39,  // 2: scale e dS of buffer t&1 written (B_PFULL: e written)
   kNumBars = 41
 };
@@ -161,7 +161,6 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar(B_PVD + s), 1);
       mbar_init(bar(B_SFULL + s), 1);
       mbar_init(bar(B_SAFULL + s), 1);
-      mbar_init(bar(B_PVI + s), 1);
       mbar_init(bar(B_PFULL + s), 2 * BM);
       mbar_init(bar(B_PDFULL + s), 2 * BM);
     }
@@ -172,7 +171,7 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int i = 0; i < 4; ++i) mbar_init(bar(B_XSUM + i), 64);
     for (int i = 0; i < int(kRing); ++i) {
       mbar_init(bar(B_IFULL + i), 1);
-      mbar_init(bar(B_IEMPTY + i), kRingReaders);
+      mbar_init(bar(B_IEMPTY + i), kRingReaders + 1);  // 3 MMA-warp cursors
     }
     *abort_flag = 0u;
     fence_mbar_init();
@@ -234,8 +233,9 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         tma_load_3d(ks + 2 * kKHalf, &tm_k, bar(B_KFULL + s), 64, y, c.bh);
         tma_load_3d(ks + 3 * kKHalf, &tm_dk, bar(B_KFULL + s), 64, y, c.bh);
         // V stage s is free once PV(t - 2) is done. PV(t - 4), the previous
-        // phase of that barrier, ran on the tensor pipe before S(t - 2),
-        // which was waited for just above, so the parity wait is unambiguous.
+        // phase of that barrier, was issued by warp 1 before S(t - 2), which
+        // completed before dQ K^T(t - 2) was issued; that was waited for just
+        // above, so the parity wait is unambiguous.
         if (c.t >= 2) ok = wait_bar(bar(B_PVD + s), (u - 1) & 1u, p, abort_flag);
         if (!ok) break;
         mbar_expect_tx(bar(B_VFULL + s), kStageBytes);
@@ -260,17 +260,16 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncwarp();
   } else if (warp == 1 || warp == 2) {
     // ----------------------------------------------------------- MMA ----
-    // Issue is split over two warps: warp 1 issues S(t) (Q [K ; dK]^T and
-    // dQ K^T), warp 2 PV(t) ([A1 | A23] += P [V | dV], A23 += Pds V). Each
-    // runs its loop as a whole warp in uniform control flow and one elected
-    // lane issues its MMAs and commits. S(t) overwrites the TMEM buffer whose
-    // P PV(t-2) reads, so warp 1 issues it only after warp 2 has issued
-    // PV(t-2) (an mbarrier arrive behind tcgen05.fence::before_thread_sync,
-    // and tcgen05.fence::after_thread_sync on the waiting side): the CTA's
-    // MMAs run in the order they enter the tensor pipe. Otherwise the two
-    // streams are independent.
+    // Issue is split over two warps, each running its loop as a whole warp
+    // in uniform control flow with one elected lane issuing its MMAs and
+    // commits. Warp 1 issues PV(t) ([A1 | A23] += P [V | dV], A23 += Pds V)
+    // and then [S | Q dK^T](t+2) = Q [K ; dK]^T: S(t+2) overwrites the TMEM
+    // buffer whose P PV(t) reads, and the MMAs of one thread run in issue
+    // order. Warp 2 issues dS += dQ K^T(t) once the N=128 MMAs of tile t
+    // have completed (their commit, which the softmax also waits for): MMAs
+    // of different warps are ordered only through completions.
     {
-      const bool s_warp = warp == 1;
+      const bool w1 = warp == 1;
       bool ok = true;
       // Descriptors of the fixed shared-memory operands; an MMA's operand
       // is the base plus a compile-time byte offset >> 4 (the start-address
@@ -279,56 +278,51 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint64_t dq_desc = sdesc_sw128(base + SM_DQ, 16, 1024);
       const uint64_t k_desc = sdesc_sw128(base + SM_K, 16, 1024);       // stage 0
       const uint64_t v_desc = sdesc_sw128(base + SM_V, kKHalf, 1024);   // stage 0
-      Cursor c;
-      c.start(p, ring, kConsumerWarp);
-      // Failure-detection test: wait on the drain barrier's first phase,
-      // which nothing completes before this warp's own drain commit, so the
-      // bounded wait runs out and the abort path below is taken.
-      if (p.stall_test && s_warp)
-        ok = __all_sync(0xffffffffu, wait_bar(bar(B_DRAIN), 0u, p, abort_flag));
-      if (s_warp) {
-        while (ok && c.valid) {
-          const uint32_t b = c.t & 1u, par = (c.t >> 1) & 1u;
-          const bool need_q = c.j == 0, need_pv = c.t >= 2;
-          // All of the tile's barriers are tested back to back (they are
-          // normally complete already), then waited for one by one.
-          bool r = mbar_test(bar(B_KFULL + b), par);
-          r = r && (!need_q || mbar_test(bar(B_QFULL), c.item_idx & 1));
-          r = r && (!need_pv || mbar_test(bar(B_PVI + b), par ^ 1u));
-          if (!__all_sync(0xffffffffu, r)) {
-            bool w = !need_pv || wait_bar(bar(B_PVI + b), par ^ 1u, p, abort_flag);
-            w = w && (!need_q || wait_bar(bar(B_QFULL), c.item_idx & 1, p, abort_flag));
-            w = w && wait_bar(bar(B_KFULL + b), par, p, abort_flag);
-            ok = __all_sync(0xffffffffu, w);
-            if (!ok) break;
-          }
-          tc_fence_after();
-          const bool last = c.j == c.n - 1;
-          const uint64_t kb = k_desc + b * (kStageBytes >> 4);
-          // [S | Q dK^T] = Q [K ; dK]^T: one N=128 MMA per 16-wide k-step.
+      // Each wait first tests all of its barriers back to back (they are
+      // normally complete already) and falls back to the bounded waits one
+      // by one.
+      // S(t): K|dK stage, and Q for a new item.
+      auto wait_k = [&](const Cursor& c) -> bool {
+        const uint32_t b = c.t & 1u, par = (c.t >> 1) & 1u;
+        const bool need_q = c.j == 0;
+        const bool r = mbar_test(bar(B_KFULL + b), par) &&
+                       (!need_q || mbar_test(bar(B_QFULL), c.item_idx & 1));
+        if (__all_sync(0xffffffffu, r)) return true;
+        bool w = !need_q || wait_bar(bar(B_QFULL), c.item_idx & 1, p, abort_flag);
+        w = w && wait_bar(bar(B_KFULL + b), par, p, abort_flag);
+        return __all_sync(0xffffffffu, w);
+      };
+      // [S | Q dK^T] = Q [K ; dK]^T: one N=128 MMA per 16-wide k-step.
+      auto issue_sa = [&](const Cursor& c) {
+        const uint32_t b = c.t & 1u;
+        const uint64_t kb = k_desc + b * (kStageBytes >> 4);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t oq = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
-            const uint32_t ob = ((kk >> 2) * (2 * kKHalf) + (kk & 3) * 32) >> 4;
-            mma_ss_elect(tmem + b * 128u, q_desc + oq, kb + ob, IDESC_SK, kk > 0);
-          }
-          mma_commit_elect(bar(B_SAFULL + b));  // S ready: the softmax starts on it
-          // dS = Q dK^T + dQ K^T: N=64 MMAs accumulate dQ K^T onto it.
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t oq = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
-            const uint32_t ob = ((kk >> 2) * (2 * kKHalf) + (kk & 3) * 32) >> 4;
-            mma_ss_elect(tmem + b * 128u + 64u, dq_desc + oq, kb + ob, IDESC_S, 1u);
-          }
-          mma_commit_elect(bar(B_SFULL + b));  // also releases K stage b to the producer
-          if (last) mma_commit_elect(bar(B_QEMPTY));
-          c.next(p, ring, kConsumerWarp);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t oq = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
+          const uint32_t ob = ((kk >> 2) * (2 * kKHalf) + (kk & 3) * 32) >> 4;
+          mma_ss_elect(tmem + b * 128u, q_desc + oq, kb + ob, IDESC_SK, kk > 0);
         }
-      } else {
-        while (ok && c.valid) {
-          const uint32_t b = c.t & 1u, par = (c.t >> 1) & 1u;
-          const bool need_a = c.j == 0 && c.item_idx > 0;
-          const uint32_t pa = (c.item_idx - 1) & 1;
+        mma_commit_elect(bar(B_SAFULL + b));  // S ready: the softmax and warp 2 go on
+      };
+      if (w1) {
+        Cursor cs, cp;  // S runs up to two tiles ahead of PV
+        cs.start(p, ring, kConsumerWarp);
+        cp.start(p, ring, kConsumerWarp);
+        // Failure-detection test: wait on the drain barrier's first phase,
+        // which nothing completes before this warp's own drain commit, so the
+        // bounded wait runs out and the abort path below is taken.
+        if (p.stall_test) ok = __all_sync(0xffffffffu, wait_bar(bar(B_DRAIN), 0u, p, abort_flag));
+        for (int pre = 0; pre < 2 && ok && cs.valid; ++pre) {
+          ok = wait_k(cs);
+          if (!ok) break;
+          tc_fence_after();
+          issue_sa(cs);
+          cs.next(p, ring, kConsumerWarp);
+        }
+        while (ok && cp.valid) {
+          const uint32_t b = cp.t & 1u, par = (cp.t >> 1) & 1u;
+          const bool need_a = cp.j == 0 && cp.item_idx > 0;
+          const uint32_t pa = (cp.item_idx - 1) & 1;
           bool r = mbar_test(bar(B_PFULL + b), par);
           r = r && mbar_test(bar(B_VFULL + b), par);
           r = r && (!need_a || mbar_test(bar(B_AFREE), pa));
@@ -341,7 +335,7 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
           tc_fence_after();
           const uint64_t vb = v_desc + b * (kStageBytes >> 4);
-          const uint32_t first = c.j == 0 ? 0u : 1u;
+          const uint32_t first = cp.j == 0 ? 0u : 1u;
           // [A1 | A23] += P [V | dV]: one N=256 MMA per 16-key step (A1 and
           // A23 are adjacent in TMEM; V h0, V h1, dV h0, dV h1 are 8 KB apart).
 #pragma unroll
@@ -361,17 +355,55 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             mma_ts_elect(tmem + TM_A23, tmem + b * 128u + 64u + (ks >> 1) * 32u + (ks & 1) * 8u,
                          vb + ((ks * 2048) >> 4), IDESC_PV, 1u);
           mma_commit_elect(bar(B_PVD + b));  // PV(t) done: V stage free, A1/A23 current
-          // PV(t) is in the tensor pipe's queue: S(t+2) may follow it (the
-          // pipe runs the CTA's MMAs in the order they enter the queue).
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_PVI + b));
+          cp.next(p, ring, kConsumerWarp);
+          // S(t+2) follows PV(t) in this thread's order. (dQ K^T(t) has
+          // completed too: the softmax waited for it before publishing the
+          // scale e dS that PV(t) read.)
+          if (cs.valid) {
+            ok = wait_k(cs);
+            if (!ok) break;
+            tc_fence_after();
+            issue_sa(cs);
+            cs.next(p, ring, kConsumerWarp);
+          }
+        }
+      } else {
+        // dS = Q dK^T + dQ K^T: N=64 MMAs accumulate dQ K^T onto the N=128
+        // result once it has completed. This warp waits for its own operands
+        // (K stage, dQ) as well.
+        Cursor c;
+        c.start(p, ring, kConsumerWarp);
+        while (ok && c.valid) {
+          const uint32_t b = c.t & 1u, par = (c.t >> 1) & 1u;
+          const bool need_q = c.j == 0;
+          bool r = mbar_test(bar(B_SAFULL + b), par) && mbar_test(bar(B_KFULL + b), par) &&
+                   (!need_q || mbar_test(bar(B_QFULL), c.item_idx & 1));
+          if (!__all_sync(0xffffffffu, r)) {
+            bool w = wait_bar(bar(B_SAFULL + b), par, p, abort_flag);
+            w = w && wait_bar(bar(B_KFULL + b), par, p, abort_flag);
+            w = w && (!need_q || wait_bar(bar(B_QFULL), c.item_idx & 1, p, abort_flag));
+            ok = __all_sync(0xffffffffu, w);
+            if (!ok) break;
+          }
+          tc_fence_after();
+          const uint64_t kb = k_desc + b * (kStageBytes >> 4);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t oq = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
+            const uint32_t ob = ((kk >> 2) * (2 * kKHalf) + (kk & 3) * 32) >> 4;
+            mma_ss_elect(tmem + b * 128u + 64u, dq_desc + oq, kb + ob, IDESC_S, 1u);
+          }
+          // dS ready; with the N=128 MMAs of tile t complete before these
+          // were issued, this also releases K stage b (and, after the
+          // item's last tile, Q and dQ).
+          mma_commit_elect(bar(B_SFULL + b));
+          if (c.j == c.n - 1) mma_commit_elect(bar(B_QEMPTY));
           c.next(p, ring, kConsumerWarp);
         }
       }
       if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
         // Wait for every MMA this warp issued before TMEM is freed.
-        const uint32_t db = bar(s_warp ? B_DRAIN : B_DRAIN2);
+        const uint32_t db = bar(w1 ? B_DRAIN : B_DRAIN2);
         mma_commit_elect(db);
         drain_wait(db, 0);
       }
@@ -456,9 +488,9 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         g *= alpha;
         // A1/A23 hold PV(t-1); wait for it, then scale this quarter's rows:
         // the first warpgroup scales A1, the second A23.
-        // (PV(t-3), the previous phase of that barrier, entered the tensor
-        // pipe before S(t-1), whose completion this warp has seen, and the
-        // pipe runs the CTA's MMAs in order.)
+        // (PV(t-3), the previous phase of that barrier, was issued by warp 1
+        // before S(t), whose commit, covering all of that warp's earlier
+        // MMAs, this warp has seen land.)
         ok = wait_bar(bar(B_PVD + ((c.t - 1) & 1u)), ((c.t - 1) >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
@@ -540,9 +572,10 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
       if (c.j == c.n - 1) {
         // ------------------------------------------------------ epilogue --
-        // PV(t) done. PV(t-2), the previous phase of this barrier, entered
-        // the tensor pipe before S(t), whose completion this warp has seen,
-        // so it has completed and the parity wait is unambiguous.
+        // PV(t) done. PV(t-2), the previous phase of this barrier, was issued
+        // by warp 1 before S(t), whose commit (covering all of that warp's
+        // earlier MMAs) this warp has seen land, so the parity wait is
+        // unambiguous.
         ok = wait_bar(bar(B_PVD + (c.t & 1u)), (c.t >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         // Row totals of l and g from both halves.
