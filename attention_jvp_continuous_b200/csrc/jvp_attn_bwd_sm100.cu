@@ -90,8 +90,7 @@ enum : uint32_t {
   B_DRAIN = 29,  // 2: one per issuer
   B_IF = 31,     // 4: work-item ring
   B_IE = 35,     // 4
-  B_AI = 39,     // 2: accumulating MMAs of the buffer's last tile issued
-  kNumBars = 41
+  kNumBars = 39
 };
 static_assert(kNumBars <= 44, "barrier slots");
 static_assert(Layout<false>::RING + 16 <= Layout<false>::BAR + 512, "barrier area overflow");
@@ -135,11 +134,12 @@ using Cursor = pipe::Cursor<Params>;
 // 128 x 64 x 16 MMA takes 32:
 //   issuer A (warp 1): S(t) = A0 X(t)^T and dP(t) = A1 Y(t)^T into buffer
 //                      t&1, once the accumulating MMAs of tile t-2 (same
-//                      buffer) have entered the tensor pipe;
+//                      buffer) have completed (MMAs of different warps are
+//                      ordered only through completions);
 //   issuer B (warp 2): acc(t) once the softmax warps have written tile t's
 //                      bf16 operands.
-// The pipe executes the CTA's MMAs in the order they enter it; every
-// hand-over between the issuers and the other roles goes through an mbarrier.
+// One thread's MMAs run in issue order; every hand-over between the issuers
+// and the other roles goes through an mbarrier.
 template <bool kKV>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
@@ -174,7 +174,6 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       mbar_init(bar(B_SF + b), 2);
       mbar_init(bar(B_PF + b), 2 * BR);
       mbar_init(bar(B_MD + b), 1);
-      mbar_init(bar(B_AI + b), 1);
       mbar_init(bar(B_DRAIN + b), 1);
     }
     mbar_init(bar(B_CF), 2 * BR);
@@ -278,11 +277,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         uint64_t bdesc;
         if (s_mma) {
           // Buffer b last held tile t-2, whose operands acc(t-2) reads: S(t)
-          // is issued once acc(t-2) has entered the tensor pipe (issuer B
-          // arrives behind tcgen05.fence::before_thread_sync; the
-          // tc_fence_after below completes the pair), and the pipe runs the
-          // CTA's MMAs in the order they enter it.
-          if (c.t >= 2 && !wait_w(bar(B_AI + b), ((c.t >> 1) - 1) & 1u))
+          // and dP(t) wait until those MMAs (issuer B's) have completed.
+          if (c.t >= 2 && !wait_w(bar(B_MD + b), ((c.t >> 1) - 1) & 1u))
             return false;
           stage = c.t % NX;
           if (!wait_w(bar(B_XF + stage), (c.t / NX) & 1u)) return false;
@@ -342,9 +338,6 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         mma_commit_elect(bar(B_XE + sx));
         if (kKV) mma_commit_elect(bar(B_YE + sy));
         mma_commit_elect(bar(B_MD + b));
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_AI + b));  // acc(t) issued: S(t+2) may follow
         return true;
       };
       bool ok = true;
@@ -517,9 +510,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
 
       if (c.j == c.n - 1) {
         // ------------------------------------------------------ epilogue --
-        // acc(t-2), the previous phase of this barrier, has completed: it
-        // entered the tensor pipe before S(t) and dP(t), whose completion
-        // this warp has seen, and the pipe runs the CTA's MMAs in order.
+        // acc(t-2), the previous phase of this barrier, has completed:
+        // issuer A waited for it before issuing S(t) and dP(t), which this
+        // warp has seen complete.
         ok = wait_bar(bar(B_MD + (c.t & 1u)), (c.t >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
