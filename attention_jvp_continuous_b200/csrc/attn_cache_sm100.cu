@@ -11,7 +11,8 @@
 //   warp 1       TMEM owner; issues S = Q K^T (N = 128) into a double
 //                buffer
 //   warp 2       issues O += P V (N = 128, P from TMEM); S(t+2) is issued
-//                only once PV(t) is in the tensor pipe's queue
+//                once PV(t) has completed (MMAs of different warps are
+//                ordered only through completions)
 //   warps 4-11   softmax: two warpgroups, each 64 of a tile's 128 keys of
 //                every row with its own running max and its own O
 //                accumulator (lazy rescale only when its row max grows by
@@ -78,7 +79,6 @@ enum : uint32_t {
   B_XSUM = 20,    // 4: [lane quarter], end-of-item merge of the halves
   B_IFULL = 24,   // 4
   B_IEMPTY = 28,  // 4
-  B_PVI = 32,     // 2: PV MMAs of the buffer's latest tile issued (not complete)
   B_DRAIN2 = 34,  // drain barrier of the PV-issuing warp
   kNumBars = 35
 };
@@ -140,7 +140,6 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar(B_SFULL + s), 1);
       mbar_init(bar(B_PFULL + s), 2 * BM);
       mbar_init(bar(B_PVD + s), 1);
-      mbar_init(bar(B_PVI + s), 1);
     }
     mbar_init(bar(B_AFREE), 2 * BM);
     mbar_init(bar(B_DRAIN), 1);
@@ -231,10 +230,10 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       auto issue_s = [&](const Cursor& c) -> bool {
         const uint32_t b = c.t & 1u, sk = c.t % NK;
         if (c.j == 0 && !wait_w(bar(B_QFULL), c.item_idx & 1)) return false;
-        // Buffer b last held tile t-2, whose P PV(t-2) reads: issue S(t) once
-        // PV(t-2) is in the tensor pipe's queue (the pipe runs the CTA's MMAs
-        // in the order they enter it).
-        if (c.t >= 2 && !wait_w(bar(B_PVI + b), ((c.t >> 1) - 1) & 1u)) return false;
+        // Buffer b last held tile t-2, whose P PV(t-2) reads: S(t) waits
+        // until those MMAs (warp 2's) have completed; MMAs of different warps
+        // are ordered only through completions.
+        if (c.t >= 2 && !wait_w(bar(B_PVD + b), ((c.t >> 1) - 1) & 1u)) return false;
         if (!wait_w(bar(B_KFULL + sk), (c.t / NK) & 1u)) return false;
         tc_fence_after();
         const uint64_t kb = k_desc + sk * (kStage >> 4);
@@ -269,12 +268,9 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                  vb + ((ks * 2048) >> 4), IDESC_PV, first | ((ks & 3) > 0));
         mma_commit_elect(bar(B_VEMPTY + b));
         mma_commit_elect(bar(B_PVD + b));
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_PVI + b));  // PV(t) issued: S(t+2) may follow
         return true;
       };
-      // Warp 1 issues S(t), warp 2 PV(t); S(t+2) follows PV(t) in the pipe.
+      // Warp 1 issues S(t), warp 2 PV(t); S(t+2) waits for PV(t) to complete.
       const bool s_warp = warp == 1;
       Cursor c;
       c.start(p, ring, kConsumerWarp);
@@ -361,8 +357,7 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (__any_sync(0xffffffffu, need)) {
         l *= alpha;
         // This O holds PV(t-1); wait for it. (PV(t-3), the previous phase of
-        // that barrier, entered the tensor pipe before S(t-1), whose
-        // completion this warp has seen.)
+        // that barrier, completed before S(t-1) was issued.)
         ok = wait_bar(bar(B_PVD + ((c.t - 1) & 1u)), ((c.t - 1) >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
@@ -405,8 +400,8 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
       if (c.j == c.n - 1) {
         // ------------------------------------------------------ epilogue --
-        // PV(t) done; PV(t-2), the previous phase of this barrier, entered
-        // the tensor pipe before S(t), whose completion this warp has seen.
+        // PV(t) done; PV(t-2), the previous phase of this barrier, completed
+        // before S(t) was issued.
         ok = wait_bar(bar(B_PVD + (c.t & 1u)), (c.t >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         xsum[hw * BM + r] = m_ref;
