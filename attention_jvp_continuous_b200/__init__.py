@@ -19,7 +19,7 @@ FRAME_CAUSAL = 1
 CHUNK_CAUSAL = 2
 TEACHER_FORCING = 3
 
-__all__ = ["Mask", "jvp_attn", "jvp_attn_fwd", "attn_bwd", "jvp_attn_bwd", "bwd_scratch_len",
+__all__ = ["Mask", "jvp_attn", "jvp_attn_fwd", "jvp_attn_scatter", "attn_bwd", "jvp_attn_bwd", "bwd_scratch_len",
            "cache_attn", "rope_copy", "qkv_prologue", "mask_stats", "tile_classes",
            "schedule", "schedule_kv", "check_device_error", "set_wait_limit", "set_stall_test", "release",
            "JvpAttnError",
@@ -68,6 +68,48 @@ def jvp_attn_fwd(q, k, v, dq, dk, dv, o, d_o, lse, mask: Mask,
         B, H, L, d, _dtype_code(q), mask.desc(),
         0.0 if scale is None else float(scale), ctypes.c_void_p(stream))
     _lib.check(rc, "jvp_attn_fwd")
+
+
+def jvp_attn_scatter(q, k, v, dq, dk, dv, mask: Mask, o_dst, do_dst, lse_dst, h0: int,
+                     scale: Optional[float] = None) -> None:
+    """Masked attention JVP of this rank's head group whose epilogue writes
+    every output row into the token shard that owns it (the output exchange
+    of Ulysses context parallelism, fused into the kernel).
+
+    q, k, v, dq, dk, dv: CUDA bf16 [B, H, L, d] (d = 128), the head group
+    h0 .. h0 + H - 1 of all L tokens. o_dst, do_dst: sequences of P bf16
+    tensors [B, H_total, L/P, d]; lse_dst: P float32 tensors [B, H_total,
+    L/P]. Entry r may be a view of another GPU's memory (a symmetric-memory
+    buffer); row n goes to entry n // (L/P). Rows of heads outside this
+    group are not written. Enqueued on the current stream; peers see the
+    rows after this launch completes and the ranks synchronise.
+    """
+    import torch
+    ts = (q, k, v, dq, dk, dv)
+    for t in ts:
+        if not t.is_cuda or t.dtype != torch.bfloat16 or t.shape != q.shape or not t.is_contiguous():
+            raise ValueError("q, k, v, dq, dk, dv must be contiguous CUDA bf16 [B, H, L, d]")
+    B, H, L, d = q.shape
+    P = len(o_dst)
+    if not (len(do_dst) == P == len(lse_dst)) or P < 1:
+        raise ValueError("o_dst, do_dst and lse_dst must list the same number of shards")
+    if L % P:
+        raise ValueError(f"{L} tokens do not split over {P} shards")
+    Ht = o_dst[0].shape[1]
+    for o_, do_, l_ in zip(o_dst, do_dst, lse_dst):
+        if (o_.shape != (B, Ht, L // P, d) or do_.shape != o_.shape or o_.dtype != torch.bfloat16
+                or do_.dtype != torch.bfloat16 or not o_.is_contiguous() or not do_.is_contiguous()):
+            raise ValueError("o_dst / do_dst entries must be contiguous bf16 [B, H_total, L/P, d]")
+        if l_.shape != (B, Ht, L // P) or l_.dtype != torch.float32 or not l_.is_contiguous():
+            raise ValueError("lse_dst entries must be contiguous float32 [B, H_total, L/P]")
+    arr = lambda ts_: (ctypes.c_void_p * P)(*[t.data_ptr() for t in ts_])
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    rc = _lib.lib().jvp_attn_fwd_scatter(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+        arr(o_dst), arr(do_dst), arr(lse_dst), P, int(h0), Ht,
+        B, H, L, d, _dtype_code(q), mask.desc(),
+        0.0 if scale is None else float(scale), ctypes.c_void_p(stream))
+    _lib.check(rc, "jvp_attn_fwd_scatter")
 
 
 def jvp_attn(q, k, v, dq, dk, dv, mask: Mask, scale: Optional[float] = None,

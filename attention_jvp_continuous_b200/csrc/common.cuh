@@ -20,6 +20,9 @@ struct WorkList {
   int n_segs = 0;
 };
 
+// Destinations of the scatter epilogue (token shards of a Ulysses group).
+constexpr int kMaxShards = 8;
+
 struct LaunchArgs {
   const void *q, *k, *v, *dq, *dk, *dv;
   void *o, *d_o;
@@ -35,6 +38,14 @@ struct LaunchArgs {
   unsigned* item_ctr = nullptr;
   unsigned long long wait_limit_ns;
   bool stall_test = false;  // jvp_attn_set_stall_test
+  // Scatter epilogue (jvp_attn_fwd_scatter), tensor-core kernel only: when
+  // n_shards > 0, o / d_o / lse are unused and row n of local head (b, h)
+  // goes to token-shard owner r = n / (L / n_shards), row n % (L / n_shards)
+  // of head h0 + h in o_dst[r], d_o_dst[r], lse_dst[r] ([B, h_total, L/n_shards, d]).
+  int n_shards = 0, h0 = 0, h_total = 0;
+  void* o_dst[kMaxShards] = {};
+  void* d_o_dst[kMaxShards] = {};
+  float* lse_dst[kMaxShards] = {};
 };
 
 // CUDA-core kernel (fp32 arithmetic) for fp32 or bf16 inputs, d in {32,64,96,128}.

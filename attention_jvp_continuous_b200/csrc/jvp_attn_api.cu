@@ -265,6 +265,65 @@ int jvp_attn_fwd(const void* q, const void* k, const void* v, const void* dq, co
   return launch_sm100(a, w, di->sms);
 }
 
+int jvp_attn_fwd_scatter(const void* q, const void* k, const void* v, const void* dq,
+                         const void* dk, const void* dv, void* const* o_dst,
+                         void* const* d_o_dst, float* const* lse_dst, int n_shards, int h0,
+                         int h_total, int B, int H, int L, int d, jvp_dtype dtype,
+                         jvp_mask_desc mask, float softmax_scale, void* stream) {
+  if (!q || !k || !v || !dq || !dk || !dv || !o_dst || !d_o_dst || !lse_dst)
+    return JVP_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || L <= 0 || d <= 0) return JVP_ERR_INVALID_ARG;
+  if (dtype != JVP_BF16 && dtype != JVP_FP32) return JVP_ERR_INVALID_ARG;
+  if (std::isnan(softmax_scale) || std::isinf(softmax_scale)) return JVP_ERR_INVALID_ARG;
+  if (n_shards < 1 || n_shards > kMaxShards || L % n_shards != 0) return JVP_ERR_INVALID_ARG;
+  if (h0 < 0 || h_total < H || h0 > h_total - H) return JVP_ERR_INVALID_ARG;
+  int rc = validate_mask(mask, L);
+  if (rc != JVP_OK) return rc;
+  if ((long long)B * h_total * L >= (1LL << 31) || (long long)B * H >= (1LL << 31) / 2)
+    return JVP_ERR_TOO_LARGE;
+  if (dtype != JVP_BF16 || d != 128) return JVP_ERR_UNSUPPORTED_HEAD_DIM;
+  const void* ptrs[] = {q, k, v, dq, dk, dv};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return JVP_ERR_MISALIGNED;
+  for (int r = 0; r < n_shards; ++r) {
+    if (!o_dst[r] || !d_o_dst[r] || !lse_dst[r]) return JVP_ERR_INVALID_ARG;
+    if (!aligned16(o_dst[r]) || !aligned16(d_o_dst[r]) || !aligned16(lse_dst[r]))
+      return JVP_ERR_MISALIGNED;
+  }
+
+  DevInfo* di = nullptr;
+  rc = device_info(&di);
+  if (rc != JVP_OK) return rc;
+  if (di->major != 10 || di->minor != 0) return JVP_ERR_UNSUPPORTED_DEVICE;
+
+  LaunchArgs a;
+  a.q = q; a.k = k; a.v = v; a.dq = dq; a.dk = dk; a.dv = dv;
+  a.o = nullptr; a.d_o = nullptr; a.lse = nullptr;
+  a.B = B; a.H = H; a.L = L; a.d = d;
+  a.mask = mask;
+  a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(d));
+  a.stream = static_cast<cudaStream_t>(stream);
+  a.err = di->err;
+  a.wait_limit_ns = wait_limit_ns();
+  a.stall_test = stall_test();
+  a.n_shards = n_shards;
+  a.h0 = h0;
+  a.h_total = h_total;
+  for (int r = 0; r < n_shards; ++r) {
+    a.o_dst[r] = o_dst[r];
+    a.d_o_dst[r] = d_o_dst[r];
+    a.lse_dst[r] = lse_dst[r];
+  }
+  int dev = 0;
+  cudaGetDevice(&dev);
+  WorkList w;
+  rc = get_worklist(dev, mask, L, &w);
+  if (rc != JVP_OK) return rc;
+  rc = get_counter(dev, a.stream, &a.item_ctr);
+  if (rc != JVP_OK) return rc;
+  return launch_sm100(a, w, di->sms);
+}
+
 int jvp_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* g_o,
                  const float* lse, void* g_q, void* g_k, void* g_v, float* scratch,
                  int64_t scratch_len, int B, int H, int L, int d, jvp_dtype dtype,

@@ -121,6 +121,13 @@ struct Params {
   unsigned* item_ctr;  // zero at launch; CTAs take work items from it in list order
   unsigned long long wait_limit_ns;
   int stall_test;  // the MMA warp first waits on a phase that nothing completes
+  // Scatter epilogue: 0 = rows go to o, d_o, lse ([B*H, L, d]); otherwise
+  // row n of local head (b, h) goes to shard r = n / shard_len, row
+  // n % shard_len, head h0 + h of [B, h_total, shard_len, d] in o_dst[r] etc.
+  int n_shards, shard_len, h_local, h0, h_total;
+  __nv_bfloat16* o_dst[kMaxShards];
+  __nv_bfloat16* d_o_dst[kMaxShards];
+  float* lse_dst[kMaxShards];
 };
 
 using pipe::wait_bar;
@@ -590,7 +597,27 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
         const float mu = p.scale * gt * inv;
         const bool row_ok = grow < p.L;
-        const size_t off = (size_t(c.bh) * p.L + (row_ok ? grow : 0)) * D;
+        // Destination rows: this launch's [B*H, L, d] outputs, or (scatter
+        // epilogue) the token-shard owner's buffers, possibly a peer GPU's
+        // memory reached with plain stores over NVLink.
+        __nv_bfloat16 *orow, *dorow;
+        float* lrow;
+        {
+          const int n = row_ok ? grow : 0;
+          if (p.n_shards == 0) {
+            const size_t off = (size_t(c.bh) * p.L + n) * D;
+            orow = p.o + off;
+            dorow = p.d_o + off;
+            lrow = p.lse + size_t(c.bh) * p.L + n;
+          } else {
+            const int r = n / p.shard_len, nr = n - r * p.shard_len;
+            const int bb = c.bh / p.h_local, hh = c.bh - bb * p.h_local;
+            const size_t row = (size_t(bb) * p.h_total + p.h0 + hh) * p.shard_len + nr;
+            orow = p.o_dst[r] + row * D;
+            dorow = p.d_o_dst[r] + row * D;
+            lrow = p.lse_dst[r] + row;
+          }
+        }
         // This warpgroup writes head-dim columns [64 hw, 64 hw + 64).
 #pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {
@@ -610,8 +637,8 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             pdo[i] = pack_bf16(d0, d1);
           }
           if (row_ok) {
-            uint4* go = reinterpret_cast<uint4*>(p.o + off + col);
-            uint4* gd = reinterpret_cast<uint4*>(p.d_o + off + col);
+            uint4* go = reinterpret_cast<uint4*>(orow + col);
+            uint4* gd = reinterpret_cast<uint4*>(dorow + col);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               go[i] = make_uint4(po[4 * i], po[4 * i + 1], po[4 * i + 2], po[4 * i + 3]);
@@ -622,7 +649,7 @@ jvp_attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         tc_fence_before();
         mbar_arrive(bar(B_AFREE));
         if (row_ok && hw == 0)
-          p.lse[size_t(c.bh) * p.L + grow] =
+          *lrow =
               lt > 0.f ? (m_ref + log2f(lt)) * 0.69314718055994531f : -CUDART_INF_F;
       }
       c.next(p, ring, kConsumerWarp);
@@ -698,6 +725,16 @@ int launch_sm100(const LaunchArgs& a, const WorkList& w, int num_sms) {
   p.item_ctr = a.item_ctr;
   p.wait_limit_ns = a.wait_limit_ns;
   p.stall_test = a.stall_test ? 1 : 0;
+  p.n_shards = a.n_shards;
+  p.shard_len = a.n_shards > 0 ? a.L / a.n_shards : 0;
+  p.h_local = a.H;
+  p.h0 = a.h0;
+  p.h_total = a.h_total;
+  for (int r = 0; r < kMaxShards; ++r) {
+    p.o_dst[r] = static_cast<__nv_bfloat16*>(a.o_dst[r]);
+    p.d_o_dst[r] = static_cast<__nv_bfloat16*>(a.d_o_dst[r]);
+    p.lse_dst[r] = a.lse_dst[r];
+  }
   // The dynamic shared-memory opt-in is a per-device function attribute.
   static std::mutex attr_mu;
   static bool attr_done[64] = {};

@@ -126,6 +126,41 @@ int jvp_attn_fwd(const void* q, const void* k, const void* v,
                  jvp_mask_desc mask, float softmax_scale, void* stream);
 
 /*
+ * jvp_attn_fwd_scatter: jvp_attn_fwd whose epilogue performs the output
+ * exchange of Ulysses context parallelism (Causal-rCM report, Sec. 3.2.1
+ * "Parallelisms" and Sec. 3.2.2 "JVP Ulysses CP"): this rank holds a head
+ * group of all L tokens, and each output row is stored directly into the
+ * token shard that owns it instead of into a local [B, H, L, d] array that
+ * an all-to-all would then redistribute.
+ *   q, k, v, dq, dk, dv  this rank's head group [B, H, L, d], bf16, d = 128
+ *                        (the tensor-core kernel; anything else returns
+ *                        JVP_ERR_UNSUPPORTED_HEAD_DIM).
+ *   o_dst, d_o_dst, lse_dst  HOST arrays of n_shards device pointers; entry
+ *                        r is token-shard owner r's output, [B, h_total,
+ *                        L / n_shards, d] bf16 for O and dO and [B, h_total,
+ *                        L / n_shards] float32 for LSE. Row n (0 <= n < L) of
+ *                        local head h goes to shard r = n / (L / n_shards),
+ *                        row n % (L / n_shards), head h0 + h. An entry may
+ *                        point into another GPU's memory (peer access or a
+ *                        symmetric-memory mapping set up by the caller); the
+ *                        kernel writes it with plain stores. The arrays are
+ *                        read during the call only.
+ *   1 <= n_shards <= 8, L % n_shards == 0, 0 <= h0, h0 + H <= h_total.
+ * Rows of a destination not owned by this head group are left untouched;
+ * with every rank's call, each shard receives all h_total heads. Visibility
+ * on a peer: after this launch completes (e.g. stream synchronisation
+ * followed by a barrier between the ranks). Errors as jvp_attn_fwd, plus
+ * JVP_ERR_INVALID_ARG for a null or out-of-range shard argument and
+ * JVP_ERR_MISALIGNED for a destination not 16-byte aligned.
+ */
+int jvp_attn_fwd_scatter(const void* q, const void* k, const void* v,
+                         const void* dq, const void* dk, const void* dv,
+                         void* const* o_dst, void* const* d_o_dst, float* const* lse_dst,
+                         int n_shards, int h0, int h_total,
+                         int B, int H, int L, int d, jvp_dtype dtype,
+                         jvp_mask_desc mask, float softmax_scale, void* stream);
+
+/*
  * jvp_attn_fwd_noalloc: jvp_attn_fwd for callers that cannot allocate
  * device memory. The paper has no counterpart: it is a deployment variant.
  *

@@ -199,3 +199,41 @@ def test_size_limits():
                                  None)
     assert rc == _lib.JVP_ERR_TOO_LARGE
     assert call_prologue(B=1 << 20, L=1 << 15, rope_rows=1 << 15) == _lib.JVP_ERR_TOO_LARGE
+
+
+def call_scatter(ptr=0x1000, dst=0x2000, P=2, h0=0, Ht=2, B=1, H=1, L=64, d=128,
+                 dtype=_lib.JVP_BF16, mask=(ja.TEACHER_FORCING, 8, 4, 1), scale=0.0,
+                 o_dst=None, null_arrays=False):
+    arr = lambda xs: (ctypes.c_void_p * max(1, len(xs)))(*xs)
+    o = arr([dst] * P if o_dst is None else o_dst)
+    do = arr([dst + 0x1000] * P)
+    ls = arr([dst + 0x2000] * P)
+    if null_arrays:
+        o = None
+    return _lib.lib().jvp_attn_fwd_scatter(
+        *[ctypes.c_void_p(ptr)] * 6, o, do, ls, P, h0, Ht,
+        B, H, L, d, dtype, _lib.MaskDesc(*mask), scale, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(null_arrays=True), _lib.JVP_ERR_INVALID_ARG),
+    (dict(P=0), _lib.JVP_ERR_INVALID_ARG),
+    (dict(P=9), _lib.JVP_ERR_INVALID_ARG),          # more shards than the kernel's table
+    (dict(P=3), _lib.JVP_ERR_INVALID_ARG),          # 64 tokens do not split in 3
+    (dict(h0=2, Ht=2), _lib.JVP_ERR_INVALID_ARG),   # head group past the total
+    (dict(h0=-1), _lib.JVP_ERR_INVALID_ARG),
+    (dict(Ht=0), _lib.JVP_ERR_INVALID_ARG),
+    (dict(o_dst=[0x2000, 0]), _lib.JVP_ERR_INVALID_ARG),
+    (dict(o_dst=[0x2000, 0x2008]), _lib.JVP_ERR_MISALIGNED),
+    (dict(d=64), _lib.JVP_ERR_UNSUPPORTED_HEAD_DIM),  # tensor-core kernel only
+    (dict(dtype=_lib.JVP_FP32), _lib.JVP_ERR_UNSUPPORTED_HEAD_DIM),
+    (dict(ptr=0x1008), _lib.JVP_ERR_MISALIGNED),
+    (dict(L=63), _lib.JVP_ERR_INVALID_ARG),
+])
+def test_scatter_argument_errors(kw, code):
+    assert call_scatter(**kw) == code
+
+
+def test_scatter_valid_call_without_gpu_fails_cleanly():
+    rc = call_scatter()
+    assert rc in (_lib.JVP_ERR_LAUNCH_FAILED, _lib.JVP_ERR_UNSUPPORTED_DEVICE)
