@@ -542,7 +542,8 @@ def run_ours_cache(args, w):
         "gpu_launches": args.steps * 4,
         "roofline": {
             "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": UNIT,
-            "frac": round(achieved / peak, 4), "traffic": None,
+            "frac": round(achieved / peak, 4),
+            "traffic": stored_traffic(w.name + "_cache", "cache", H=H, Lq=Lq, Lk=Lk),
             "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
             "frac_of_sustained": round(achieved / float(peaks.get(
                 "bf16_tflops_sustained", peak)), 4),
