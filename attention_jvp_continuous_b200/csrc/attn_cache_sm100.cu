@@ -95,6 +95,33 @@ constexpr uint32_t TM_O = 256;  // O_a [256, 384) for keys [0, 64), O_b [384, 51
 constexpr uint32_t IDESC_S = ptx::idesc_bf16(BM, BN, false, false);  // 128 x 128, K-major B
 constexpr uint32_t IDESC_PV = ptx::idesc_bf16(BM, D, false, true);   // 128 x 128, MN-major B
 
+// 2^x for a pair on the FMA pipe, for the share of the exponentials that the
+// MUFU unit (16 per cycle per SM, as many per tile as the tensor pipe has
+// cycles of work here) would otherwise serialise. Cody-Waite range
+// reduction: x = n + f with n = round(x), taken from the low bits of
+// x + 1.5 * 2^23, and |f| <= 1/2; 2^f from a cubic whose coefficients were
+// fitted here by iteratively reweighted least squares on [-1/2, 1/2]
+// (relative error below 8e-5 in fp32, well inside the bf16 rounding of P);
+// 2^n assembled in the exponent field. x is clamped at -127 first, where
+// 2^n is exactly 0, so masked entries (x = -inf) give 0. Range: x <= 127.
+__device__ __forceinline__ uint64_t ex2_fma2(float x0, float x1) {
+  constexpr float kShift = 12582912.f;  // 1.5 * 2^23: ulp 1, round to nearest
+  const uint64_t xv = f2pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+  const uint64_t t = add2(xv, f2pack(kShift, kShift));
+  const uint64_t n = add2(t, f2pack(-kShift, -kShift));  // round(x), exact
+  const uint64_t f = fma2(n, f2pack(-1.f, -1.f), xv);    // x - round(x)
+  uint64_t q = fma2(f2pack(0.055171605f, 0.055171605f), f, f2pack(0.24261111f, 0.24261111f));
+  q = fma2(q, f, f2pack(0.69326097f, 0.69326097f));
+  q = fma2(q, f, f2pack(0.99992806f, 0.99992806f));
+  float t0, t1;
+  f2unpack(t, t0, t1);
+  // The low bits of t hold round(x) + 0x4B400000; shifted into the exponent
+  // field the 0x4B400000 part vanishes and +127 << 23 biases it.
+  const float s0 = __uint_as_float((__float_as_uint(t0) << 23) + 0x3F800000u);
+  const float s1 = __uint_as_float((__float_as_uint(t1) << 23) + 0x3F800000u);
+  return mul2(q, f2pack(s0, s1));
+}
+
 struct Params {
   const int4* qtiles;  // {qt, seg_begin, seg_count, n_ktiles}; entry = split * n_qt + qt
   const int2* segs;    // {kt_begin, (count << 1) | partial}
@@ -383,7 +410,14 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       for (int i = 0; i < 32; ++i) {
         float x0, x1;
         f2unpack(fma2(f2pack(s[2 * i], s[2 * i + 1]), c2v, mv), x0, x1);
-        const float e0 = ex2(x0), e1 = ex2(x1);
+        // A quarter of the pairs on the FMA pipe, the rest on MUFU.
+        float e0, e1;
+        if ((i & 3) == 3) {
+          f2unpack(ex2_fma2(x0, x1), e0, e1);
+        } else {
+          e0 = ex2(x0);
+          e1 = ex2(x1);
+        }
         if (i & 1) lb = add2(lb, f2pack(e0, e1));
         else la = add2(la, f2pack(e0, e1));
         pp[i] = pack_bf16(e0, e1);
