@@ -51,11 +51,12 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const P&
 
 // Work items reach the roles through a 4-slot ring in shared memory: the
 // producer takes the next item index from the global counter (dynamic
-// longest-first scheduling) and publishes it; the MMA thread's two cursors
-// and the eight softmax warps read it and release the slot.
-enum Role { kProducer, kConsumerThread, kConsumerWarp };
+// longest-first scheduling) and publishes it; every other role's cursor (a
+// whole warp each: the MMA warps' and the softmax warps') reads it and
+// releases the slot. Each kernel sets the slot's reader count.
+enum Role { kProducer, kConsumerWarp };  // one producer thread; consumer warps
 constexpr uint32_t kRing = 4;
-constexpr uint32_t kRingReaders = 2 + 8;  // MMA S and PV cursors, softmax warps
+constexpr uint32_t kRingReaders = 2 + 8;  // two MMA-warp cursors, eight softmax warps
 
 struct ItemRing {
   uint32_t full_bar, empty_bar;  // first slot's mbarrier; slots are 8 B apart
@@ -95,16 +96,12 @@ struct Cursor {
       mbar_arrive(r.full_bar + 8 * slot);  // release: readers see the slot
       return true;
     }
-    bool ok = wait_bar(r.full_bar + 8 * slot, use & 1u, p, r.abort_flag);
-    if (role == kConsumerWarp) ok = __all_sync(0xffffffffu, ok);
+    // A consumer is a whole warp: one arrive per warp releases the slot.
+    const bool ok = __all_sync(0xffffffffu, wait_bar(r.full_bar + 8 * slot, use & 1u, p, r.abort_flag));
     if (!ok) return false;
     item = r.slots[slot];
-    if (role == kConsumerWarp) {
-      __syncwarp();
-      if ((threadIdx.x & 31) == 0) mbar_arrive(r.empty_bar + 8 * slot);
-    } else {
-      mbar_arrive(r.empty_bar + 8 * slot);
-    }
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(r.empty_bar + 8 * slot);
     return true;
   }
   __device__ void load_item(const P& p, const ItemRing& r, Role role) {
