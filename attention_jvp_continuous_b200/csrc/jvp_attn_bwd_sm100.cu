@@ -51,8 +51,8 @@ constexpr int kThreads = 384;
 constexpr uint32_t kRHalf = BR * 128;  // 16 KB: 128 rows x 64 head-dim columns
 constexpr uint32_t kTHalf = BT * 128;  //  8 KB: 64 rows x 64 columns
 constexpr uint32_t kTile = 2 * kTHalf; // 16 KB: one streamed 64-row operand
-// Readers of the work-item ring: issuers A and B, 8 softmax warps.
-constexpr uint32_t kReaders = 2 + 8;
+// Readers of the work-item ring: issuer A's two cursors, issuer B, 8 softmax warps.
+constexpr uint32_t kReaders = 3 + 8;
 
 // Shared memory: the dK/dV pass's two stationary operands (A0, A1; the dQ
 // pass keeps its stationary Q and G in TMEM), then the streamed operands in
@@ -132,12 +132,14 @@ using Cursor = pipe::Cursor<Params>;
 // MMA issue is split over two warps (one elected lane of each issues), since
 // one lane issues at most about one tcgen05.mma per ~47 cycles while a
 // 128 x 64 x 16 MMA takes 32:
-//   issuer A (warp 1): S(t) = A0 X(t)^T and dP(t) = A1 Y(t)^T into buffer
-//                      t&1, once the accumulating MMAs of tile t-2 (same
-//                      buffer) have completed (MMAs of different warps are
-//                      ordered only through completions);
-//   issuer B (warp 2): acc(t) once the softmax warps have written tile t's
-//                      bf16 operands.
+//   issuer A (warp 1): acc(t) once the softmax warps have written tile t's
+//                      bf16 operands, then S(t+2) = A0 X(t+2)^T into the S
+//                      part of the same buffer (thread order protects it);
+//   issuer B (warp 2): dP(t) = A1 Y(t)^T into the dP part of buffer t&1,
+//                      once the softmax has read dP(t-2) from it (dQ pass)
+//                      or acc(t-2), which reads dS^T there, has completed
+//                      (dK/dV pass): MMAs of different warps are ordered
+//                      only through completions.
 // One thread's MMAs run in issue order; every hand-over between the issuers
 // and the other roles goes through an mbarrier.
 template <bool kKV>
@@ -269,21 +271,27 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       const uint64_t xm_desc = sdesc_sw128(base + LY::X, kTHalf, 1024);   // MN-major view
       const uint64_t yk_desc = sdesc_sw128(base + LY::Y, 16, 1024);
       const uint64_t ym_desc = sdesc_sw128(base + LY::Y, kTHalf, 1024);
-      // First MMAs of tile t (issuer A): S = A0 X^T or dP = A1 Y^T.
+      // First MMAs of tile t: S = A0 X^T (issuer A) or dP = A1 Y^T (issuer B).
       auto issue_first = [&](const Cursor& c, bool s_mma) -> bool {
         const uint32_t b = c.t & 1u;
         if (c.j == 0 && !wait_w(bar(B_AF), c.item_idx & 1)) return false;
         uint32_t stage;
         uint64_t bdesc;
         if (s_mma) {
-          // Buffer b last held tile t-2, whose operands acc(t-2) reads: S(t)
-          // and dP(t) wait until those MMAs (issuer B's) have completed.
-          if (c.t >= 2 && !wait_w(bar(B_MD + b), ((c.t >> 1) - 1) & 1u))
-            return false;
+          // Buffer b last held tile t-2: issuer A issued acc(t-2), which
+          // reads its S part, before this in its own order.
           stage = c.t % NX;
           if (!wait_w(bar(B_XF + stage), (c.t / NX) & 1u)) return false;
           bdesc = xk_desc + stage * (kTile >> 4);
         } else {
+          // dP(t) overwrites the dP part of buffer b. dQ pass: the softmax
+          // read dP(t-2) from it before publishing tile t-2 (acc reads only
+          // the S part there); dK/dV pass: acc(t-2) reads dS^T from it, so
+          // wait for that MMA batch (issuer A's) to complete.
+          if (c.t >= 2) {
+            const uint32_t pk = ((c.t >> 1) - 1) & 1u;
+            if (!wait_w(bar((kKV ? B_MD : B_PF) + b), pk)) return false;
+          }
           stage = c.t % NY;
           if (!wait_w(bar(B_YF + stage), (c.t / NY) & 1u)) return false;
           bdesc = yk_desc + stage * (kTile >> 4);
@@ -305,7 +313,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         if (kKV && c.j == c.n - 1) mma_commit_elect(bar(B_AE));   // done with A0 (A) / A1 (B)
         return true;
       };
-      // Accumulating MMAs (issuer B). The bf16 operands of a tile sit in
+      // Accumulating MMAs (issuer A). The bf16 operands of a tile sit in
       // TMEM columns {0, 8} and {32, 40} (one pair of 16-wide k-steps per
       // warpgroup) of the S part (and, dK/dV pass, of the dP part).
       auto issue_acc = [&](const Cursor& c) -> bool {
@@ -333,30 +341,43 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
                    first | (ks > 0));
           }
         }
-        // X(t) was also read by S(t), which completed before the softmax
-        // warps released tile t.
+        // X(t) was also read by S(t) (this thread's, earlier); Y(t) (dK/dV
+        // pass) by dP(t), which completed before the softmax warps
+        // published tile t.
         mma_commit_elect(bar(B_XE + sx));
         if (kKV) mma_commit_elect(bar(B_YE + sy));
         mma_commit_elect(bar(B_MD + b));
         return true;
       };
       bool ok = true;
-      Cursor c;
-      c.start(p, ring, kConsumerWarp);
       if (issuer_a) {
+        // acc(t), then S(t+2) in this thread's order: S(t+2) overwrites the
+        // S part of the buffer acc(t) reads. S runs up to two tiles ahead of
+        // acc but not into the next item: that item's stationary rows (dQ
+        // pass) are stored only after this item's epilogue, which waits for
+        // this item's last acc.
+        Cursor cs, ca;
+        cs.start(p, ring, kConsumerWarp);
+        ca.start(p, ring, kConsumerWarp);
         // Failure-detection test: wait on the drain barrier's first phase,
         // which nothing completes before this warp's own drain commit, so the
         // bounded wait runs out and the abort path below is taken.
         if (p.stall_test) ok = __all_sync(0xffffffffu, wait_bar(bar(B_DRAIN + 0), 0u, p, abort_flag));
-        // S(t), then dP(t): both overwrite buffer t&1 and follow acc(t-2).
-        while (c.valid && ok) {
-          ok = issue_first(c, true) && issue_first(c, false);
-          c.next(p, ring, kConsumerWarp);
+        while (ok && ca.valid) {
+          while (ok && cs.valid && cs.t < ca.t + 2 && cs.item_idx == ca.item_idx) {
+            ok = issue_first(cs, true);
+            cs.next(p, ring, kConsumerWarp);
+          }
+          if (!ok) break;
+          ok = issue_acc(ca);
+          ca.next(p, ring, kConsumerWarp);
         }
       } else {
-        // Issuer B only accumulates, so it takes P(t) as soon as it lands.
+        // dP of every tile, as soon as its buffer part is free.
+        Cursor c;
+        c.start(p, ring, kConsumerWarp);
         while (c.valid && ok) {
-          ok = issue_acc(c);
+          ok = issue_first(c, false);
           c.next(p, ring, kConsumerWarp);
         }
       }
@@ -511,8 +532,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       if (c.j == c.n - 1) {
         // ------------------------------------------------------ epilogue --
         // acc(t-2), the previous phase of this barrier, has completed:
-        // issuer A waited for it before issuing S(t) and dP(t), which this
-        // warp has seen complete.
+        // issuer A issued it before S(t), whose commit (covering all of
+        // issuer A's earlier MMAs) this warp has seen land.
         ok = wait_bar(bar(B_MD + (c.t & 1u)), (c.t >> 1) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
