@@ -90,7 +90,8 @@ enum : uint32_t {
   B_DRAIN = 29,  // 2: one per issuer
   B_IF = 31,     // 4: work-item ring
   B_IE = 35,     // 4
-  kNumBars = 39
+  B_MP = 39,     // 2: dK/dV pass: the MMAs that read a buffer's dP part complete
+  kNumBars = 41
 };
 static_assert(kNumBars <= 44, "barrier slots");
 static_assert(Layout<false>::RING + 16 <= Layout<false>::BAR + 512, "barrier area overflow");
@@ -176,6 +177,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       mbar_init(bar(B_SF + b), 2);
       mbar_init(bar(B_PF + b), 2 * BR);
       mbar_init(bar(B_MD + b), 1);
+      mbar_init(bar(B_MP + b), 1);
       mbar_init(bar(B_DRAIN + b), 1);
     }
     mbar_init(bar(B_CF), 2 * BR);
@@ -286,11 +288,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         } else {
           // dP(t) overwrites the dP part of buffer b. dQ pass: the softmax
           // read dP(t-2) from it before publishing tile t-2 (acc reads only
-          // the S part there); dK/dV pass: acc(t-2) reads dS^T from it, so
-          // wait for that MMA batch (issuer A's) to complete.
+          // the S part there); dK/dV pass: the gK MMAs of acc(t-2) read
+          // dS^T from it, so wait for them (issuer A's) to complete.
           if (c.t >= 2) {
             const uint32_t pk = ((c.t >> 1) - 1) & 1u;
-            if (!wait_w(bar((kKV ? B_MD : B_PF) + b), pk)) return false;
+            if (!wait_w(bar((kKV ? B_MP : B_PF) + b), pk)) return false;
           }
           stage = c.t % NY;
           if (!wait_w(bar(B_YF + stage), (c.t / NY) & 1u)) return false;
@@ -333,12 +335,20 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
             mma_ts_elect(tmem + TM_C0, a_p + col, xm_desc + sx * (kTile >> 4) + ((ks * 2048) >> 4),
                    IDESC_MN, first | (ks > 0));
           } else {
-            // gV += P^T G ; gK += dS^T Q
-            mma_ts_elect(tmem + TM_C0, a_p + col, ym_desc + sy * (kTile >> 4) + ((ks * 2048) >> 4),
-                   IDESC_MN, first | (ks > 0));
+            // gK += dS^T Q first: their completion frees the dP part
             mma_ts_elect(tmem + TM_C1, a_p + 64u + col,
                    xm_desc + sx * (kTile >> 4) + ((ks * 2048) >> 4), IDESC_MN,
                    first | (ks > 0));
+          }
+        }
+        if (kKV) {
+          mma_commit_elect(bar(B_MP + b));  // dP(t+2) may overwrite the dP part
+          // gV += P^T G
+#pragma unroll
+          for (int ks = 0; ks < BT / 16; ++ks) {
+            const uint32_t col = (ks >> 1) * 32u + (ks & 1) * 8u;
+            mma_ts_elect(tmem + TM_C0, a_p + col, ym_desc + sy * (kTile >> 4) + ((ks * 2048) >> 4),
+                   IDESC_MN, first | (ks > 0));
           }
         }
         // X(t) was also read by S(t) (this thread's, earlier); Y(t) (dK/dV
