@@ -51,8 +51,9 @@ constexpr int kThreads = 384;
 constexpr uint32_t kRHalf = BR * 128;  // 16 KB: 128 rows x 64 head-dim columns
 constexpr uint32_t kTHalf = BT * 128;  //  8 KB: 64 rows x 64 columns
 constexpr uint32_t kTile = 2 * kTHalf; // 16 KB: one streamed 64-row operand
-// Readers of the work-item ring: issuer A's two cursors, issuer B, 8 softmax warps.
-constexpr uint32_t kReaders = 3 + 8;
+// Readers of the work-item ring: issuer A's two cursors, issuer B's one (dQ)
+// or two (dK/dV), 8 softmax warps.
+template <bool kKV> constexpr uint32_t kReaders = (kKV ? 4 : 3) + 8;
 
 // Shared memory: the dK/dV pass's two stationary operands (A0, A1; the dQ
 // pass keeps its stationary Q and G in TMEM), then the streamed operands in
@@ -90,8 +91,7 @@ enum : uint32_t {
   B_DRAIN = 29,  // 2: one per issuer
   B_IF = 31,     // 4: work-item ring
   B_IE = 35,     // 4
-  B_MP = 39,     // 2: dK/dV pass: the MMAs that read a buffer's dP part complete
-  kNumBars = 41
+  kNumBars = 39
 };
 static_assert(kNumBars <= 44, "barrier slots");
 static_assert(Layout<false>::RING + 16 <= Layout<false>::BAR + 512, "barrier area overflow");
@@ -165,25 +165,26 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
     // dQ: the 256 softmax threads store Q / G rows and arrive; dK/dV: TMA bytes.
     mbar_init(bar(B_AF), kKV ? 1 : 2 * BR);
     mbar_init(bar(B_AE), 2);
+    // dK/dV pass: a streamed stage is released and a tile's accumulation
+    // is complete once both issuers have committed (each runs half of it).
     for (uint32_t s = 0; s < NX; ++s) {
       mbar_init(bar(B_XF + s), 1);
-      mbar_init(bar(B_XE + s), 1);
+      mbar_init(bar(B_XE + s), kKV ? 2 : 1);
     }
     for (uint32_t s = 0; s < NY; ++s) {
       mbar_init(bar(B_YF + s), 1);
-      mbar_init(bar(B_YE + s), 1);
+      mbar_init(bar(B_YE + s), kKV ? 2 : 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(B_SF + b), 2);
       mbar_init(bar(B_PF + b), 2 * BR);
-      mbar_init(bar(B_MD + b), 1);
-      mbar_init(bar(B_MP + b), 1);
+      mbar_init(bar(B_MD + b), kKV ? 2 : 1);
       mbar_init(bar(B_DRAIN + b), 1);
     }
     mbar_init(bar(B_CF), 2 * BR);
     for (uint32_t i = 0; i < kRing; ++i) {
       mbar_init(bar(B_IF + i), 1);
-      mbar_init(bar(B_IE + i), kReaders);
+      mbar_init(bar(B_IE + i), kReaders<kKV>);
     }
     *abort_flag = 0u;
     fence_mbar_init();
@@ -288,12 +289,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         } else {
           // dP(t) overwrites the dP part of buffer b. dQ pass: the softmax
           // read dP(t-2) from it before publishing tile t-2 (acc reads only
-          // the S part there); dK/dV pass: the gK MMAs of acc(t-2) read
-          // dS^T from it, so wait for them (issuer A's) to complete.
-          if (c.t >= 2) {
-            const uint32_t pk = ((c.t >> 1) - 1) & 1u;
-            if (!wait_w(bar((kKV ? B_MP : B_PF) + b), pk)) return false;
-          }
+          // the S part there). dK/dV pass: gK(t-2), which reads dS^T from
+          // it, was issued by this thread first.
+          if (!kKV && c.t >= 2 && !wait_w(bar(B_PF + b), ((c.t >> 1) - 1) & 1u))
+            return false;
           stage = c.t % NY;
           if (!wait_w(bar(B_YF + stage), (c.t / NY) & 1u)) return false;
           bdesc = yk_desc + stage * (kTile >> 4);
@@ -312,13 +311,17 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         }
         mma_commit_elect(bar(B_SF + b));
         if (!s_mma && !kKV) mma_commit_elect(bar(B_YE + stage));  // dQ pass: V feeds dP only
-        if (kKV && c.j == c.n - 1) mma_commit_elect(bar(B_AE));   // done with A0 (A) / A1 (B)
+        if (kKV && c.j == c.n - 1) mma_commit_elect(bar(B_AE));   // done with A0 (S) / A1 (dP)
         return true;
       };
-      // Accumulating MMAs (issuer A). The bf16 operands of a tile sit in
-      // TMEM columns {0, 8} and {32, 40} (one pair of 16-wide k-steps per
-      // warpgroup) of the S part (and, dK/dV pass, of the dP part).
-      auto issue_acc = [&](const Cursor& c) -> bool {
+      // Accumulating MMAs. The bf16 operands of a tile sit in TMEM columns
+      // {0, 8} and {32, 40} (one pair of 16-wide k-steps per warpgroup) of
+      // the S part (dQ pass: dS; dK/dV pass: P^T) and, dK/dV pass, of the dP
+      // part (dS^T). dQ pass: gQ += dS K, issuer A. dK/dV pass: gV += P^T G
+      // by issuer A (it reads the S part), gK += dS^T Q by issuer B (the dP
+      // part), each followed in its own thread by the first MMA that
+      // overwrites that part two tiles later.
+      auto issue_acc = [&](const Cursor& c, bool s_part) -> bool {
         const uint32_t b = c.t & 1u, sx = c.t % NX, sy = c.t % NY;
         if (c.j == 0 && c.item_idx > 0 &&
             !wait_w(bar(B_CF), (c.item_idx - 1) & 1))
@@ -326,34 +329,20 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         if (!wait_w(bar(B_PF + b), (c.t >> 1) & 1u)) return false;
         tc_fence_after();
         const uint32_t first = c.j == 0 ? 0u : 1u;
-        const uint32_t a_p = tmem + b * 128u;  // dQ pass: dS; dK/dV pass: P^T
+        const uint32_t a_p = tmem + b * 128u + (s_part ? 0u : 64u);
+        // B operand: dQ pass K (X); dK/dV pass G (Y) for gV, Q (X) for gK.
+        const uint64_t bm = (!kKV || !s_part) ? xm_desc + sx * (kTile >> 4)
+                                              : ym_desc + sy * (kTile >> 4);
+        const uint32_t acc = (!kKV || s_part) ? TM_C0 : TM_C1;
 #pragma unroll
         for (int ks = 0; ks < BT / 16; ++ks) {
           const uint32_t col = (ks >> 1) * 32u + (ks & 1) * 8u;
-          if (!kKV) {
-            // gQ += dS K
-            mma_ts_elect(tmem + TM_C0, a_p + col, xm_desc + sx * (kTile >> 4) + ((ks * 2048) >> 4),
-                   IDESC_MN, first | (ks > 0));
-          } else {
-            // gK += dS^T Q first: their completion frees the dP part
-            mma_ts_elect(tmem + TM_C1, a_p + 64u + col,
-                   xm_desc + sx * (kTile >> 4) + ((ks * 2048) >> 4), IDESC_MN,
-                   first | (ks > 0));
-          }
+          mma_ts_elect(tmem + acc, a_p + col, bm + ((ks * 2048) >> 4), IDESC_MN, first | (ks > 0));
         }
-        if (kKV) {
-          mma_commit_elect(bar(B_MP + b));  // dP(t+2) may overwrite the dP part
-          // gV += P^T G
-#pragma unroll
-          for (int ks = 0; ks < BT / 16; ++ks) {
-            const uint32_t col = (ks >> 1) * 32u + (ks & 1) * 8u;
-            mma_ts_elect(tmem + TM_C0, a_p + col, ym_desc + sy * (kTile >> 4) + ((ks * 2048) >> 4),
-                   IDESC_MN, first | (ks > 0));
-          }
-        }
-        // X(t) was also read by S(t) (this thread's, earlier); Y(t) (dK/dV
-        // pass) by dP(t), which completed before the softmax warps
-        // published tile t.
+        // Stage releases and the tile's accumulation-done: dQ pass, this
+        // thread read X(t) (also with S(t), earlier) and Y(t) only through
+        // dP(t); dK/dV pass, both issuers commit each (X and Y feed one MMA
+        // batch of each issuer: S^T and gK, dP^T and gV).
         mma_commit_elect(bar(B_XE + sx));
         if (kKV) mma_commit_elect(bar(B_YE + sy));
         mma_commit_elect(bar(B_MD + b));
@@ -379,16 +368,31 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
             cs.next(p, ring, kConsumerWarp);
           }
           if (!ok) break;
-          ok = issue_acc(ca);
+          ok = issue_acc(ca, true);
           ca.next(p, ring, kConsumerWarp);
         }
-      } else {
+      } else if (!kKV) {
         // dP of every tile, as soon as its buffer part is free.
         Cursor c;
         c.start(p, ring, kConsumerWarp);
         while (c.valid && ok) {
           ok = issue_first(c, false);
           c.next(p, ring, kConsumerWarp);
+        }
+      } else {
+        // gK(t), then dP^T(t+2) in this thread's order (it overwrites the dP
+        // part gK(t) reads), as issuer A does with the S part.
+        Cursor cd, ck;
+        cd.start(p, ring, kConsumerWarp);
+        ck.start(p, ring, kConsumerWarp);
+        while (ok && ck.valid) {
+          while (ok && cd.valid && cd.t < ck.t + 2 && cd.item_idx == ck.item_idx) {
+            ok = issue_first(cd, false);
+            cd.next(p, ring, kConsumerWarp);
+          }
+          if (!ok) break;
+          ok = issue_acc(ck, false);
+          ck.next(p, ring, kConsumerWarp);
         }
       }
       if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
