@@ -81,18 +81,20 @@ enum : uint32_t {
   B_AF = 0,      // stationary operands ready (TMA bytes, or TMEM rows stored)
   B_AE = 1,      // dK/dV: stationary smem operands may be overwritten (2 issuers)
   B_XF = 2,      // 5
-  B_XE = 7,      // 5
+  B_XE = 7,      // 5 (dK/dV pass: releases the X and the Y stage)
   B_YF = 12,     // 5
-  B_YE = 17,     // 5
-  B_SF = 22,     // 2: S and dP of a buffer complete (one commit per issuer)
-  B_PF = 24,     // 2: bf16 operands written by the softmax warps
-  B_MD = 26,     // 2: accumulating MMAs of the buffer's last tile complete
-  B_CF = 28,     // accumulators read by the epilogue
-  B_DRAIN = 29,  // 2: one per issuer
-  B_IF = 31,     // 4: work-item ring
-  B_IE = 35,     // 4
-  kNumBars = 39
+  B_YE = 17,     // 4 (dQ pass only)
+  B_SF = 21,     // 2: S and dP of a buffer complete (one commit per issuer)
+  B_PF = 23,     // 2: bf16 operands written by the softmax warps
+  B_MD = 25,     // accumulating MMAs of an item's last tile complete
+  B_CF = 26,     // accumulators read by the epilogue
+  B_DRAIN = 27,  // 2: one per issuer
+  B_IF = 29,     // 4: work-item ring
+  B_IE = 33,     // 4
+  kNumBars = 37
 };
+static_assert(Layout<false>::NY <= B_SF - B_YE, "Y-empty slots");
+static_assert(Layout<true>::NX == Layout<true>::NY, "dK/dV pass: X and Y stages pair up");
 static_assert(kNumBars <= 44, "barrier slots");
 static_assert(Layout<false>::RING + 16 <= Layout<false>::BAR + 512, "barrier area overflow");
 
@@ -165,22 +167,23 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
     // dQ: the 256 softmax threads store Q / G rows and arrive; dK/dV: TMA bytes.
     mbar_init(bar(B_AF), kKV ? 1 : 2 * BR);
     mbar_init(bar(B_AE), 2);
-    // dK/dV pass: a streamed stage is released and a tile's accumulation
-    // is complete once both issuers have committed (each runs half of it).
+    // dK/dV pass: a stage pair (Q and G of one tile) is released and an
+    // item's accumulation is complete once both issuers have committed
+    // (each runs half of the accumulation).
     for (uint32_t s = 0; s < NX; ++s) {
       mbar_init(bar(B_XF + s), 1);
       mbar_init(bar(B_XE + s), kKV ? 2 : 1);
     }
     for (uint32_t s = 0; s < NY; ++s) {
       mbar_init(bar(B_YF + s), 1);
-      mbar_init(bar(B_YE + s), kKV ? 2 : 1);
+      if (!kKV) mbar_init(bar(B_YE + s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(B_SF + b), 2);
       mbar_init(bar(B_PF + b), 2 * BR);
-      mbar_init(bar(B_MD + b), kKV ? 2 : 1);
       mbar_init(bar(B_DRAIN + b), 1);
     }
+    mbar_init(bar(B_MD), kKV ? 2 : 1);
     mbar_init(bar(B_CF), 2 * BR);
     for (uint32_t i = 0; i < kRing; ++i) {
       mbar_init(bar(B_IF + i), 1);
@@ -236,7 +239,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         tma_load_3d(base + LY::X + sx * kTile, &tm_x, bar(B_XF + sx), 0, y, c.bh);
         tma_load_3d(base + LY::X + sx * kTile + kTHalf, &tm_x, bar(B_XF + sx), 64, y, c.bh);
         const uint32_t sy = c.t % NY, uy = c.t / NY;
-        if (c.t >= NY) ok = wait_bar(bar(B_YE + sy), (uy - 1) & 1u, p, abort_flag);
+        if (!kKV && c.t >= NY) ok = wait_bar(bar(B_YE + sy), (uy - 1) & 1u, p, abort_flag);
         if (!ok) break;
         mbar_expect_tx(bar(B_YF + sy), kTile);
         ++y_issued;
@@ -339,13 +342,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
           const uint32_t col = (ks >> 1) * 32u + (ks & 1) * 8u;
           mma_ts_elect(tmem + acc, a_p + col, bm + ((ks * 2048) >> 4), IDESC_MN, first | (ks > 0));
         }
-        // Stage releases and the tile's accumulation-done: dQ pass, this
-        // thread read X(t) (also with S(t), earlier) and Y(t) only through
-        // dP(t); dK/dV pass, both issuers commit each (X and Y feed one MMA
-        // batch of each issuer: S^T and gK, dP^T and gV).
+        // Stage release: dQ pass, this thread read X(t) (also with S(t),
+        // earlier) and Y(t) only through dP(t); dK/dV pass, both issuers
+        // commit to the pair's one barrier (X and Y feed one MMA batch of
+        // each: S^T and gK, dP^T and gV). At an item's last tile, the
+        // accumulation-done the epilogue waits for.
         mma_commit_elect(bar(B_XE + sx));
-        if (kKV) mma_commit_elect(bar(B_YE + sy));
-        mma_commit_elect(bar(B_MD + b));
+        if (c.j == c.n - 1) mma_commit_elect(bar(B_MD));
         return true;
       };
       bool ok = true;
@@ -545,10 +548,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
 
       if (c.j == c.n - 1) {
         // ------------------------------------------------------ epilogue --
-        // acc(t-2), the previous phase of this barrier, has completed:
-        // issuer A issued it before S(t), whose commit (covering all of
-        // issuer A's earlier MMAs) this warp has seen land.
-        ok = wait_bar(bar(B_MD + (c.t & 1u)), (c.t >> 1) & 1u, p, abort_flag);
+        // The previous phase of this barrier (the previous item's) is the
+        // one this warp waited for in that item's epilogue; the next cannot
+        // complete before this epilogue arrives on B_CF.
+        ok = wait_bar(bar(B_MD), c.item_idx & 1, p, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
         const bool row_ok = grow < p.L;
