@@ -58,8 +58,9 @@ struct BwdArgs {
   const void *q, *k, *v, *o, *g;  // g: cotangent of o
   const float* lse;               // forward LSE
   void *gq, *gk, *gv;
-  float* scratch;                 // [B*H, Lp, 2] {LSE*log2(e), D = <g, o>} per row,
-                                  // Lp = L rounded up to a multiple of 128
+  float* scratch;                 // [B*H, Lp, 2]: per row pair, -LSE*log2(e) of both
+                                  // rows then -D = -<g, o> of both; Lp = L rounded
+                                  // up to a multiple of 128
   int B, H, L, d;
   jvp_mask_desc mask;
   float scale;

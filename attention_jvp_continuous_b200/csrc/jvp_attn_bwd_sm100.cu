@@ -118,8 +118,11 @@ struct Params {
   int Lp;  // L rounded up to whole 128-row tiles: row stride of the scratch
   float scale, c2;
   const float* lse;     // forward LSE (natural log)
-  float2* sd;           // scratch [B*H, Lp] of {LSE * log2(e), D_i = <g_i, o_i>}: written
-                        // by the dQ pass (rows past L: {+inf, 0}), read by the dK/dV pass
+  // Scratch [B*H, Lp / 2] of one float4 per row pair (2m, 2m+1):
+  // {-LSE2_2m, -LSE2_2m+1, -D_2m, -D_2m+1}, LSE2 = LSE log2(e), D_i = <g_i, o_i>;
+  // written by the dQ pass (rows past L: LSE2 = +inf, D = 0), read by the
+  // dK/dV pass as packed fp32 pairs.
+  float* sd;
   const __nv_bfloat16* q;  // dQ pass: stationary rows, stored into TMEM
   const __nv_bfloat16* g;  // cotangent: stationary rows and D (dQ pass)
   const __nv_bfloat16* o;  // forward output, for D (dQ pass)
@@ -449,7 +452,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
             dval = acc;
           }
           // grow < Lp always: the last query tile covers the padding rows.
-          if (hw == 0) p.sd[size_t(c.bh) * p.Lp + grow] = make_float2(lse2, dval);
+          if (hw == 0) {
+            float* sdp = p.sd + (size_t(c.bh) * p.Lp + (grow & ~1)) * 2 + (grow & 1);
+            sdp[0] = -lse2;
+            sdp[2] = -dval;
+          }
           // The item's stationary rows into TMEM, as bf16 pairs (the A
           // operands of the first MMAs): warpgroup 0 stores Q, warpgroup 1
           // G; rows past L are zero. The previous item's S and dP MMAs all
@@ -486,12 +493,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       // Column indices of this thread's 32 elements: keys (dQ pass) or
       // queries (dK/dV pass) [col0, col0 + 32).
       const int col0 = c.kt * BT + 32 * hw;
-      // dK/dV pass: {LSE2, D} of the 32 queries, the same for every lane
-      // (col0 + 32 <= Lp, 16-byte aligned since col0 and Lp are even).
+      // dK/dV pass: -LSE2 and -D of the 32 queries as 16 row pairs, the same
+      // for every lane (col0 + 32 <= Lp; 16-byte aligned as col0 and Lp are even).
       float4 w[16];
       if (kKV) {
         const float4* src =
-            reinterpret_cast<const float4*>(p.sd + size_t(c.bh) * p.Lp + col0);
+            reinterpret_cast<const float4*>(p.sd + (size_t(c.bh) * p.Lp + col0) * 2);
 #pragma unroll
         for (int i = 0; i < 16; ++i) w[i] = __ldg(src + i);
       }
@@ -504,37 +511,36 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       tmem_ld32(tl + b * 128u + 64u + 32u * hw, dr);
       tmem_wait_ld();
       uint32_t pp[16], pd[16];
-      // Element (2i + h): P = 2^(c2 S - LSE2), dS = P (dP - D); zero where
-      // the mask excludes the pair (only partial tiles test it).
-      auto elem = [&](int i, int h, bool masked, float& e, float& ds) {
-        const float sv = __uint_as_float(sr[2 * i + h]);
-        const float dp = __uint_as_float(dr[2 * i + h]);
-        const float l2 = kKV ? (h ? w[i].z : w[i].x) : lse2;
-        const float dd = kKV ? (h ? w[i].w : w[i].y) : dval;
-        const float pe = ex2(fmaf(sv, p.c2, -l2));
-        const float dsv = pe * (dp - dd);
-        const bool keep = !masked || key_ok(rk, col0 + 2 * i + h);
-        e = keep ? pe : 0.f;
-        ds = keep ? dsv : 0.f;
+      // Elements (2i, 2i+1) as one packed fp32 pair: P = 2^(c2 S - LSE2),
+      // dS = P (dP - D), each rounded as the scalar expression would be;
+      // zero where the mask excludes the pair (only partial tiles test it).
+      const uint64_t c2v = f2pack(p.c2, p.c2);
+      const uint64_t nl_row = f2pack(-lse2, -lse2), nd_row = f2pack(-dval, -dval);  // dQ pass
+      auto pair = [&](int i, bool masked) {
+        const uint64_t nl = kKV ? f2pack(w[i].x, w[i].y) : nl_row;
+        const uint64_t nd = kKV ? f2pack(w[i].z, w[i].w) : nd_row;
+        float x0, x1, e0, e1, d0, d1;
+        f2unpack(fma2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), c2v, nl),
+                 x0, x1);
+        e0 = ex2(x0);
+        e1 = ex2(x1);
+        const uint64_t dsv =
+            mul2(f2pack(e0, e1),
+                 add2(f2pack(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1])), nd));
+        f2unpack(dsv, d0, d1);
+        if (masked) {
+          if (!key_ok(rk, col0 + 2 * i)) e0 = d0 = 0.f;
+          if (!key_ok(rk, col0 + 2 * i + 1)) e1 = d1 = 0.f;
+        }
+        pp[i] = pack_bf16(e0, e1);
+        pd[i] = pack_bf16(d0, d1);
       };
       if (c.partial) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float e0, e1, d0, d1;
-          elem(i, 0, true, e0, d0);
-          elem(i, 1, true, e1, d1);
-          pp[i] = pack_bf16(e0, e1);
-          pd[i] = pack_bf16(d0, d1);
-        }
+        for (int i = 0; i < 16; ++i) pair(i, true);
       } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float e0, e1, d0, d1;
-          elem(i, 0, false, e0, d0);
-          elem(i, 1, false, e1, d1);
-          pp[i] = pack_bf16(e0, e1);
-          pd[i] = pack_bf16(d0, d1);
-        }
+        for (int i = 0; i < 16; ++i) pair(i, false);
       }
       if (!kKV) {
         tmem_st16(tl + b * 128u + 32u * hw, pd);  // dS over this warpgroup's S columns
@@ -652,7 +658,7 @@ static int launch_pass(const BwdArgs& a, const WorkList& w, int num_sms, unsigne
   p.c2 = a.scale * 1.4426950408889634f;
   p.lse = a.lse;
   p.Lp = (a.L + 127) / 128 * 128;
-  p.sd = reinterpret_cast<float2*>(a.scratch);
+  p.sd = a.scratch;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.g = static_cast<const __nv_bfloat16*>(a.g);
   p.o = static_cast<const __nv_bfloat16*>(a.o);
