@@ -305,14 +305,18 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         }
         tc_fence_after();
         const uint32_t d = tmem + b * 128u + (s_mma ? 0u : 64u);
+        // k-steps 4h .. 4h+3 (head-dim columns [64 h, 64 h + 64), one
+        // swizzled half of each operand), four MMAs per elect.
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ob = ((kk >> 2) * kTHalf + (kk & 3) * 32) >> 4;
+        for (int h = 0; h < D / 64; ++h) {
+          const uint64_t bh = bdesc + ((h * kTHalf) >> 4);
           if (!kKV) {
-            mma_ts_elect(d, tmem + (s_mma ? TM_QA : TM_GA) + 8u * kk, bdesc + ob, IDESC_N64, kk > 0);
+            const uint32_t ah = tmem + (s_mma ? TM_QA : TM_GA) + 32u * h;
+            mma_ts4_elect(d, ah, ah + 8u, ah + 16u, ah + 24u, bh, bh + 2, bh + 4, bh + 6, IDESC_N64,
+                          h > 0);
           } else {
-            const uint32_t oa = ((kk >> 2) * kRHalf + (kk & 3) * 32) >> 4;
-            mma_ss_elect(d, (s_mma ? a0_desc : a1_desc) + oa, bdesc + ob, IDESC_N64, kk > 0);
+            const uint64_t ah = (s_mma ? a0_desc : a1_desc) + ((h * kRHalf) >> 4);
+            mma_ss4_elect(d, ah, ah + 2, ah + 4, ah + 6, bh, bh + 2, bh + 4, bh + 6, IDESC_N64, h > 0);
           }
         }
         mma_commit_elect(bar(B_SF + b));
@@ -340,11 +344,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         const uint64_t bm = (!kKV || !s_part) ? xm_desc + sx * (kTile >> 4)
                                               : ym_desc + sy * (kTile >> 4);
         const uint32_t acc = (!kKV || s_part) ? TM_C0 : TM_C1;
-#pragma unroll
-        for (int ks = 0; ks < BT / 16; ++ks) {
-          const uint32_t col = (ks >> 1) * 32u + (ks & 1) * 8u;
-          mma_ts_elect(tmem + acc, a_p + col, bm + ((ks * 2048) >> 4), IDESC_MN, first | (ks > 0));
-        }
+        // k-steps 0..3: TMEM columns {0, 8, 32, 40}; B rows 16 ks.
+        static_assert(BT == 64, "four accumulating k-steps per tile");
+        mma_ts4_elect(tmem + acc, a_p, a_p + 8u, a_p + 32u, a_p + 40u, bm, bm + 128, bm + 256,
+                      bm + 384, IDESC_MN, first);
         // Stage release: dQ pass, this thread read X(t) (also with S(t),
         // earlier) and Y(t) only through dP(t); dK/dV pass, both issuers
         // commit to the pair's one barrier (X and Y feed one MMA batch of
