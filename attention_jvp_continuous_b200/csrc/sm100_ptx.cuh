@@ -136,43 +136,6 @@ __device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, u
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// Four MMAs into one accumulator behind a single elect.sync: the whole warp
-// runs the block, the elected lane issues all four (in order). acc0 is the
-// first one's enable-input-d; the other three accumulate.
-__device__ __forceinline__ void mma_ts4_elect(uint32_t d_tmem, uint32_t a0, uint32_t a1,
-                                              uint32_t a2, uint32_t a3, uint64_t b0, uint64_t b1,
-                                              uint64_t b2, uint64_t b3, uint32_t idesc,
-                                              uint32_t acc0) {
-  asm volatile(
-      "{\n\t.reg .pred e, p, q;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %10, 0;\n\t"
-      "setp.ne.b32 q, %11, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %5, %9, p;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %9, q;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %9, q;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %9, q;\n\t}" ::"r"(d_tmem),
-      "r"(a0), "r"(a1), "r"(a2), "r"(a3), "l"(b0), "l"(b1), "l"(b2), "l"(b3), "r"(idesc),
-      "r"(acc0), "r"(1u)
-      : "memory");
-}
-__device__ __forceinline__ void mma_ss4_elect(uint32_t d_tmem, uint64_t a0, uint64_t a1,
-                                              uint64_t a2, uint64_t a3, uint64_t b0, uint64_t b1,
-                                              uint64_t b2, uint64_t b3, uint32_t idesc,
-                                              uint32_t acc0) {
-  asm volatile(
-      "{\n\t.reg .pred e, p, q;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %10, 0;\n\t"
-      "setp.ne.b32 q, %11, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %5, %9, p;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %9, q;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %9, q;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %9, q;\n\t}" ::"r"(d_tmem),
-      "l"(a0), "l"(a1), "l"(a2), "l"(a3), "l"(b0), "l"(b1), "l"(b2), "l"(b3), "r"(idesc),
-      "r"(acc0), "r"(1u)
-      : "memory");
-}
 __device__ __forceinline__ void mma_commit_elect(uint32_t bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
