@@ -173,6 +173,18 @@ struct Params {
 };
 using Cursor = pipe::Cursor<Params>;
 
+// Ring stage of a cursor's tile t and the parity of its use, kept in step
+// with the cursor (t % N and (t / N) & 1 without the division).
+struct Stage {
+  uint32_t s = 0, ph = 0;
+  __device__ void step(uint32_t n) {
+    if (++s == n) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+};
+
 // MMA issue is split over two warps (one elected lane of each issues), since
 // one lane issues at most about one tcgen05.mma per ~47 cycles while a
 // 128 x 64 x 16 MMA takes 32:
@@ -319,7 +331,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       const uint64_t yk_desc = sdesc_sw128(base + LY::Y, 16, 1024);
       const uint64_t ym_desc = sdesc_sw128(base + LY::Y, kTHalf, 1024);
       // First MMAs of tile t: S = A0 X^T (issuer A) or dP = A1 Y^T (issuer B).
-      auto issue_first = [&](const Cursor& c, bool s_mma) -> bool {
+      auto issue_first = [&](const Cursor& c, bool s_mma, const Stage& st) -> bool {
         const uint32_t b = c.t & 1u;
         if (c.j == 0 && !wait_w(bar(B_AF), c.item_idx & 1)) return false;
         uint32_t stage;
@@ -327,8 +339,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         if (s_mma) {
           // Buffer b last held tile t-2: issuer A issued acc(t-2), which
           // reads its S part, before this in its own order.
-          stage = c.t % NX;
-          if (!wait_w(bar(B_XF + stage), (c.t / NX) & 1u)) return false;
+          stage = st.s;
+          if (!wait_w(bar(B_XF + stage), st.ph)) return false;
           bdesc = xk_desc + stage * (kTile >> 4);
         } else {
           // dP(t) overwrites the dP part of buffer b. dQ pass: the softmax
@@ -337,8 +349,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
           // it, was issued by this thread first.
           if (!kKV && c.t >= 2 && !wait_w(bar(B_PF + b), ((c.t >> 1) - 1) & 1u))
             return false;
-          stage = c.t % NY;
-          if (!wait_w(bar(B_YF + stage), (c.t / NY) & 1u)) return false;
+          stage = st.s;
+          if (!wait_w(bar(B_YF + stage), st.ph)) return false;
           bdesc = yk_desc + stage * (kTile >> 4);
         }
         tc_fence_after();
@@ -369,8 +381,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       // by issuer A (it reads the S part), gK += dS^T Q by issuer B (the dP
       // part), each followed in its own thread by the first MMA that
       // overwrites that part two tiles later.
-      auto issue_acc = [&](const Cursor& c, bool s_part) -> bool {
-        const uint32_t b = c.t & 1u, sx = c.t % NX, sy = c.t % NY;
+      auto issue_acc = [&](const Cursor& c, bool s_part, const Stage& st) -> bool {
+        // X stage of tile t; in the dK/dV pass (NX == NY) also its Y stage.
+        const uint32_t b = c.t & 1u, sx = st.s, sy = st.s;
         if (c.j == 0 && c.item_idx > 0 &&
             !wait_w(bar(B_CF), (c.item_idx - 1) & 1))
           return false;
@@ -403,6 +416,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         // pass) are stored only after this item's epilogue, which waits for
         // this item's last acc.
         Cursor cs, ca;
+        Stage ss, sa;  // X stages of cs.t and ca.t
         cs.start(p, ring, kConsumerWarp);
         ca.start(p, ring, kConsumerWarp);
         // Failure-detection test: wait on the drain barrier's first phase,
@@ -411,35 +425,42 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         if (p.stall_test) ok = __all_sync(0xffffffffu, wait_bar(bar(B_DRAIN + 0), 0u, p, abort_flag));
         while (ok && ca.valid) {
           while (ok && cs.valid && cs.t < ca.t + 2 && cs.item_idx == ca.item_idx) {
-            ok = issue_first(cs, true);
+            ok = issue_first(cs, true, ss);
             cs.next(p, ring, kConsumerWarp);
+            ss.step(NX);
           }
           if (!ok) break;
-          ok = issue_acc(ca, true);
+          ok = issue_acc(ca, true, sa);
           ca.next(p, ring, kConsumerWarp);
+          sa.step(NX);
         }
       } else if (!kKV) {
         // dP of every tile, as soon as its buffer part is free.
         Cursor c;
+        Stage sc;  // Y stage of c.t
         c.start(p, ring, kConsumerWarp);
         while (c.valid && ok) {
-          ok = issue_first(c, false);
+          ok = issue_first(c, false, sc);
           c.next(p, ring, kConsumerWarp);
+          sc.step(NY);
         }
       } else {
         // gK(t), then dP^T(t+2) in this thread's order (it overwrites the dP
         // part gK(t) reads), as issuer A does with the S part.
         Cursor cd, ck;
+        Stage sd, sk;  // stages (X and Y alike) of cd.t and ck.t
         cd.start(p, ring, kConsumerWarp);
         ck.start(p, ring, kConsumerWarp);
         while (ok && ck.valid) {
           while (ok && cd.valid && cd.t < ck.t + 2 && cd.item_idx == ck.item_idx) {
-            ok = issue_first(cd, false);
+            ok = issue_first(cd, false, sd);
             cd.next(p, ring, kConsumerWarp);
+            sd.step(NY);
           }
           if (!ok) break;
-          ok = issue_acc(ck, false);
+          ok = issue_acc(ck, false, sk);
           ck.next(p, ring, kConsumerWarp);
+          sk.step(NX);
         }
       }
       if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
