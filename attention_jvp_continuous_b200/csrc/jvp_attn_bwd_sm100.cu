@@ -10,14 +10,16 @@
 //                               A operands, K and V tiles from shared memory)
 //      softmax warps: P, dS    (one row per thread, bf16 dS back to TMEM)
 //      gQ += dS K              (A = dS in TMEM, N = 128, accumulator in TMEM)
-//    and it writes {LSE, D_i} per row to a scratch vector for the second pass.
+//    and it writes -LSE2 and -D_i per row pair to a scratch vector for the
+//    second pass.
 //  * dK/dV pass (key-stationary, 128 keys per item, 64-query tiles):
 //      S^T = K Q^T, dP^T = V G^T (both operands in shared memory: TMEM holds
 //                               the two accumulators and the S/dP buffers)
 //      softmax warps: P^T, dS^T (one key per thread; per-query LSE and D)
 //      gV += P^T G, gK += dS^T Q (A in TMEM, N = 128)
-// Warp roles: warp 0 TMA, warps 1 and 2 issue MMAs (one thread each),
-// warps 4-11 two warpgroups taking 32 of each tile's 64 columns. Each
+// Warp roles: warp 0 TMA, warps 1 and 2 issue MMAs (whole warps, one
+// elected lane issuing), warps 4-11 two warpgroups taking 32 of each tile's
+// 64 columns. Each
 // warpgroup writes its bf16 operands into the TMEM columns it has just read
 // itself, so no exchange between the warpgroups is needed.
 #include <cuda.h>
@@ -187,15 +189,15 @@ struct Stage {
 
 // MMA issue is split over two warps (one elected lane of each issues), since
 // one lane issues at most about one tcgen05.mma per ~47 cycles while a
-// 128 x 64 x 16 MMA takes 32:
-//   issuer A (warp 1): acc(t) once the softmax warps have written tile t's
-//                      bf16 operands, then S(t+2) = A0 X(t+2)^T into the S
-//                      part of the same buffer (thread order protects it);
-//   issuer B (warp 2): dP(t) = A1 Y(t)^T into the dP part of buffer t&1,
-//                      once the softmax has read dP(t-2) from it (dQ pass)
-//                      or acc(t-2), which reads dS^T there, has completed
-//                      (dK/dV pass): MMAs of different warps are ordered
-//                      only through completions.
+// 128 x 64 x 16 MMA takes 32. MMAs of different warps are ordered only
+// through completions, so the warp that reads a TMEM part in tile t's
+// accumulating MMAs is the one that overwrites it at tile t+2:
+//   dQ pass:    issuer A (warp 1): gQ(t) once the softmax warps have written
+//               tile t's dS into the S part, then S(t+2) = A0 X(t+2)^T into
+//               that part; issuer B (warp 2): dP(t) = A1 Y(t)^T into the dP
+//               part of buffer t&1 once the softmax has read dP(t-2) there.
+//   dK/dV pass: issuer A: gV(t) (P^T, S part) then S^T(t+2); issuer B:
+//               gK(t) (dS^T, dP part) then dP^T(t+2).
 // One thread's MMAs run in issue order; every hand-over between the issuers
 // and the other roles goes through an mbarrier.
 template <bool kKV>

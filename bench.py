@@ -42,6 +42,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -86,11 +87,31 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+_TOKEN = re.compile(r'"(?:\\.|[^"\\\n])*"'       # string literal
+                    r"|'(?:\\.|[^'\\\n])*'"       # character literal
+                    r"|//[^\n]*"                     # line comment
+                    r"|/\*.*?\*/"                    # block comment
+                    r"|\s+", re.S)
+
+
+def code_only(src: str) -> str:
+    """C/C++ source without comments, with every run of whitespace as one
+    space: what a comment or layout edit leaves unchanged."""
+    def keep(m):
+        t = m.group(0)
+        if t.startswith("//") or t.startswith("/*"):
+            return " "
+        return " " if t.isspace() else t
+    return re.sub(r"\s+", " ", _TOKEN.sub(keep, src)).strip()
+
+
 def kernel_hash(op: str = "jvp") -> str:
+    """Hash of the code (comments and layout aside) of the sources that make
+    up one op's kernels: a stored ncu figure is used only while it matches."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES[op]:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            h.update(code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -26,6 +26,14 @@ def test_kernel_hash_is_per_op_and_stable(bench):
     assert all(bench.kernel_hash(op) == h for op, h in hashes.items())
 
 
+def test_kernel_hash_ignores_comments_and_layout_only(bench):
+    src = 'int f(int a) {  // first\n  return a + 1; /* "x" */\n}\nconst char* s = "// kept";\n'
+    assert bench.code_only(src) == bench.code_only(
+        'int f(int a) {\n    return a + 1;\n}  // other words\nconst char* s = "// kept";')
+    assert bench.code_only(src) != bench.code_only(src.replace("a + 1", "a + 2"))
+    assert bench.code_only(src) != bench.code_only(src.replace('"// kept"', '"// gone"'))
+
+
 def test_stored_traffic_requires_matching_source_and_shape(bench, tmp_path, monkeypatch):
     path = tmp_path / "traffic.json"
     path.write_text(json.dumps({
