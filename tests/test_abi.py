@@ -156,6 +156,42 @@ def test_rope_copy_argument_errors(kw, code):
     assert call_rope(**kw) == code
 
 
+def call_bwd(B=1, H=2, L=64, d=128, dtype=_lib.JVP_BF16, mask=(ja.TEACHER_FORCING, 8, 4, 1),
+             scale=0.0, scratch_len=None, ptrs=None):
+    p = [FAKE] * 10 if ptrs is None else ptrs
+    if scratch_len is None:
+        scratch_len = max(_lib.lib().jvp_attn_bwd_scratch_len(B, H, L), 0)
+    fp = ctypes.POINTER(ctypes.c_float)
+    vp = [ctypes.c_void_p(x) for x in p]
+    return _lib.lib().jvp_attn_bwd(*vp[:5], ctypes.cast(vp[5], fp), *vp[6:9],
+                                   ctypes.cast(vp[9], fp), scratch_len, B, H, L, d, dtype,
+                                   _lib.MaskDesc(*mask), scale, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ptrs=[FAKE] * 9 + [0]), _lib.JVP_ERR_INVALID_ARG),            # no scratch
+    (dict(ptrs=[FAKE] * 5 + [0] + [FAKE] * 4), _lib.JVP_ERR_INVALID_ARG),  # no lse
+    (dict(L=0), _lib.JVP_ERR_INVALID_ARG),
+    (dict(dtype=_lib.JVP_FP32), _lib.JVP_ERR_INVALID_ARG),               # bf16 only
+    (dict(scale=float("inf")), _lib.JVP_ERR_INVALID_ARG),
+    (dict(d=64), _lib.JVP_ERR_UNSUPPORTED_HEAD_DIM),
+    (dict(L=63), _lib.JVP_ERR_SHAPE_MISMATCH),                           # mask covers 64
+    (dict(mask=(9, 8, 4, 1)), _lib.JVP_ERR_INVALID_ARG),
+    (dict(B=70000, H=70000), _lib.JVP_ERR_TOO_LARGE),
+    (dict(scratch_len=2 * 2 * 128 - 1), _lib.JVP_ERR_INVALID_ARG),      # one float short
+    (dict(ptrs=[FAKE] * 6 + [FAKE + 8] + [FAKE] * 3), _lib.JVP_ERR_MISALIGNED),
+])
+def test_bwd_argument_errors(kw, code):
+    assert call_bwd(**kw) == code
+
+
+def test_bwd_valid_call_without_gpu_fails_cleanly():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert call_bwd() in (_lib.JVP_ERR_LAUNCH_FAILED, _lib.JVP_ERR_UNSUPPORTED_DEVICE)
+
+
 def test_bwd_scratch_len():
     assert _lib.lib().jvp_attn_bwd_scratch_len(1, 12, 65520) == 2 * 12 * 65536
     assert _lib.lib().jvp_attn_bwd_scratch_len(2, 3, 1) == 2 * 6 * 128
