@@ -80,6 +80,30 @@ def test_argument_errors(kw, code):
     assert call_fwd(**kw) == code
 
 
+def call_fwd_noalloc(ptr=0x1000, B=1, H=1, L=64, d=128, dtype=_lib.JVP_BF16,
+                     mask=(ja.TEACHER_FORCING, 8, 4, 1), scale=0.0):
+    return _lib.lib().jvp_attn_fwd_noalloc(
+        *[ctypes.c_void_p(ptr) for _ in range(8)],
+        ctypes.cast(ctypes.c_void_p(ptr), ctypes.POINTER(ctypes.c_float)),
+        B, H, L, d, dtype, _lib.MaskDesc(*mask), scale, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ptr=0), _lib.JVP_ERR_INVALID_ARG),
+    (dict(B=0), _lib.JVP_ERR_INVALID_ARG),
+    (dict(dtype=_lib.JVP_FP32), _lib.JVP_ERR_INVALID_ARG),       # tensor-core configuration only
+    (dict(d=64), _lib.JVP_ERR_UNSUPPORTED_HEAD_DIM),
+    (dict(scale=float("nan")), _lib.JVP_ERR_INVALID_ARG),
+    (dict(L=63), _lib.JVP_ERR_SHAPE_MISMATCH),
+    (dict(ptr=0x1008), _lib.JVP_ERR_MISALIGNED),
+    (dict(B=70000, H=70000), _lib.JVP_ERR_TOO_LARGE),
+    # a work list larger than the fixed array: rejected before any device work
+    (dict(L=4096 * 513, mask=(ja.DENSE, 4096, 513, 1)), _lib.JVP_ERR_TOO_LARGE),
+])
+def test_noalloc_argument_errors(kw, code):
+    assert call_fwd_noalloc(**kw) == code
+
+
 def test_valid_call_without_gpu_fails_cleanly():
     import torch
     if torch.cuda.is_available():
