@@ -14,7 +14,8 @@ SRC = os.path.join(os.path.dirname(__file__), "..", "attention_jvp_continuous_b2
 
 
 def _constants():
-    src = open(SRC).read()
+    with open(SRC) as f:
+        src = f.read()
     body = src[src.index("uint64_t ex2_fma2("):]
     body = body[:body.index("\n}\n")]
     shift = float(re.search(r"kShift = ([0-9.]+)f", body).group(1))

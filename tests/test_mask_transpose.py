@@ -46,7 +46,8 @@ def test_key_queries_is_transpose_of_row_keys():
     with tempfile.TemporaryDirectory() as d:
         src = os.path.join(d, "t.cpp")
         exe = os.path.join(d, "t")
-        open(src, "w").write(PROGRAM)
+        with open(src, "w") as f:
+            f.write(PROGRAM)
         subprocess.run([gxx, "-std=c++17", "-O1", "-I", CSRC, src, "-o", exe], check=True)
         out = subprocess.run([exe], capture_output=True, text=True)
         assert out.returncode == 0, out.stdout

@@ -68,7 +68,8 @@ def test_dense_split_schedule():
     with tempfile.TemporaryDirectory() as d:
         src = os.path.join(d, "t.cpp")
         exe = os.path.join(d, "t")
-        open(src, "w").write(PROGRAM)
+        with open(src, "w") as f:
+            f.write(PROGRAM)
         subprocess.run([gxx, "-std=c++17", "-O1", "-I", CSRC, src,
                         os.path.join(CSRC, "schedule.cpp"), "-o", exe], check=True)
         out = subprocess.run([exe], capture_output=True, text=True)
