@@ -46,6 +46,7 @@ import re
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -165,7 +166,10 @@ class ClockSampler:
     def __init__(self, bus_id: str | None):
         self.bus_id = (bus_id or "").lower()
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        # The raw samples go to BENCH_CLOCK_DIR (default: the system temp
+        # directory); the JSON line carries their summary.
+        log_dir = os.environ.get("BENCH_CLOCK_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(log_dir, f"clocks_{os.getpid()}.csv")
 
     @staticmethod
     def bus_id_of(props) -> str | None:
