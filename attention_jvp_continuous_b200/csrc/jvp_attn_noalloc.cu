@@ -81,6 +81,17 @@ extern "C" int jvp_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   if (dev < 0 || dev >= kMaxDevices) return JVP_ERR_UNSUPPORTED_DEVICE;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The cached (mask, L) key below lives on the host. A call recorded into
+  // a graph on a cache hit would bake in the list sizes of that moment and
+  // replay against whatever list a later call left in the array, so calls
+  // on a capturing stream are refused. A failed query (e.g. the legacy
+  // stream while another stream captures globally) is refused too.
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) {
+    cudaGetLastError();
+    return JVP_ERR_INVALID_ARG;
+  }
+  if (cap != cudaStreamCaptureStatusNone) return JVP_ERR_INVALID_ARG;
   WorkList w;
   unsigned* counter = nullptr;
   {

@@ -185,8 +185,11 @@ int jvp_attn_fwd_scatter(const void* q, const void* k, const void* v,
  * device work.
  *
  * The first call on a device looks the array's address up
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture. The array holds the kernel's work-item counter
+ * (cudaGetSymbolAddress) with that device current. The entry point must not
+ * be called while `stream` is capturing (it returns JVP_ERR_INVALID_ARG
+ * then): which list the array holds is tracked on the host, so a recorded
+ * call would replay against whatever list a later call left there. The
+ * array holds the kernel's work-item counter
  * (its first 64 words, cleared on `stream` before every launch) and the work
  * list (the rest). A call whose (mask, L) differs from the list the array
  * holds rewrites the list with an asynchronous copy on `stream`; every word

@@ -73,3 +73,43 @@ def test_noalloc_rejects_oversized_work_list():
         ctypes.cast(ctypes.c_void_p(fake[8]), ctypes.POINTER(ctypes.c_float)),
         1, 1, 4096 * 513, 128, _lib.JVP_BF16, _lib.MaskDesc(ja.DENSE, 4096, 513, 1), 0.0, None)
     assert rc == _lib.JVP_ERR_TOO_LARGE
+
+
+def _outputs_of(fn, ins, w):
+    o, do = torch.empty_like(ins[0]), torch.empty_like(ins[0])
+    lse = torch.empty(ins[0].shape[:3], dtype=torch.float32, device="cuda")
+    assert call(fn, *ins, o, do, lse, w) == 0
+    ja.check_device_error()
+    return o, do, lse
+
+
+def test_noalloc_list_kept_and_rewritten_across_masks():
+    # Mask A, then B (longer, so its list overwrites more of the shared
+    # array), then A twice: the third call must rewrite A's list, the fourth
+    # reuses it without a copy. Every call is checked against jvp_attn_fwd.
+    lib = _lib.lib()
+    wa = Workload("na_a", 1, 2, 128, ja.TEACHER_FORCING, 120, 3, 1, "bf16", 0.1)
+    wb = Workload("na_b", 1, 2, 128, ja.FRAME_CAUSAL, 300, 5, 1, "bf16", 0.1)
+    ins = {w.name: make_inputs(w, device="cuda")[0] for w in (wa, wb)}
+    ref = {w.name: _outputs_of(lib.jvp_attn_fwd, ins[w.name], w) for w in (wa, wb)}
+    for w in (wa, wb, wa, wa):
+        o, do, lse = _outputs_of(lib.jvp_attn_fwd_noalloc, ins[w.name], w)
+        o1, do1, l1 = ref[w.name]
+        close(o, o1)
+        close(do, do1)
+        assert (lse - l1).abs().max().item() <= 1e-3
+
+
+def test_noalloc_refuses_a_capturing_stream():
+    lib = _lib.lib()
+    w = Workload("na_cap", 1, 1, 128, ja.TEACHER_FORCING, 64, 2, 1, "bf16", 0.1)
+    ins, _ = make_inputs(w, device="cuda")
+    o, do, lse = _outputs_of(lib.jvp_attn_fwd_noalloc, ins, w)  # first call: set-up
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=torch.cuda.Stream()):
+        rc = call(lib.jvp_attn_fwd_noalloc, *ins, o, do, lse, w)
+    assert rc == _lib.JVP_ERR_INVALID_ARG
+    # nothing was recorded or left pending: a plain call still works
+    o2, do2, l2 = _outputs_of(lib.jvp_attn_fwd_noalloc, ins, w)
+    assert torch.equal(o2, o) and torch.equal(do2, do) and torch.equal(l2, lse)
+
