@@ -343,3 +343,28 @@ def test_head_function_rejects_length_mismatch():
     x = np.zeros((15, 8))
     with pytest.raises(ValueError):
         jvp_attention_head(x, x, x, x, x, x, spec)
+
+
+def test_fully_masked_row_convention(monkeypatch):
+    # No descriptor of the four modes leaves a query row without keys, so
+    # the oracle's empty-row branch is reached by injecting an empty key
+    # set for some rows. Their O and dO are sums over no keys (zero) and
+    # their LSE is the log-sum-exp of no scores, which torch gives as -inf;
+    # every other row must be exactly what the unmodified mask gives.
+    import sys
+    oj = sys.modules["oracle.jvp_attention"]  # the package re-exports a function of that name
+    spec = MaskSpec(TEACHER_FORCING, 4, 3, 1)
+    q, k, v, dq, dk, dv = rand_inputs(21, 1, 2, spec.length, 8)
+    ref = jvp_attention(q, k, v, dq, dk, dv, spec)
+    empty = {0, 5, 13, 20}
+    real = oj.key_intervals
+    monkeypatch.setattr(oj, "key_intervals",
+                        lambda s, i: [] if i in empty else real(s, i))
+    o, do, lse = jvp_attention(q, k, v, dq, dk, dv, spec)
+    rows = sorted(empty)
+    others = [i for i in range(spec.length) if i not in empty]
+    assert np.all(o[:, :, rows] == 0) and np.all(do[:, :, rows] == 0)
+    lse_empty = torch.logsumexp(torch.full((3,), float("-inf"), dtype=torch.float64), 0)
+    assert np.all(lse[:, :, rows] == lse_empty.item())
+    for a, b in zip((o, do, lse), ref):
+        np.testing.assert_array_equal(a[:, :, others], b[:, :, others])

@@ -140,3 +140,27 @@ def test_backward_row_subsets_partition():
             a += x
     for a, x in zip(acc, full):
         np.testing.assert_allclose(a, x, atol=1e-12)
+
+
+def test_fully_masked_row_contributes_nothing(monkeypatch):
+    # A query row without keys (injected: no descriptor of the four modes
+    # has one) has O = 0 whatever q, k, v are, so its cotangent reaches
+    # nothing: the gradients equal those of the unmodified mask with that
+    # row's cotangent set to zero, and its own query gradient is zero.
+    import sys
+    ob = sys.modules["oracle.attention_backward"]
+    oj = sys.modules["oracle.jvp_attention"]  # the package re-exports a function of that name
+    spec = MaskSpec(TEACHER_FORCING, 4, 3, 1)
+    q, k, v, g = rand(31, 1, 2, spec.length, 8)
+    empty = [2, 9, 17]
+    g0 = g.clone()
+    g0[:, :, empty] = 0
+    ref = attention_backward(q, k, v, g0, spec)
+    real = oj.key_intervals
+    monkeypatch.setattr(oj, "key_intervals",
+                        lambda s, i: [] if i in empty else real(s, i))
+    assert ob._group_rows is oj._group_rows
+    got = attention_backward(q, k, v, g, spec)
+    assert np.all(got[0][:, :, empty] == 0)
+    for a, b in zip(got, ref):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
