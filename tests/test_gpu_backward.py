@@ -72,6 +72,73 @@ def test_backward_matches_oracle(w):
         compare(got, want, name)
 
 
+@pytest.mark.parametrize("w", [
+    # 2 x 32 heads x 5 query tiles (and 5 key tiles) = 320 work items per
+    # pass, more than the 148 SMs: persistent CTAs carry over from one item
+    # to the next in both passes. 600 tokens end in a ragged 88-row tile.
+    Workload("bwd_many_items_tf", 2, 32, 128, ja.TEACHER_FORCING, 100, 3, 1, "bf16", 1.0),
+    Workload("bwd_many_items_chunk", 2, 40, 128, ja.CHUNK_CAUSAL, 90, 6, 2, "bf16", 1.0),
+], ids=lambda w: w.name)
+def test_backward_more_items_than_sms(w):
+    n_items = w.B * w.H * -(-w.L // 128)
+    assert n_items > 148
+    (q, k, v, g, _, _), _ = make_inputs(w, device="cpu")
+    spec = MaskSpec(w.mode, w.tokens_per_frame, w.n_frames, w.chunk)
+    ref = attention_backward(q, k, v, g, spec)
+    _, _, grads = forward_and_backward(w, *(t.cuda() for t in (q, k, v, g)))
+    for name, got, want in zip(("gQ", "gK", "gV"), grads, ref):
+        compare(got, want, name)
+
+
+def parity_rows(w, n_random=96):
+    """Seeded random query rows plus the mask's frame, half and tile edges."""
+    L, T, F = w.L, w.tokens_per_frame, w.n_frames
+    rng = np.random.default_rng(1234)
+    rows = set(rng.choice(L, size=n_random, replace=False).tolist())
+    FT = T * F
+    for base in ([0, FT] if w.mode == ja.TEACHER_FORCING else [0]):
+        for f in (0, 1, F // 2, F - 1):
+            rows.update({base + f * T, base + f * T + T - 1})
+    rows.update({L - 1, L - 2, 127, 128})
+    return np.array(sorted(r for r in rows if 0 <= r < L))
+
+
+def full_size_case(name):
+    w = WORKLOADS[name]
+    (q, k, v, _, _, _), _ = make_inputs(w, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(99)
+    g = torch.randn(q.shape, generator=gen, device="cuda").to(q.dtype)
+    _, _, grads = forward_and_backward(w, q, k, v, g)
+    spec = MaskSpec(w.mode, w.tokens_per_frame, w.n_frames, w.chunk)
+    return w, spec, (q, k, v, g), grads
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["tf", "chunk_tf"])
+def test_full_size_gq_on_sampled_rows(name):
+    # The launch the backward bench times (all heads, full length); gQ of a
+    # row depends only on that row's cotangent, so the oracle restricted to
+    # the sampled rows gives gQ exactly there.
+    w, spec, ins, (gq, _, _) = full_size_case(name)
+    rows = parity_rows(w)
+    ref_gq = attention_backward(*(t.cpu() for t in ins), spec, rows=rows)[0]
+    idx = torch.as_tensor(rows, device=gq.device)
+    compare(gq[:, :, idx], ref_gq[:, :, rows], "gQ")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,h", [("tf", 7), ("chunk_tf", 2)])
+def test_full_size_one_head_all_gradients(name, h):
+    # Key and value gradients gather over every query row that sees a key,
+    # so one head of the full launch is compared whole: gQ, gK and gV on
+    # all 65,520 rows (about a minute of float64 per head).
+    from oracle.attention_backward import attention_backward_head
+    w, spec, ins, grads = full_size_case(name)
+    ref = attention_backward_head(*(t[0, h].cpu() for t in ins), spec)
+    for what, got, want in zip(("gQ", "gK", "gV"), grads, ref):
+        compare(got[0, h], want, what)
+
+
 def test_backward_deterministic():
     w = CASES[0]
     (q, k, v, g, _, _), _ = make_inputs(w, device="cuda")
