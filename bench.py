@@ -426,9 +426,7 @@ def run_ours(args, w):
         "ms_per_step": round(total_ms_max / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {
-            "workload": f"{w.name}: teacher-forcing mask, B={w.B} H={w.H} d={w.d}, "
-                        f"{w.n_frames} frames x {w.tokens_per_frame} tokens x "
-                        f"{{clean,noisy}} = {w.L} tokens, chunk={w.chunk}",
+            "workload": describe_workload(w),
             "B": w.B, "H": w.H, "L": w.L, "d": w.d, "mode": w.mode,
             "tokens_per_frame": w.tokens_per_frame, "n_frames": w.n_frames, "chunk": w.chunk,
             "pairs_per_head": pairs, "flops_per_step": flops,
@@ -462,6 +460,35 @@ def run_ours(args, w):
                                 if bwd else
                                 cpu_baseline(w, inputs, rows_per_head=args.cpu_rows))
     return line
+
+
+def describe_workload(w) -> str:
+    """One-line name of a workload: its mask, shape and value recipe."""
+    from attention_jvp_continuous_b200.inputs import CHUNK_CAUSAL, FRAME_CAUSAL, TEACHER_FORCING
+    head = f"B={w.B} H={w.H} d={w.d}"
+    if w.mode == TEACHER_FORCING:
+        kind = ("frame-wise teacher-forcing mask" if w.chunk == 1 else
+                f"chunk-wise teacher-forcing mask (chunks of {w.chunk} frames)")
+        toks = f"{w.n_frames} frames x {w.tokens_per_frame} tokens x {{clean,noisy}}"
+    elif w.mode == FRAME_CAUSAL:
+        kind, toks = "frame-causal mask", f"{w.n_frames} frames x {w.tokens_per_frame} tokens"
+    elif w.mode == CHUNK_CAUSAL:
+        kind = f"chunk-causal mask (chunks of {w.chunk} frames)"
+        toks = f"{w.n_frames} frames x {w.tokens_per_frame} tokens"
+    else:
+        kind, toks = "dense (no mask)", f"{w.n_frames} frames x {w.tokens_per_frame} tokens"
+    text = f"{w.name}: {kind}, {head}, {toks} = {w.L} tokens, {w.dtype}"
+    if w.head_scale is not None:
+        lo, hi = w.head_scale
+        text += f", Q and K of each head scaled by s_h ~ U({lo:g}, {hi:g})"
+    return text
+
+
+# The oracle evaluates all sampled rows of one admissible key set with one
+# BLAS call, so its speed per pair grows with the number of rows sampled per
+# head: two samples of one workload give different rates.
+SAMPLE_NOTE = ("the oracle batches the sampled rows that share a key set into one BLAS "
+               "call, so its rate per pair depends on how many rows are sampled")
 
 
 def cache_shape(w):
@@ -724,7 +751,7 @@ def cpu_baseline(w, inputs, rows_per_head: int):
     return {"value": round(12.0 * w.d * sp / dt / 1e12, 6), "unit": UNIT,
             "cores": blas_threads(), "kind": "oracle",
             "sample": f"{rows_per_head} seeded query rows per head x {w.B * w.H} heads "
-                      f"({sp} admitted pairs, {dt:.1f} s, float64 numpy)"}
+                      f"({sp} admitted pairs, {dt:.1f} s, float64 numpy); {SAMPLE_NOTE}"}
 
 
 def oracle_sample_bwd(w, host_in, rows_per_head: int, seed: int = 1234):
@@ -752,7 +779,7 @@ def cpu_baseline_bwd(w, step_in, rows_per_head: int):
             "cores": blas_threads(), "kind": "oracle",
             "sample": f"gradient contributions of {rows_per_head} seeded query rows per "
                       f"head x {w.B * w.H} heads ({sp} admitted pairs, {dt:.1f} s, "
-                      f"float64 numpy)"}
+                      f"float64 numpy); {SAMPLE_NOTE}"}
 
 
 def oracle_sample_cache(w, q, kc, vc, rows_per_head: int, seed: int = 1234):
@@ -852,7 +879,7 @@ def run_reference(args, w):
     total = sum(times)
     value = (4.0 * w.d if args.op == "cache" else flops_per_pair(w, args.op)) * pairs / total / 1e12
     cores = blas_threads()
-    sample = f"{rows} seeded query rows per head x {w.B * w.H} heads per step"
+    sample = f"{rows} seeded query rows per head x {w.B * w.H} heads per step; {SAMPLE_NOTE}"
     line = {
         "impl": "reference",
         "metric": {"bwd": METRIC_BWD, "cache": METRIC_CACHE}.get(args.op, METRIC),

@@ -64,3 +64,13 @@ def test_flops_per_pair(bench):
         d = 128
     assert bench.flops_per_pair(W, "jvp") == 12 * 128
     assert bench.flops_per_pair(W, "bwd") == 10 * 128
+
+
+def test_workload_label_names_its_own_mask(bench):
+    from attention_jvp_continuous_b200.inputs import WORKLOADS
+    labels = {n: bench.describe_workload(w) for n, w in WORKLOADS.items()}
+    assert "frame-causal" in labels["frame_causal"] and "teacher" not in labels["frame_causal"]
+    assert "clean,noisy" not in labels["frame_causal"]
+    assert "chunks of 3 frames" in labels["chunk_tf"]
+    assert "frame-wise teacher-forcing" in labels["tf"]
+    assert "U(0.5, 2)" in labels["tf_long"] and "102960 tokens" in labels["tf_long"]
