@@ -333,7 +333,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       const uint64_t yk_desc = sdesc_sw128(base + LY::Y, 16, 1024);
       const uint64_t ym_desc = sdesc_sw128(base + LY::Y, kTHalf, 1024);
       // First MMAs of tile t: S = A0 X^T (issuer A) or dP = A1 Y^T (issuer B).
-      auto issue_first = [&](const Cursor& c, bool s_mma, const Stage& st) -> bool {
+      // ready: the stage barrier was already seen complete (a test this
+      // thread ran during its previous accumulating MMAs).
+      auto issue_first = [&](const Cursor& c, bool s_mma, const Stage& st, bool ready) -> bool {
         const uint32_t b = c.t & 1u;
         if (c.j == 0 && !wait_w(bar(B_AF), c.item_idx & 1)) return false;
         uint32_t stage;
@@ -342,7 +344,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
           // Buffer b last held tile t-2: issuer A issued acc(t-2), which
           // reads its S part, before this in its own order.
           stage = st.s;
-          if (!wait_w(bar(B_XF + stage), st.ph)) return false;
+          if (!__all_sync(0xffffffffu, ready) && !wait_w(bar(B_XF + stage), st.ph)) return false;
           bdesc = xk_desc + stage * (kTile >> 4);
         } else {
           // dP(t) overwrites the dP part of buffer b. dQ pass: the softmax
@@ -352,7 +354,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
           if (!kKV && c.t >= 2 && !wait_w(bar(B_PF + b), ((c.t >> 1) - 1) & 1u))
             return false;
           stage = st.s;
-          if (!wait_w(bar(B_YF + stage), st.ph)) return false;
+          if (!__all_sync(0xffffffffu, ready) && !wait_w(bar(B_YF + stage), st.ph)) return false;
           bdesc = yk_desc + stage * (kTile >> 4);
         }
         tc_fence_after();
@@ -383,13 +385,21 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       // by issuer A (it reads the S part), gK += dS^T Q by issuer B (the dP
       // part), each followed in its own thread by the first MMA that
       // overwrites that part two tiles later.
-      auto issue_acc = [&](const Cursor& c, bool s_part, const Stage& st) -> bool {
+      // next_bar / next_ph: the stage barrier of this issuer's next first
+      // MMAs (0: none). It is tested here, before this tile's MMAs are
+      // issued, and the result is used only after them, so the test's
+      // latency overlaps the issue. A completed phase stays complete until
+      // this thread has issued the MMAs that read the stage, and every
+      // earlier use of the stage completed under this thread's own waits.
+      auto issue_acc = [&](const Cursor& c, bool s_part, const Stage& st, uint32_t next_bar,
+                           uint32_t next_ph, bool& next_ready) -> bool {
         // X stage of tile t; in the dK/dV pass (NX == NY) also its Y stage.
         const uint32_t b = c.t & 1u, sx = st.s, sy = st.s;
         if (c.j == 0 && c.item_idx > 0 &&
             !wait_w(bar(B_CF), (c.item_idx - 1) & 1))
           return false;
         if (!wait_w(bar(B_PF + b), (c.t >> 1) & 1u)) return false;
+        next_ready = next_bar != 0u && mbar_test(next_bar, next_ph);
         tc_fence_after();
         const uint32_t first = c.j == 0 ? 0u : 1u;
         const uint32_t a_p = tmem + b * 128u + (s_part ? 0u : 64u);
@@ -425,14 +435,16 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         // which nothing completes before this warp's own drain commit, so the
         // bounded wait runs out and the abort path below is taken.
         if (p.stall_test) ok = __all_sync(0xffffffffu, wait_bar(bar(B_DRAIN + 0), 0u, p, abort_flag));
+        bool xr = false;  // XF of cs.t seen complete
         while (ok && ca.valid) {
           while (ok && cs.valid && cs.t < ca.t + 2 && cs.item_idx == ca.item_idx) {
-            ok = issue_first(cs, true, ss);
+            ok = issue_first(cs, true, ss, xr);
+            xr = false;
             cs.next(p, ring, kConsumerWarp);
             ss.step(NX);
           }
           if (!ok) break;
-          ok = issue_acc(ca, true, sa);
+          ok = issue_acc(ca, true, sa, cs.valid ? bar(B_XF + ss.s) : 0u, ss.ph, xr);
           ca.next(p, ring, kConsumerWarp);
           sa.step(NX);
         }
@@ -442,7 +454,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         Stage sc;  // Y stage of c.t
         c.start(p, ring, kConsumerWarp);
         while (c.valid && ok) {
-          ok = issue_first(c, false, sc);
+          ok = issue_first(c, false, sc, false);
           c.next(p, ring, kConsumerWarp);
           sc.step(NY);
         }
@@ -453,14 +465,16 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         Stage sd, sk;  // stages (X and Y alike) of cd.t and ck.t
         cd.start(p, ring, kConsumerWarp);
         ck.start(p, ring, kConsumerWarp);
+        bool yr = false;  // YF of cd.t seen complete
         while (ok && ck.valid) {
           while (ok && cd.valid && cd.t < ck.t + 2 && cd.item_idx == ck.item_idx) {
-            ok = issue_first(cd, false, sd);
+            ok = issue_first(cd, false, sd, yr);
+            yr = false;
             cd.next(p, ring, kConsumerWarp);
             sd.step(NY);
           }
           if (!ok) break;
-          ok = issue_acc(ck, false, sk);
+          ok = issue_acc(ck, false, sk, cd.valid ? bar(B_YF + sd.s) : 0u, sd.ph, yr);
           ck.next(p, ring, kConsumerWarp);
           sk.step(NX);
         }
