@@ -31,6 +31,15 @@ each), QK-norm over all H*d channels with its tangent, RoPE, and the
 [B, H, L, d] layout of the JVP kernel; memory-bound, reported as
 algorithmic GB/s (inputs read once, outputs written once).
 
+``--op ulysses`` measures the context-parallel JVP (Ulysses, the pages'
+sequence-parallel path): every rank holds a token shard [B, H, L/P, d] of
+one workload problem; one step is one ulysses_jvp_attn_fused call (the
+input exchange, this rank's head group through the JVP kernel, the output
+rows stored into their owners' shards by the kernel's epilogue). Strong
+scaling: the job computes one problem whatever P is. The line also reports
+the bare kernel's time on the same problem at P = 1 and the overhead of
+the exchange over it.
+
 ``--op bwd`` measures the masked attention backward instead (gradients of
 <G, O> for the primal output, jvp_attn_bwd) on the same workload, counting
 10*d FLOPs per admitted pair: S recomputed (2d), dP = G V^T (2d), and the
@@ -72,7 +81,7 @@ KERNEL_SOURCES = {
     "bwd": [_CSRC + f for f in ("jvp_attn_bwd_sm100.cu", "sm100_pipeline.cuh", "sm100_ptx.cuh",
                                 "mask_rows.cuh")],
     "cache": [_CSRC + f for f in ("attn_cache_sm100.cu", "sm100_pipeline.cuh", "sm100_ptx.cuh")],
-    "prologue": [_CSRC + "qkv_prologue.cu"],
+    "prologue": [_CSRC + f for f in ("qkv_prologue.cu", "sm100_ptx.cuh")],
 }
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
@@ -459,6 +468,125 @@ def run_ours(args, w):
         line["cpu_baseline"] = (cpu_baseline_bwd(w, step_in, rows_per_head=args.cpu_rows_bwd)
                                 if bwd else
                                 cpu_baseline(w, inputs, rows_per_head=args.cpu_rows))
+    return line
+
+
+def run_ours_ulysses(args, w):
+    import datetime
+    import socket
+
+    import torch
+    import torch.distributed as dist
+
+    import attention_jvp_continuous_b200 as ja
+    from attention_jvp_continuous_b200.inputs import make_inputs
+    from attention_jvp_continuous_b200.ulysses import ShardBuffers, ulysses_jvp_attn_fused
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    if "MASTER_ADDR" not in os.environ:  # a single process outside torchrun
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    ja._lib.lib()
+    mask = ja.Mask(w.mode, w.tokens_per_frame, w.n_frames, w.chunk)
+    pairs, _, _, _ = ja.mask_stats(mask)
+    flops = flops_per_step(w, pairs)
+    if w.H % world or w.L % world:
+        raise SystemExit(f"{w.H} heads / {w.L} tokens do not split over {world} ranks")
+    Ls = w.L // world
+    # Every rank draws the same full problem and keeps its token shard.
+    full, _ = make_inputs(w, device="cuda")
+    shard = [x[:, :, rank * Ls:(rank + 1) * Ls].contiguous() for x in full]
+    bufs = ShardBuffers(w.B, w.H, w.L, w.d, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ulysses_jvp_attn_fused(*shard, mask, bufs)
+
+    for _ in range(args.warmup):
+        step()
+    ja.check_device_error()
+    per, total_ms_max, clocks = device_timed(step, args.steps, world, local, stream, ja)
+    value = flops * args.steps / (total_ms_max * 1e-3) / 1e12
+    launch_ms = sum(per) / len(per)
+
+    # The bare kernel on the whole problem, one GPU (rank 0), same loop.
+    bare_ms = None
+    if rank == 0:
+        o, d_o = torch.empty_like(full[0]), torch.empty_like(full[0])
+        lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device="cuda")
+        for _ in range(args.warmup):
+            ja.jvp_attn_fwd(*full, o, d_o, lse, mask)
+        bper, _, _ = device_timed(lambda: ja.jvp_attn_fwd(*full, o, d_o, lse, mask),
+                                  args.steps, 1, local, stream, ja)
+        bare_ms = sum(bper) / len(bper)
+        del o, d_o, lse
+
+    # End to end: pinned host shards in, the call, this rank's shard of the
+    # outputs back, every step, on the current stream.
+    host_in = [t.cpu().pin_memory() for t in shard]
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory()
+                for t in (bufs.o, bufs.do, bufs.lse)]
+    dev_in = [torch.empty_like(t) for t in shard]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    e2e_steps = max(2, min(args.steps, 10))
+
+    def e2e_step():
+        for d_, h_ in zip(dev_in, host_in):
+            d_.copy_(h_, non_blocking=True)
+        ulysses_jvp_attn_fused(*dev_in, mask, bufs)
+        for h_, d_ in zip(host_out, (bufs.o, bufs.do, bufs.lse)):
+            h_.copy_(d_, non_blocking=True)
+
+    e2e_step()
+    _, e2e_ms, _ = device_timed(e2e_step, e2e_steps, world, local, stream, ja)
+    e2e_value = flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    dist.barrier()
+    del bufs
+    dist.destroy_process_group()
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / world / (launch_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC + " (context-parallel, Ulysses)", "value": round(value, 2),
+        "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms_max / args.steps, 4), "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": describe_workload(w) + f"; token shards of {Ls} tokens on each of "
+                        f"{world} ranks", "B": w.B, "H": w.H, "L": w.L, "d": w.d,
+            "pairs_per_head": pairs, "flops_per_step": flops,
+            "l2": "inputs larger than L2; no flush",
+            "parallelism": f"cp{world} (Ulysses: token shards -> head groups, P2P exchange in, "
+                           "the kernel's scatter epilogue out)",
+            "bare_kernel_ms_one_gpu": None if bare_ms is None else round(bare_ms, 4),
+            "overhead_vs_bare_kernel": (None if bare_ms is None or world != 1
+                                        else round(launch_ms / bare_ms - 1.0, 4)),
+        },
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "note": "this rank's pinned host shards in and its output shard out, serial "
+                        "with the call on one stream"},
+        "gpu_launches": args.steps,  # the JVP kernel; the exchange runs NCCL and torch kernels
+        "roofline": {
+            "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": UNIT,
+            "frac": round(achieved / peak, 4), "traffic": None,
+            "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
+            "kernel": "jvp_attn_sm100_kernel (scatter epilogue) with the exchange around it",
+            "launch_ms": round(launch_ms, 4),
+        },
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, full, rows_per_head=args.cpu_rows)
     return line
 
 
@@ -882,7 +1010,8 @@ def run_reference(args, w):
     sample = f"{rows} seeded query rows per head x {w.B * w.H} heads per step; {SAMPLE_NOTE}"
     line = {
         "impl": "reference",
-        "metric": {"bwd": METRIC_BWD, "cache": METRIC_CACHE}.get(args.op, METRIC),
+        "metric": {"bwd": METRIC_BWD, "cache": METRIC_CACHE,
+                   "ulysses": METRIC + " (context-parallel, Ulysses)"}.get(args.op, METRIC),
         "value": round(value, 6), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * total / args.steps, 2), "higher_is_better": True,
@@ -922,9 +1051,12 @@ def main(argv=None):
                     help="query rows per head in the --op cache cpu_baseline sample")
     ap.add_argument("--cpu-tokens-prologue", type=int, default=16384,
                     help="tokens in the --op prologue cpu_baseline sample")
-    ap.add_argument("--op", choices=["jvp", "bwd", "cache", "prologue"], default="jvp",
+    ap.add_argument("--op", choices=["jvp", "bwd", "cache", "prologue", "ulysses"],
+                    default="jvp",
                     help="jvp: the attention JVP (default); bwd: the masked backward; "
-                         "cache: KV-cache chunk attention of the rollout's last chunk")
+                         "cache: KV-cache chunk attention of the rollout's last chunk; "
+                         "prologue: the layer's tangent prologue; ulysses: the "
+                         "context-parallel JVP over the ranks")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the workload's head count (small cases for ncu captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -947,6 +1079,8 @@ def main(argv=None):
         line = run_ours_cache(args, w)
     elif args.op == "prologue":
         line = run_ours_prologue(args, w)
+    elif args.op == "ulysses":
+        line = run_ours_ulysses(args, w)
     else:
         line = run_ours(args, w)
     if line is not None and rank == 0:
