@@ -19,8 +19,8 @@ FRAME_CAUSAL = 1
 CHUNK_CAUSAL = 2
 TEACHER_FORCING = 3
 
-__all__ = ["Mask", "jvp_attn", "jvp_attn_fwd", "jvp_attn_scatter", "attn_bwd", "jvp_attn_bwd", "bwd_scratch_len",
-           "cache_attn", "rope_copy", "qkv_prologue", "mask_stats", "tile_classes",
+__all__ = ["Mask", "jvp_attn", "jvp_attn_fwd", "jvp_attn_scatter", "signal_barrier", "attn_bwd",
+           "jvp_attn_bwd", "bwd_scratch_len", "cache_attn", "rope_copy", "qkv_prologue", "mask_stats", "tile_classes",
            "schedule", "schedule_kv", "check_device_error", "set_wait_limit", "set_stall_test", "release",
            "JvpAttnError",
            "DENSE", "FRAME_CAUSAL", "CHUNK_CAUSAL", "TEACHER_FORCING"]
@@ -110,6 +110,24 @@ def jvp_attn_scatter(q, k, v, dq, dk, dv, mask: Mask, o_dst, do_dst, lse_dst, h0
         B, H, L, d, _dtype_code(q), mask.desc(),
         0.0 if scale is None else float(scale), ctypes.c_void_p(stream))
     _lib.check(rc, "jvp_attn_fwd_scatter")
+
+
+def signal_barrier(flags, rank: int, epoch: int, stream: Optional[int] = None) -> None:
+    """Device-side barrier of the ranks of a context-parallel group on the
+    current stream (jvp_attn_signal_barrier). flags: one int32 CUDA tensor
+    view per rank of that rank's n_ranks flag words (this process's address
+    of it), zero before the first barrier; epoch: 1, 2, ... per barrier."""
+    import torch
+    n = len(flags)
+    for t in flags:
+        if not t.is_cuda or t.dtype != torch.int32 or t.numel() < n:
+            raise ValueError("flags must be int32 CUDA tensors of at least n_ranks words")
+    if stream is None:
+        stream = torch.cuda.current_stream(flags[0].device).cuda_stream
+    arr = (ctypes.c_void_p * n)(*[t.data_ptr() for t in flags])
+    rc = _lib.lib().jvp_attn_signal_barrier(arr, n, int(rank), ctypes.c_uint32(epoch & 0xFFFFFFFF),
+                                            ctypes.c_void_p(stream))
+    _lib.check(rc, "jvp_attn_signal_barrier")
 
 
 def jvp_attn(q, k, v, dq, dk, dv, mask: Mask, scale: Optional[float] = None,

@@ -32,7 +32,8 @@ JVP_FP32 = 1
 TILE_EMPTY, TILE_FULL, TILE_PARTIAL = 0, 1, 2
 
 # Exported functions, as declared in include/jvp_attn.h.
-EXPORTS = ("jvp_attn_fwd", "jvp_attn_fwd_noalloc", "jvp_attn_fwd_scatter", "jvp_attn_bwd", "jvp_attn_bwd_scratch_len",
+EXPORTS = ("jvp_attn_fwd", "jvp_attn_fwd_noalloc", "jvp_attn_fwd_scatter", "jvp_attn_signal_barrier",
+           "jvp_attn_bwd", "jvp_attn_bwd_scratch_len",
            "jvp_attn_cache_fwd", "jvp_attn_rope_copy", "jvp_attn_qkv_prologue",
            "jvp_attn_mask_stats",
            "jvp_attn_tile_classes", "jvp_attn_schedule", "jvp_attn_schedule_kv",
@@ -81,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.jvp_attn_fwd_scatter.argtypes = [vp] * 6 + [vpp, vpp, vpp] + [i32] * 3 + \
             [i32] * 5 + [MaskDesc, ctypes.c_float, vp]
         L.jvp_attn_fwd_scatter.restype = i32
+        L.jvp_attn_signal_barrier.argtypes = [vpp, i32, i32, ctypes.c_uint32, vp]
+        L.jvp_attn_signal_barrier.restype = i32
         fp = ctypes.POINTER(ctypes.c_float)
         L.jvp_attn_bwd.argtypes = [vp] * 5 + [fp] + [vp] * 3 + [fp, ctypes.c_int64] + \
             [i32] * 5 + [MaskDesc, ctypes.c_float, vp]

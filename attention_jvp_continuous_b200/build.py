@@ -19,7 +19,7 @@ LIB_NAME = "libjvpattn.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
 SOURCES = ["jvp_attn_api.cu", "schedule.cpp", "jvp_attn_simt.cu", "jvp_attn_sm100.cu",
            "jvp_attn_bwd_sm100.cu", "jvp_attn_noalloc.cu",
-           "attn_cache_sm100.cu", "rope_copy.cu", "qkv_prologue.cu"]
+           "attn_cache_sm100.cu", "rope_copy.cu", "qkv_prologue.cu", "signal_barrier.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

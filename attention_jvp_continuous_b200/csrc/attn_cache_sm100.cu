@@ -17,10 +17,14 @@
 //                every row with its own running max and its own O
 //                accumulator (lazy rescale only when its row max grows by
 //                more than 2^8); the epilogue merges the two halves
-// Work item = (batch*head, 128-query tile, key split). When the chunk has
-// too few query tiles to fill the GPU the key range is split and every
-// split writes an unnormalised fp32 partial (O, running max, sum) that a
-// second kernel combines; otherwise the epilogue writes O and LSE itself.
+// Work items are (batch*head, 128-query tile) pairs over all key tiles, as
+// many as fill whole waves of the grid, in head-major order (the CTAs
+// running at once read the same key tiles of a head, served from L2); the
+// items left over are cut into about one key-range piece per SM, listed
+// piece-major so that concurrent CTAs again share key ranges. A whole item
+// writes O and LSE itself; a piece writes an unnormalised fp32 partial (O,
+// running max, sum) into its own slot, and a second kernel combines the
+// pieces of each cut item. CTAs take items dynamically, in list order.
 //
 // TMEM: S buffer b at [128 b, 128 b + 128), the bf16 P of each key half
 // packed over the start of that half's S columns; O_a at [256, 384) and O_b
@@ -123,16 +127,16 @@ __device__ __forceinline__ uint64_t ex2_fma2(float x0, float x1) {
 }
 
 struct Params {
-  const int4* qtiles;  // {qt, seg_begin, seg_count, n_ktiles}; entry = split * n_qt + qt
+  const int4* qtiles;  // per piece: {qt, seg_begin, seg_count, n_ktiles}
   const int2* segs;    // {kt_begin, (count << 1) | partial}
-  int n_entries, n_segs, n_items, n_qt, n_kt;
+  const int2* piece_meta;  // per piece: {bh, partial slot or -1}
+  int n_entries, n_segs, n_items, n_qt, n_kt, n_bh;
   int Lq, Lk;
   float scale, c2;
-  int split;           // 1: write fp32 partials for the combine kernel
   __nv_bfloat16* o;    // [B*H, Lq, d]
   float* lse;          // [B*H, Lq]
-  float* part;         // [n_items, 128, d] unnormalised partial O (split only)
-  float2* ml;          // [n_items, 128] {running max (log2), sum} (split only)
+  float* part;         // [slots, 128, d] unnormalised partial O
+  float2* ml;          // [slots, 128] {running max (log2), sum}
   unsigned* err;
   unsigned* item_ctr;
   unsigned long long wait_limit_ns;
@@ -453,8 +457,10 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const float lt = w_a * l_a + w_b * l_b;
         tc_fence_after();
         const bool row_ok = grow < p.Lq;
+        const int slot = p.piece_meta[c.item].y;  // -1: this piece is the whole item
+        const bool split = slot >= 0;
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
-        const float sa_ = p.split ? w_a : w_a * inv, sb_ = p.split ? w_b : w_b * inv;
+        const float sa_ = split ? w_a : w_a * inv, sb_ = split ? w_b : w_b * inv;
         // This warpgroup writes head-dim columns [64 hw, 64 hw + 64).
 #pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {
@@ -467,7 +473,7 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             v[i] = fmaf(__uint_as_float(oa[i]), sa_, __uint_as_float(ob[i]) * sb_);
-          if (!p.split) {
+          if (!split) {
             if (row_ok) {
               uint4* go = reinterpret_cast<uint4*>(p.o + (size_t(c.bh) * p.Lq + grow) * D + col);
 #pragma unroll
@@ -478,9 +484,9 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                    pack_bf16(v[8 * i + 6], v[8 * i + 7]));
             }
           } else {
-            // Unnormalised partial of this key split relative to M, for every
+            // Unnormalised partial of this piece relative to M, for every
             // row of the tile (rows past Lq are never combined).
-            float4* dst = reinterpret_cast<float4*>(p.part + (size_t(c.item) * BM + r) * D + col);
+            float4* dst = reinterpret_cast<float4*>(p.part + (size_t(slot) * BM + r) * D + col);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
               dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
@@ -489,8 +495,8 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         tc_fence_before();
         mbar_arrive(bar(B_AFREE));
         if (hw == 0) {
-          if (p.split)
-            p.ml[size_t(c.item) * BM + r] = make_float2(M, lt);
+          if (split)
+            p.ml[size_t(slot) * BM + r] = make_float2(M, lt);
           else if (row_ok)
             p.lse[size_t(c.bh) * p.Lq + grow] =
                 lt > 0.f ? (M + log2f(lt)) * 0.69314718055994531f : -CUDART_INF_F;
@@ -508,35 +514,40 @@ attn_cache_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   }
 }
 
-// Combines the key splits of each query row: with per-split running max m_s
-// (log2 units of the scaled score), sum l_s and unnormalised partial O_s,
+// Combines the pieces of each split item, row by row: with per-piece
+// running max m_s (log2 units of the scaled score), sum l_s and unnormalised
+// partial O_s,
 //   M = max m_s,  w_s = 2^(m_s - M),  O = sum w_s O_s / sum w_s l_s,
 //   LSE = (M + log2 sum w_s l_s) ln 2.
-// One warp per (batch*head, query row), 4 head-dim columns per lane.
+// One warp per (split item, row of its query tile), 4 head-dim columns per
+// lane. splits[i] = {bh, qt, first slot, slot count}.
 __global__ void __launch_bounds__(256)
 attn_cache_combine_kernel(const float* __restrict__ part, const float2* __restrict__ ml,
-                          __nv_bfloat16* __restrict__ o, float* __restrict__ lse, int BH,
-                          int Lq, int n_qt, int n_entries, int splits) {
+                          const int4* __restrict__ splits, int n_splits, int n_slots,
+                          __nv_bfloat16* __restrict__ o, float* __restrict__ lse, int n_bh,
+                          int Lq, unsigned* err) {
   const int lane = threadIdx.x & 31;
-  const long long n_rows = (long long)BH * Lq;
+  const long long n_rows = (long long)n_splits * BM;
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
   for (long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < n_rows;
        w += warps) {
-    const int bh = int(w / Lq), i = int(w % Lq);
-    const int qt = i / BM, r = i % BM;
-    float M = -CUDART_INF_F;
-    for (int s = 0; s < splits; ++s) {
-      const size_t item = size_t(bh) * n_entries + size_t(s) * n_qt + qt;
-      M = fmaxf(M, ml[item * BM + r].x);
+    const int4 sp = splits[w / BM];
+    const int r = int(w % BM);
+    const int bh = sp.x, i = sp.y * BM + r;
+    if (bh < 0 || bh >= n_bh || sp.z < 0 || sp.w < 1 || sp.z + sp.w > n_slots) {
+      if (lane == 0) atomicOr(err, kErrBounds);
+      continue;
     }
+    if (i >= Lq) continue;
+    float M = -CUDART_INF_F;
+    for (int s = sp.z; s < sp.z + sp.w; ++s) M = fmaxf(M, ml[size_t(s) * BM + r].x);
     float lsum = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < splits; ++s) {
-      const size_t item = size_t(bh) * n_entries + size_t(s) * n_qt + qt;
-      const float2 v = ml[item * BM + r];
+    for (int s = sp.z; s < sp.z + sp.w; ++s) {
+      const float2 v = ml[size_t(s) * BM + r];
       const float ws = v.x == -CUDART_INF_F ? 0.f : exp2f(v.x - M);
       lsum += ws * v.y;
-      const float4 pv = reinterpret_cast<const float4*>(part + (item * BM + r) * D)[lane];
+      const float4 pv = reinterpret_cast<const float4*>(part + (size_t(s) * BM + r) * D)[lane];
       acc.x += ws * pv.x;
       acc.y += ws * pv.y;
       acc.z += ws * pv.z;
@@ -584,7 +595,7 @@ static bool make_map(CUtensorMap* m, const void* ptr, int rows, int rows_alloc, 
 
 }  // namespace cache
 
-int launch_cache_sm100(const CacheArgs& a, const WorkList& w, int splits, int num_sms) {
+int launch_cache_sm100(const CacheArgs& a, const CacheWork& cw, int num_sms) {
   using namespace cache;
   const int BH = a.B * a.H;
   CUtensorMap mq, mk, mv;
@@ -592,20 +603,19 @@ int launch_cache_sm100(const CacheArgs& a, const WorkList& w, int splits, int nu
       !make_map(&mv, a.v, a.Lk, a.Lcache, BH))
     return JVP_ERR_LAUNCH_FAILED;
   Params p;
-  p.qtiles = w.qtiles;
-  p.segs = w.segs;
-  p.n_entries = w.n_qtiles;
-  p.n_segs = w.n_segs;
-  const long long items = (long long)w.n_qtiles * BH;
-  if (items > 0x7fffffffLL) return JVP_ERR_TOO_LARGE;
-  p.n_items = int(items);
+  p.qtiles = cw.w.qtiles;
+  p.segs = cw.w.segs;
+  p.piece_meta = cw.meta;
+  p.n_entries = cw.w.n_qtiles;
+  p.n_segs = cw.w.n_segs;
+  p.n_items = cw.w.n_qtiles;
   p.n_qt = (a.Lq + BM - 1) / BM;
   p.n_kt = (a.Lk + BN - 1) / BN;
+  p.n_bh = BH;
   p.Lq = a.Lq;
   p.Lk = a.Lk;
   p.scale = a.scale;
   p.c2 = a.scale * 1.4426950408889634f;
-  p.split = splits > 1 ? 1 : 0;
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.lse = a.lse;
   p.part = a.part;
@@ -614,7 +624,7 @@ int launch_cache_sm100(const CacheArgs& a, const WorkList& w, int splits, int nu
   p.item_ctr = a.item_ctr;
   p.wait_limit_ns = a.wait_limit_ns;
   p.stall_test = a.stall_test ? 1 : 0;
-  if (p.split && (!p.part || !p.ml)) return JVP_ERR_LAUNCH_FAILED;
+  if (p.n_items < 1 || (cw.n_slots > 0 && (!p.part || !p.ml))) return JVP_ERR_LAUNCH_FAILED;
   static std::mutex attr_mu;
   static bool attr_done[64] = {};
   int dev = 0;
@@ -629,17 +639,18 @@ int launch_cache_sm100(const CacheArgs& a, const WorkList& w, int splits, int nu
       attr_done[dev] = true;
     }
   }
-  const int grid = int(items < num_sms ? items : num_sms);
+  const int grid = p.n_items < num_sms ? p.n_items : num_sms;
   if (!a.item_ctr || cudaMemsetAsync(a.item_ctr, 0, sizeof(unsigned), a.stream) != cudaSuccess)
     return JVP_ERR_LAUNCH_FAILED;
   attn_cache_sm100_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return JVP_ERR_LAUNCH_FAILED;
-  if (p.split) {
-    const long long rows = (long long)BH * a.Lq;
+  if (cw.n_splits > 0) {
+    const long long rows = (long long)cw.n_splits * BM;
     const long long blocks = (rows + 7) / 8;  // 8 warps per block
     const int cgrid = int(blocks < 8LL * num_sms ? blocks : 8LL * num_sms);
-    attn_cache_combine_kernel<<<cgrid, 256, 0, a.stream>>>(p.part, p.ml, p.o, p.lse, BH, a.Lq,
-                                                           p.n_qt, p.n_entries, splits);
+    attn_cache_combine_kernel<<<cgrid, 256, 0, a.stream>>>(p.part, p.ml, cw.splits, cw.n_splits,
+                                                           cw.n_slots, p.o, p.lse, BH, a.Lq,
+                                                           a.err);
     if (cudaGetLastError() != cudaSuccess) return JVP_ERR_LAUNCH_FAILED;
   }
   return JVP_OK;

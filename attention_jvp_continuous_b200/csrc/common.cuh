@@ -87,12 +87,21 @@ struct CacheArgs {
   unsigned* item_ctr;
   unsigned long long wait_limit_ns;
   bool stall_test = false;  // jvp_attn_set_stall_test
-  float* part;  // split > 1: [items, 128, 128] fp32 partial outputs
-  float* ml;    // split > 1: [items, 128] {max, sum} pairs
+  float* part;  // [slots, 128, 128] fp32 partial outputs (pieces of split items)
+  float* ml;    // [slots, 128] {max, sum} pairs
 };
 
-// w: dense split work list (build_schedule_dense with 128 x 128 tiles).
-int launch_cache_sm100(const CacheArgs& a, const WorkList& w, int splits, int num_sms);
+// Device copy of a cache-attention work list (build_schedule_cache, 128 x
+// 128 tiles): the pieces as a WorkList plus their {bh, slot}, and the cut
+// items {bh, qt, first slot, slot count}.
+struct CacheWork {
+  WorkList w;
+  const int2* meta = nullptr;
+  const int4* splits = nullptr;
+  int n_splits = 0, n_slots = 0;
+};
+
+int launch_cache_sm100(const CacheArgs& a, const CacheWork& cw, int num_sms);
 
 // Row copy with optional rotary embedding (jvp_attn_rope_copy).
 struct RopeArgs {
@@ -105,6 +114,10 @@ struct RopeArgs {
   cudaStream_t stream;
 };
 int launch_rope_copy(const RopeArgs& a, int num_sms);
+
+// Device-side barrier of n <= kMaxShards ranks (jvp_attn_signal_barrier).
+int launch_signal_barrier(uint32_t* const* flags, int n, int rank, uint32_t epoch,
+                          unsigned* err, unsigned long long limit_ns, cudaStream_t st);
 
 // Attention-layer tangent prologue (jvp_attn_qkv_prologue): bf16.
 struct PrologueArgs {

@@ -36,8 +36,8 @@ struct DevInfo {
 };
 
 struct WsKey {
-  // kind 0: query-tile list, 1: key-tile list (mask fields), 2: dense split
-  // list for cache attention (T = splits, chunk = Lq, L = Lk).
+  // kind 0: query-tile list, 1: key-tile list (mask fields), 3: cache
+  // attention list (T = grid, F = B*H, chunk = Lq, L = Lk).
   int dev, mode, T, F, chunk, L, bm, bn, kind;
   bool operator<(const WsKey& o) const {
     return std::tie(dev, mode, T, F, chunk, L, bm, bn, kind) <
@@ -48,6 +48,7 @@ struct WsKey {
 struct Ws {
   void* buf = nullptr;
   WorkList w;
+  CacheWork cw;  // kind 3 only
 };
 
 std::mutex g_mu;
@@ -126,15 +127,48 @@ int get_worklist(int dev, const jvp_mask_desc& m, int L, WorkList* out, int bm =
   return upload_schedule(key, s, out);
 }
 
-int get_worklist_dense(int dev, int Lq, int Lk, int splits, WorkList* out) {
-  const WsKey key{dev, -1, splits, 0, Lq, Lk, 128, 128, 2};
+// Work list of cache attention for (Lq, Lk, B*H) on `grid` CTAs, uploaded
+// once and cached.
+int get_worklist_cache(int dev, int Lq, int Lk, int BH, int grid, CacheWork* out) {
+  const WsKey key{dev, -1, grid, BH, Lq, Lk, 128, 128, 3};
   std::lock_guard<std::mutex> lk(g_mu);
   auto it = g_ws.find(key);
   if (it != g_ws.end()) {
-    *out = it->second.w;
+    *out = it->second.cw;
     return JVP_OK;
   }
-  return upload_schedule(key, build_schedule_dense(Lq, Lk, 128, 128, splits), out);
+  const CacheSchedule s = build_schedule_cache(Lq, Lk, 128, 128, BH, grid);
+  const std::vector<int32_t>* parts[] = {&s.entries, &s.segs, &s.meta, &s.splits};
+  size_t off[5] = {0};
+  for (int i = 0; i < 4; ++i)
+    off[i + 1] = (off[i] + parts[i]->size() * sizeof(int32_t) + 255) & ~size_t(255);
+  Ws ws;
+  if (cudaMalloc(&ws.buf, off[4] + 256) != cudaSuccess) {
+    cudaGetLastError();
+    return JVP_ERR_OUT_OF_MEMORY;
+  }
+  char* b = static_cast<char*>(ws.buf);
+  for (int i = 0; i < 4; ++i) {
+    if (parts[i]->empty()) continue;
+    if (cudaMemcpy(b + off[i], parts[i]->data(), parts[i]->size() * sizeof(int32_t),
+                   cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaFree(ws.buf);
+      return JVP_ERR_LAUNCH_FAILED;
+    }
+  }
+  CacheWork& cw = ws.cw;
+  cw.w.qtiles = reinterpret_cast<const int4*>(b + off[0]);
+  cw.w.segs = reinterpret_cast<const int2*>(b + off[1]);
+  cw.w.n_qtiles = int(s.entries.size() / 4);
+  cw.w.n_segs = int(s.segs.size() / 2);
+  cw.meta = reinterpret_cast<const int2*>(b + off[2]);
+  cw.splits = reinterpret_cast<const int4*>(b + off[3]);
+  cw.n_splits = int(s.splits.size() / 4);
+  cw.n_slots = s.n_slots;
+  ws.w = cw.w;
+  g_ws[key] = ws;
+  *out = cw;
+  return JVP_OK;
 }
 
 // Partial-result workspace of at least `bytes` for (dev, st).
@@ -162,23 +196,6 @@ int get_partials(int dev, cudaStream_t st, size_t bytes, void** out) {
   return JVP_OK;
 }
 
-// Key splits for cache attention: `units` = B*H*query tiles; minimises
-// waves(S) * (tiles per split + 2), the +2 standing for a split's partial
-// write and combine; ties go to fewer splits.
-int choose_splits(long long units, int n_kt, int sms) {
-  int best = 1;
-  double best_cost = 1e300;
-  const int smax = n_kt < 64 ? n_kt : 64;
-  for (int sp = 1; sp <= smax; ++sp) {
-    const long long waves = (units * sp + sms - 1) / sms;
-    const double cost = double(waves) * (double(n_kt) / sp + (sp > 1 ? 2.0 : 0.0));
-    if (cost < best_cost - 1e-9) {
-      best_cost = cost;
-      best = sp;
-    }
-  }
-  return best;
-}
 
 int get_counter(int dev, cudaStream_t st, unsigned** out) {
   std::lock_guard<std::mutex> lk(g_mu);
@@ -402,23 +419,21 @@ int jvp_attn_cache_fwd(const void* q, const void* k_cache, const void* v_cache, 
   a.stall_test = stall_test();
   a.part = nullptr;
   a.ml = nullptr;
-  const int n_qt = (Lq + 127) / 128, n_kt = (Lk + 127) / 128;
-  const int splits = choose_splits((long long)B * H * n_qt, n_kt, di->sms);
-  WorkList w;
-  rc = get_worklist_dense(dev, Lq, Lk, splits, &w);
+  CacheWork cw;
+  rc = get_worklist_cache(dev, Lq, Lk, B * H, di->sms, &cw);
   if (rc != JVP_OK) return rc;
-  if (splits > 1) {
-    const size_t items = size_t(B) * H * n_qt * splits;
-    const size_t part_bytes = items * 128 * 128 * sizeof(float);
+  if (cw.n_slots > 0) {
+    const size_t part_bytes = size_t(cw.n_slots) * 128 * 128 * sizeof(float);
     void* buf = nullptr;
-    rc = get_partials(dev, a.stream, part_bytes + items * 128 * 2 * sizeof(float), &buf);
+    rc = get_partials(dev, a.stream, part_bytes + size_t(cw.n_slots) * 128 * 2 * sizeof(float),
+                      &buf);
     if (rc != JVP_OK) return rc;
     a.part = static_cast<float*>(buf);
     a.ml = reinterpret_cast<float*>(static_cast<char*>(buf) + part_bytes);
   }
   rc = get_counter(dev, a.stream, &a.item_ctr);
   if (rc != JVP_OK) return rc;
-  return launch_cache_sm100(a, w, splits, di->sms);
+  return launch_cache_sm100(a, cw, di->sms);
 }
 
 int jvp_attn_rope_copy(const void* src, void* dst, int B, int H, int src_rows, int dst_rows,
@@ -574,6 +589,22 @@ int jvp_attn_check_device_error(void* stream) {
   if (w & kErrTimeout) return JVP_ERR_DEVICE_TIMEOUT;
   if (w & kErrBounds) return JVP_ERR_DEVICE_BOUNDS;
   return JVP_OK;
+}
+
+int jvp_attn_signal_barrier(uint32_t* const* flags, int n_ranks, int rank, uint32_t epoch,
+                            void* stream) {
+  if (!flags || n_ranks < 1 || n_ranks > kMaxShards || rank < 0 || rank >= n_ranks)
+    return JVP_ERR_INVALID_ARG;
+  for (int q = 0; q < n_ranks; ++q) {
+    if (!flags[q]) return JVP_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(flags[q]) & 3u) return JVP_ERR_MISALIGNED;
+  }
+  DevInfo* di = nullptr;
+  const int rc = device_info(&di);
+  if (rc != JVP_OK) return rc;
+  if (di->major != 10 || di->minor != 0) return JVP_ERR_UNSUPPORTED_DEVICE;
+  return launch_signal_barrier(flags, n_ranks, rank, epoch, di->err, wait_limit_ns(),
+                               static_cast<cudaStream_t>(stream));
 }
 
 int jvp_attn_set_wait_limit(uint64_t ns) {

@@ -251,17 +251,16 @@ Schedule build_schedule_kv(const jvp_mask_desc& m, int L, int bq, int bk) {
   return s;
 }
 
-Schedule build_schedule_dense(int Lq, int Lk, int bq, int bk, int splits) {
-  Schedule s;
-  s.L = Lk;
-  s.bm = bq;
-  s.bn = bk;
+CacheSchedule build_schedule_cache(int Lq, int Lk, int bq, int bk, int BH, int grid) {
+  CacheSchedule s;
   s.n_qt = (Lq + bq - 1) / bq;
   s.n_kt = (Lk + bk - 1) / bk;
   const bool ragged = Lk % bk != 0;
-  for (int sp = 0; sp < splits; ++sp) {
-    const int k0 = int(int64_t(sp) * s.n_kt / splits);
-    const int k1 = int(int64_t(sp + 1) * s.n_kt / splits);
+  const int64_t U = int64_t(BH) * s.n_qt;
+  const int64_t n_whole = grid > 0 ? U / grid * grid : U;  // whole waves
+  const int r = int(U - n_whole);                          // items left over
+  // Appends one piece: key tiles [k0, k1) of item u.
+  auto piece = [&](int64_t u, int k0, int k1, int slot) {
     const int seg_begin = int(s.segs.size() / 2);
     int nseg = 0;
     const int full_end = (ragged && k1 == s.n_kt) ? k1 - 1 : k1;
@@ -275,16 +274,42 @@ Schedule build_schedule_dense(int Lq, int Lk, int bq, int bk, int splits) {
       s.segs.push_back((1 << 1) | 1);
       ++nseg;
     }
-    s.max_ktiles = std::max<int64_t>(s.max_ktiles, k1 - k0);
-    for (int qt = 0; qt < s.n_qt; ++qt) {
-      s.qtiles.push_back(qt);
-      s.qtiles.push_back(seg_begin);
-      s.qtiles.push_back(nseg);
-      s.qtiles.push_back(k1 - k0);
-      s.n_full += full_end - k0;
-      s.n_partial += k1 - full_end;
+    s.entries.push_back(int32_t(u % s.n_qt));
+    s.entries.push_back(seg_begin);
+    s.entries.push_back(nseg);
+    s.entries.push_back(k1 - k0);
+    s.meta.push_back(int32_t(u / s.n_qt));
+    s.meta.push_back(slot);
+  };
+  for (int64_t u = 0; u < n_whole; ++u) piece(u, 0, s.n_kt, -1);
+  if (r == 0) return s;
+  // About `grid` pieces over the r leftover items, at least 4 key tiles
+  // each: item i gets p_i pieces, the first grid % r items one more.
+  const int cap = std::max(1, s.n_kt / 4);
+  std::vector<int> np(r), slot0(r, -1);
+  int max_p = 0;
+  for (int i = 0; i < r; ++i) {
+    np[i] = std::min(cap, std::max(1, grid / r + (i < grid % r ? 1 : 0)));
+    max_p = std::max(max_p, np[i]);
+    if (np[i] > 1) {
+      slot0[i] = s.n_slots;
+      s.n_slots += np[i];
+      const int64_t u = n_whole + i;
+      s.splits.push_back(int32_t(u / s.n_qt));
+      s.splits.push_back(int32_t(u % s.n_qt));
+      s.splits.push_back(slot0[i]);
+      s.splits.push_back(np[i]);
     }
   }
+  // Piece-major order: concurrent CTAs take the same key range of the
+  // leftover items, which share it in L2.
+  for (int j = 0; j < max_p; ++j)
+    for (int i = 0; i < r; ++i)
+      if (j < np[i]) {
+        const int k0 = int(int64_t(j) * s.n_kt / np[i]);
+        const int k1 = int(int64_t(j + 1) * s.n_kt / np[i]);
+        piece(n_whole + i, k0, k1, np[i] > 1 ? slot0[i] + j : -1);
+      }
   return s;
 }
 

@@ -48,14 +48,30 @@ Schedule build_schedule(const jvp_mask_desc& m, int L, int bm, int bn);
 // here, since the pass reads per-query LSE and D values).
 Schedule build_schedule_kv(const jvp_mask_desc& m, int L, int bq, int bk);
 
-// Dense rectangular work list for chunk attention over a key/value cache:
-// Lq query rows against the first Lk keys, all admitted. The key tiles of
-// bk keys are cut into `splits` contiguous ranges of near-equal length
-// (split s: tiles [s n_kt / splits, (s+1) n_kt / splits)); entry e = s *
-// n_qt + qt covers query tile qt of split s: {qt, seg_begin, seg_count,
-// n_ktiles}. The last key tile is PARTIAL when Lk is not a multiple of bk
-// (its own segment); all others are FULL. Requires 1 <= splits <= n_kt.
-Schedule build_schedule_dense(int Lq, int Lk, int bq, int bk, int splits);
+// Work list for chunk attention over a key/value cache: Lq query rows
+// against the first Lk keys, all admitted, for BH (batch, head) pairs, on
+// `grid` persistent CTAs taking items in list order. The items (bh, query
+// tile of bq rows) of n_kt key tiles of bk keys each come first, whole and
+// in (bh, query tile) order, as many as fill whole waves of the grid
+// (concurrent CTAs then read the same key tiles of one head, which stay in
+// L2). The r items left over are cut into about `grid` pieces in all (key
+// ranges of near-equal length, at least 4 tiles where possible), listed
+// piece-major so that concurrent CTAs again share key ranges. A piece of a
+// cut item writes an fp32 partial into its own slot (the slots of an item
+// are consecutive) for a combine step; a whole item writes the output
+// itself. The last key tile is PARTIAL when Lk is not a multiple of bk.
+struct CacheSchedule {
+  int n_qt = 0, n_kt = 0, n_slots = 0;
+  // Per piece, in list order: {qt, seg_begin, seg_count, n_ktiles}.
+  std::vector<int32_t> entries;
+  // Segments: {kt_begin, (kt_count << 1) | partial}.
+  std::vector<int32_t> segs;
+  // Per piece: {bh, partial slot, or -1 for a whole item}.
+  std::vector<int32_t> meta;
+  // Per cut item: {bh, qt, first slot, slot count}.
+  std::vector<int32_t> splits;
+};
+CacheSchedule build_schedule_cache(int Lq, int Lk, int bq, int bk, int BH, int grid);
 
 // The same work list as build_schedule (same entries, same order), written
 // into caller-provided arrays without any heap allocation: entries of 4

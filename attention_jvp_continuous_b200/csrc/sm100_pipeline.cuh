@@ -11,6 +11,8 @@
 
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "sm100_ptx.cuh"
 
@@ -64,9 +66,18 @@ struct ItemRing {
   volatile uint32_t* abort_flag;
 };
 
+// Kernels whose parameters carry `piece_meta` ({bh, ...} per work item)
+// list every item explicitly: item i is entry i of the work list, and its
+// (batch*head) comes from piece_meta[i] instead of from the item index.
+template <class P, class = void>
+struct PieceMeta : std::false_type {};
+template <class P>
+struct PieceMeta<P, std::void_t<decltype(&P::piece_meta)>> : std::true_type {};
+
 // Walks this CTA's (item, inner tile) sequence; every role runs its own copy.
 // P provides: qtiles / segs (the work list), n_entries, n_segs, n_items,
-// n_qt (outer tiles), n_kt (inner tiles), err, item_ctr, wait_limit_ns.
+// n_qt (outer tiles), n_kt (inner tiles), err, item_ctr, wait_limit_ns (and,
+// for explicit item lists, piece_meta and n_bh).
 template <class P>
 struct Cursor {
   int item, item_idx, bh, qt;
@@ -107,8 +118,19 @@ struct Cursor {
   __device__ void load_item(const P& p, const ItemRing& r, Role role) {
     valid = acquire(p, r, role) && item < p.n_items;
     if (!valid) return;
-    const int e = item % p.n_entries;
-    bh = item / p.n_entries;
+    int e;
+    if constexpr (PieceMeta<P>::value) {
+      e = item;
+      bh = p.piece_meta[item].x;
+      if (bh < 0 || bh >= p.n_bh) {
+        atomicOr(p.err, kErrBounds);
+        valid = false;
+        return;
+      }
+    } else {
+      e = item % p.n_entries;
+      bh = item / p.n_entries;
+    }
     const int4 en = p.qtiles[e];
     qt = en.x;
     seg = en.y;

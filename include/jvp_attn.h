@@ -148,8 +148,8 @@ int jvp_attn_fwd(const void* q, const void* k, const void* v,
  *   1 <= n_shards <= 8, L % n_shards == 0, 0 <= h0, h0 + H <= h_total.
  * Rows of a destination not owned by this head group are left untouched;
  * with every rank's call, each shard receives all h_total heads. Visibility
- * on a peer: after this launch completes (e.g. stream synchronisation
- * followed by a barrier between the ranks). Errors as jvp_attn_fwd, plus
+ * on a peer: after this launch completes on every rank, e.g. after a
+ * jvp_attn_signal_barrier enqueued behind it on each rank. Errors as jvp_attn_fwd, plus
  * JVP_ERR_INVALID_ARG for a null or out-of-range shard argument and
  * JVP_ERR_MISALIGNED for a destination not 16-byte aligned.
  */
@@ -159,6 +159,35 @@ int jvp_attn_fwd_scatter(const void* q, const void* k, const void* v,
                          int n_shards, int h0, int h_total,
                          int B, int H, int L, int d, jvp_dtype dtype,
                          jvp_mask_desc mask, float softmax_scale, void* stream);
+
+/*
+ * jvp_attn_signal_barrier: a barrier of the n_ranks processes (one per GPU)
+ * of a context-parallel group, enqueued on `stream`. It brackets the fused
+ * output exchange of Ulysses context parallelism (Causal-rCM report, Sec.
+ * 3.2.2 "JVP Ulysses CP"), where jvp_attn_fwd_scatter stores rows into
+ * other ranks' shards: before the launch no rank may still be reading the
+ * shard it will receive, and after it a shard is complete only once every
+ * rank's kernel is done.
+ *
+ * flags       host array of n_ranks device pointers: flags[q] is this
+ *             process's address of rank q's n_ranks uint32 flag words
+ *             (memory every rank can reach, e.g. symmetric memory), all
+ *             zero before the first barrier; 4-byte aligned
+ * rank        this process's rank, 0 <= rank < n_ranks <= 8
+ * epoch       1 for the first barrier on these flags, then 2, 3, ...; every
+ *             rank passes the same sequence
+ * Once the work enqueued before it on `stream` is complete, the barrier
+ * stores epoch into word `rank` of every rank's flags (release, system
+ * scope) and waits (acquire loads) until all words of its own flags have
+ * reached epoch; work enqueued after it on `stream` starts only then. The
+ * wait is bounded by the limit of jvp_attn_set_wait_limit: a rank that
+ * never arrives makes the kernel record JVP_ERR_DEVICE_TIMEOUT (read by
+ * jvp_attn_check_device_error) and return. Errors: JVP_ERR_INVALID_ARG for a
+ * null or out-of-range argument, JVP_ERR_MISALIGNED, JVP_ERR_LAUNCH_FAILED.
+ * Allocates nothing.
+ */
+int jvp_attn_signal_barrier(uint32_t* const* flags, int n_ranks, int rank, uint32_t epoch,
+                            void* stream);
 
 /*
  * jvp_attn_fwd_noalloc: jvp_attn_fwd for callers that cannot allocate

@@ -298,3 +298,31 @@ def test_scatter_argument_errors(kw, code):
 def test_scatter_valid_call_without_gpu_fails_cleanly():
     rc = call_scatter()
     assert rc in (_lib.JVP_ERR_LAUNCH_FAILED, _lib.JVP_ERR_UNSUPPORTED_DEVICE)
+
+
+def call_barrier(flags=(0x1000, 0x2000), n=None, rank=0, epoch=1):
+    n = len(flags) if n is None else n
+    arr = (ctypes.c_void_p * max(len(flags), 1))(*flags) if flags is not None else None
+    return _lib.lib().jvp_attn_signal_barrier(arr, n, rank, epoch, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(flags=None, n=2), _lib.JVP_ERR_INVALID_ARG),
+    (dict(n=0), _lib.JVP_ERR_INVALID_ARG),
+    (dict(flags=tuple(0x1000 * (i + 1) for i in range(9))), _lib.JVP_ERR_INVALID_ARG),
+    (dict(rank=2), _lib.JVP_ERR_INVALID_ARG),
+    (dict(rank=-1), _lib.JVP_ERR_INVALID_ARG),
+    (dict(flags=(0x1000, 0)), _lib.JVP_ERR_INVALID_ARG),
+    (dict(flags=(0x1000, 0x2002)), _lib.JVP_ERR_MISALIGNED),
+])
+def test_signal_barrier_argument_errors(kw, code):
+    assert call_barrier(**kw) == code
+
+
+def test_signal_barrier_valid_call_without_gpu_fails_cleanly():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    # valid arguments reach the device query, which fails without a GPU
+    rc = call_barrier()
+    assert rc in (_lib.JVP_ERR_UNSUPPORTED_DEVICE, _lib.JVP_ERR_LAUNCH_FAILED)
