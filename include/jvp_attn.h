@@ -289,11 +289,12 @@ int64_t jvp_attn_bwd_scratch_len(int B, int H, int L);
  * lse      [B, H, Lq] float32, natural log (output)
  * softmax_scale <= 0 selects 1/sqrt(d). Requires 1 <= Lk <= Lcache, Lq >= 1,
  * dtype JVP_BF16 (else JVP_ERR_INVALID_ARG) and d = 128 (else
- * JVP_ERR_UNSUPPORTED_HEAD_DIM); all pointers 16-byte aligned. When the
- * chunk has too few 128-row query tiles to fill the GPU the key range is
- * split across CTAs and a second kernel combines the splits; the library
- * keeps the partial-result workspace per (device, stream), grows it when a
- * larger call needs it (JVP_ERR_OUT_OF_MEMORY on failure) and frees it in
+ * JVP_ERR_UNSUPPORTED_HEAD_DIM); all pointers 16-byte aligned. The
+ * (b, h, 128-row query tile) items that fill whole waves of the GPU run
+ * whole; the items left over are cut into key ranges spread over the SMs,
+ * and a second kernel combines their partial results. The library keeps the
+ * partial-result workspace per (device, stream), grows it when a larger
+ * call needs it (JVP_ERR_OUT_OF_MEMORY on failure) and frees it in
  * jvp_attn_release. Asynchronous on `stream`; errors as jvp_attn_fwd.
  */
 int jvp_attn_cache_fwd(const void* q, const void* k_cache, const void* v_cache, void* o,

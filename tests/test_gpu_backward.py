@@ -114,7 +114,7 @@ def full_size_case(name):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name", ["tf", "chunk_tf"])
+@pytest.mark.parametrize("name", ["frame_causal", "tf", "chunk_tf", "tf_long"])
 def test_full_size_gq_on_sampled_rows(name):
     # The launch the backward bench times (all heads, full length); gQ of a
     # row depends only on that row's cotangent, so the oracle restricted to

@@ -75,6 +75,8 @@ CASES = [  # B, H, Lq, Lk, Lcache
     (2, 3, 5, 1000, 1003),       # tiny chunk, many splits
     (1, 2, 1560, 3120, 4000),    # one frame over two frames of context
     (1, 4, 4096, 2000, 2048),    # enough query tiles for no split
+    (1, 149, 128, 2000, 2000),   # one whole wave of 148 items, one leftover cut into pieces
+    (1, 100, 384, 1000, 1024),   # two whole waves, four leftover items cut in two
 ]
 
 
