@@ -33,6 +33,10 @@ CASES = [  # B, L, H, d, norm group ("C", "d" or None), rotate
     (1, 50, 2, 128, "d", False),
     (1, 20, 2, 128, None, True),
     (2, 9, 8, 32, None, False),
+    (1, 40, 16, 128, "d", True),   # 8 vectors per lane: the widest register-resident form
+    (1, 30, 24, 128, "C", True),   # H*d = 3072: the two-pass loop for wider layers
+    (1, 25, 2, 256, "d", True),    # d = 256: a head spans all 32 lanes
+    (2, 17, 32, 8, "d", True),     # d = 8: a head is one vector
 ]
 
 

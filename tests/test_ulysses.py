@@ -20,11 +20,11 @@ def free_port():
         return s.getsockname()[1]
 
 
-def problem(H=4, T=6, F=4, d=16, seed=3):
+def problem(B=1, H=4, T=6, F=4, d=16, seed=3):
     from oracle import MaskSpec, TEACHER_FORCING
     spec = MaskSpec(TEACHER_FORCING, T, F, 1)
     g = torch.Generator().manual_seed(seed)
-    xs = [torch.randn(1, H, spec.length, d, generator=g) for _ in range(6)]
+    xs = [torch.randn(B, H, spec.length, d, generator=g) for _ in range(6)]
     return spec, xs
 
 
@@ -38,7 +38,7 @@ def oracle_attn(spec):
     return attn
 
 
-def worker(rank, world, port, out):
+def worker(rank, world, B, port, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port),
                       RANK=str(rank), WORLD_SIZE=str(world))
     import datetime
@@ -47,7 +47,7 @@ def worker(rank, world, port, out):
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
     try:
-        spec, xs = problem()
+        spec, xs = problem(B=B)
         L, P = spec.length, world
         Ls, Hp = L // P, xs[0].shape[1] // P
         shard = [x[:, :, rank * Ls:(rank + 1) * Ls].contiguous() for x in xs]
@@ -62,13 +62,13 @@ def worker(rank, world, port, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 4])
-def test_ulysses_matches_single_process(world):
+@pytest.mark.parametrize("world,B", [(2, 1), (4, 1), (2, 2)])
+def test_ulysses_matches_single_process(world, B):
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
-    mp.start_processes(worker, args=(world, free_port(), out), nprocs=world,
+    mp.start_processes(worker, args=(world, B, free_port(), out), nprocs=world,
                        start_method="spawn", join=True)
-    spec, xs = problem()
+    spec, xs = problem(B=B)
     ro, rdo, rl = oracle_attn(spec)(*xs, None)
     Ls = spec.length // world
     for r in range(world):
