@@ -196,7 +196,6 @@ int get_partials(int dev, cudaStream_t st, size_t bytes, void** out) {
   return JVP_OK;
 }
 
-
 int get_counter(int dev, cudaStream_t st, unsigned** out) {
   std::lock_guard<std::mutex> lk(g_mu);
   const auto key = std::make_pair(dev, st);

@@ -57,14 +57,14 @@ def _shards(B, Ht, L, d, P, fill):
     return o, do, lse
 
 
-@pytest.mark.parametrize("P", [1, 2, 4])
+@pytest.mark.parametrize("P", [1, 2, 4, 8])
 @pytest.mark.parametrize("mode", [ja.TEACHER_FORCING, ja.FRAME_CAUSAL])
 def test_scatter_equals_token_slices(P, mode):
-    # 4 heads, TF: 2 x 3 frames x 100 tokens = 600 tokens; frame-causal: 6 x
-    # 100. Shards of 600 / P tokens: tile boundaries and shard boundaries
-    # do not line up.
+    # 4 heads (8 for 8 shards, the most the epilogue takes), TF: 2 x 3
+    # frames x 100 tokens = 600 tokens; frame-causal: 6 x 100. Shards of
+    # 600 / P tokens: tile boundaries and shard boundaries do not line up.
     F = 3 if mode == ja.TEACHER_FORCING else 6
-    w = Workload("scatter", 2, 4, 128, mode, 100, F, 1, "bf16", 0.1)
+    w = Workload("scatter", 2, max(4, P), 128, mode, 100, F, 1, "bf16", 0.1)
     xs, _ = make_inputs(w, device="cuda")
     mask = ja.Mask(w.mode, w.tokens_per_frame, w.n_frames, w.chunk)
     B, Ht, L, d = xs[0].shape

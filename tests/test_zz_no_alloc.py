@@ -113,3 +113,35 @@ def test_noalloc_refuses_a_capturing_stream():
     o2, do2, l2 = _outputs_of(lib.jvp_attn_fwd_noalloc, ins, w)
     assert torch.equal(o2, o) and torch.equal(do2, do) and torch.equal(l2, lse)
 
+
+def test_noalloc_at_its_largest_work_list():
+    # 255 frames of 1560 tokens under the teacher-forcing mask: 795,600
+    # tokens, whose work list takes 64,478 of the array's 65,472 words.
+    # Sampled rows (frame and half edges included) against the float64
+    # oracle; 260 frames (65,762 words) no longer fit.
+    from oracle import MaskSpec, jvp_attention_head
+    lib = _lib.lib()
+    w = Workload("na_max", 1, 1, 128, ja.TEACHER_FORCING, 1560, 255, 1, "bf16", 0.1)
+    ins, _ = make_inputs(w, device="cuda")
+    o, do, lse = _outputs_of(lib.jvp_attn_fwd_noalloc, ins, w)
+    FT = w.tokens_per_frame * w.n_frames
+    rng = np.random.default_rng(5)
+    rows = sorted(set(rng.choice(w.L, size=16, replace=False).tolist())
+                  | {0, 1559, 1560, FT - 1, FT, FT + 1559, w.L - 1})
+    spec = MaskSpec(w.mode, w.tokens_per_frame, w.n_frames, w.chunk)
+    ref_o, ref_do, ref_lse = jvp_attention_head(*(t[0, 0].cpu() for t in ins), spec, rows=rows)
+    idx = torch.as_tensor(rows, device="cuda")
+    for got, want in ((o[0, 0, idx], ref_o), (do[0, 0, idx], ref_do)):
+        g = got.float().cpu().numpy().astype(np.float64)
+        assert np.linalg.norm(g - want) <= 5e-3 * np.linalg.norm(want)
+        assert np.abs(g - want).max() <= 2e-2 * np.abs(want).max()
+    assert np.abs(lse[0, 0, idx].cpu().numpy() - ref_lse).max() <= 1e-3
+    fake = [0x1000] * 9  # never dereferenced: the size check comes first
+    big = w.with_(n_frames=260)
+    rc = lib.jvp_attn_fwd_noalloc(
+        *[ctypes.c_void_p(x) for x in fake[:8]],
+        ctypes.cast(ctypes.c_void_p(fake[8]), ctypes.POINTER(ctypes.c_float)),
+        1, 1, big.L, 128, _lib.JVP_BF16,
+        _lib.MaskDesc(big.mode, big.tokens_per_frame, big.n_frames, big.chunk), 0.0, None)
+    assert rc == _lib.JVP_ERR_TOO_LARGE
+
