@@ -7,15 +7,18 @@
 // Two persistent tcgen05 kernels over the same admissible-tile work lists:
 //  * dQ pass (query-stationary, 128 query rows per item, 64-key tiles):
 //      S = Q K^T, dP = G V^T   (N = 64; Q and G rows held in TMEM as the
-//                               A operands, K and V tiles from shared memory)
+//                               A operands, K and V tiles from shared memory;
+//                               three S parts, one dP part)
 //      softmax warps: P, dS    (one row per thread, bf16 dS back to TMEM)
 //      gQ += dS K              (A = dS in TMEM, N = 128, accumulator in TMEM)
 //    and it writes -LSE2 and -D_i per row pair to a scratch vector for the
 //    second pass.
 //  * dK/dV pass (key-stationary, 128 keys per item, 64-query tiles):
 //      S^T = K Q^T, dP^T = V G^T (both operands in shared memory: TMEM holds
-//                               the two accumulators and the S/dP buffers)
-//      softmax warps: P^T, dS^T (one key per thread; per-query LSE and D)
+//                               the two accumulators and two S/dP buffers)
+//      softmax warps: P^T, dS^T (one key per thread; per-query LSE and D
+//                               from the scratch, copied into shared memory
+//                               with each Q tile)
 //      gV += P^T G, gK += dS^T Q (A in TMEM, N = 128)
 // Warp roles: warp 0 TMA, warps 1 and 2 issue MMAs (whole warps, one
 // elected lane issuing), warps 4-11 two warpgroups taking 32 of each tile's
@@ -95,21 +98,35 @@ __device__ __forceinline__ void mma_ss4_elect(uint32_t d_tmem, uint64_t a0, uint
       : "memory");
 }
 
+// Plain bulk copy global -> shared, completing on an mbarrier (no tensor map,
+// no multicast): dst and src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 // Shared memory: the dK/dV pass's two stationary operands (A0, A1; the dQ
 // pass keeps its stationary Q and G in TMEM), then the streamed operands in
-// two rings X and Y. A streamed tile that feeds both the first and the
-// accumulating MMAs of a tile stays resident across two tiles (S(t+1) is
-// issued before acc(t)), so such a ring has 5 stages to keep two loads in
-// flight; V in the dQ pass feeds dP only and has 4.
+// two rings X and Y, and in the dK/dV pass each X stage's per-query slice
+// of the scratch (W: 32 row pairs {-LSE2, -LSE2, -D, -D}, 512 B), loaded
+// with the stage. Stages: dQ pass, K feeds S(t) and gQ(t) and S runs up to
+// three tiles ahead of gQ: 6; V feeds dP only: 4. dK/dV pass: Q and G feed
+// one first and one accumulating batch each, the first batch one tile ahead
+// of the accumulating one: 4 each.
 template <bool kKV>
 struct Layout {
-  static constexpr uint32_t NX = 5;            // dQ: K    dK/dV: Q
-  static constexpr uint32_t NY = kKV ? 5 : 4;  // dQ: V    dK/dV: G
+  static constexpr uint32_t NX = kKV ? 4 : 6;  // dQ: K    dK/dV: Q
+  static constexpr uint32_t NY = 4;            // dQ: V    dK/dV: G
   static constexpr uint32_t A0 = 0;
   static constexpr uint32_t A1 = kKV ? 2 * kRHalf : 0;
   static constexpr uint32_t X = kKV ? 4 * kRHalf : 0;
   static constexpr uint32_t Y = X + NX * kTile;
-  static constexpr uint32_t BAR = Y + NY * kTile;  // 144 KB (dQ) / 224 KB (dK/dV)
+  static constexpr uint32_t W = Y + NY * kTile;
+  static constexpr uint32_t BAR = W + (kKV ? NX * 512 : 0);  // 160 KB (dQ) / 194 KB (dK/dV)
   static constexpr uint32_t TMEM_SLOT = BAR + 8 * 44;
   static constexpr uint32_t ABORT = TMEM_SLOT + 4;
   static constexpr uint32_t RING = ABORT + 4;
@@ -120,27 +137,39 @@ static_assert(Layout<true>::kBytes <= 232448, "shared memory over the per-block 
 enum : uint32_t {
   B_AF = 0,      // stationary operands ready (TMA bytes, or TMEM rows stored)
   B_AE = 1,      // dK/dV: stationary smem operands may be overwritten (2 issuers)
-  B_XF = 2,      // 5
-  B_XE = 7,      // 5 (dK/dV pass: releases the X and the Y stage)
-  B_YF = 12,     // 5
-  B_YE = 17,     // 4 (dQ pass only)
-  B_SF = 21,     // 2: S and dP of a buffer complete (one commit per issuer)
-  B_PF = 23,     // 2: bf16 operands written by the softmax warps
-  B_MD = 25,     // accumulating MMAs of an item's last tile complete
-  B_CF = 26,     // accumulators read by the epilogue
-  B_DRAIN = 27,  // 2: one per issuer
-  B_IF = 29,     // 4: work-item ring
-  B_IE = 33,     // 4
-  kNumBars = 37
+  B_XF = 2,      // 6
+  B_XE = 8,      // 6 (dK/dV pass: releases the X and the Y stage)
+  B_YF = 14,     // 5
+  B_YE = 19,     // 4 (dQ pass only)
+  B_SF = 23,     // 3: S and dP of a buffer complete (one commit per issuer)
+  B_PF = 26,     // 3: bf16 operands written by the softmax warps
+  B_DR = 29,     // dQ pass: the softmax warps have read the dP part
+  B_MD = 30,     // accumulating MMAs of an item's last tile complete
+  B_CF = 31,     // accumulators read by the epilogue
+  B_DRAIN = 32,  // 2: one per issuer
+  B_IF = 34,     // 4: work-item ring
+  B_IE = 38,     // 4
+  kNumBars = 42
 };
 static_assert(Layout<false>::NY <= B_SF - B_YE, "Y-empty slots");
+static_assert(Layout<false>::NX <= B_XE - B_XF && Layout<false>::NX <= B_YF - B_XE, "X slots");
 static_assert(Layout<true>::NX == Layout<true>::NY, "dK/dV pass: X and Y stages pair up");
 static_assert(kNumBars <= 44, "barrier slots");
 static_assert(Layout<false>::RING + 16 <= Layout<false>::BAR + 512, "barrier area overflow");
 
-// TMEM columns: S/dP double buffer [0, 256) (buffer b at 128 b: S or S^T at
-// +0, dP or dP^T at +64), accumulators C0 and C1, and in the dQ pass the
-// stationary bf16 Q and G rows (A operands of the first MMAs) in place of C1.
+// TMEM columns [0, 256): dK/dV pass, two buffers (buffer b at 128 b: S^T at
+// +0, dP^T at +64); dQ pass, three S parts (part b at 64 b) and one dP part
+// at 192, since the softmax warps are done with dP as soon as they have
+// loaded it, while the S part holds dS until the accumulating MMAs have read
+// it. Then the accumulators C0 and C1, and in the dQ pass the stationary bf16
+// Q and G rows (A operands of the first MMAs) in place of C1.
+template <bool kKV> constexpr uint32_t kBufs = kKV ? 2 : 3;
+template <bool kKV> __device__ __forceinline__ uint32_t s_col(uint32_t b) {
+  return kKV ? 128u * b : 64u * b;
+}
+template <bool kKV> __device__ __forceinline__ uint32_t dp_col(uint32_t b) {
+  return kKV ? 128u * b + 64u : 192u;
+}
 constexpr uint32_t TM_C0 = 256;  // gQ, or gV
 constexpr uint32_t TM_C1 = 384;  // gK
 constexpr uint32_t TM_QA = 384;  // dQ pass: Q rows, 64 columns of bf16 pairs
@@ -233,11 +262,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       mbar_init(bar(B_YF + s), 1);
       if (!kKV) mbar_init(bar(B_YE + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (uint32_t b = 0; b < kBufs<kKV>; ++b) {
       mbar_init(bar(B_SF + b), 2);
       mbar_init(bar(B_PF + b), 2 * BR);
-      mbar_init(bar(B_DRAIN + b), 1);
     }
+    mbar_init(bar(B_DR), 2 * BR);
+    for (int b = 0; b < 2; ++b) mbar_init(bar(B_DRAIN + b), 1);
     mbar_init(bar(B_MD), kKV ? 2 : 1);
     mbar_init(bar(B_CF), 2 * BR);
     for (uint32_t i = 0; i < kRing; ++i) {
@@ -289,8 +319,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         const uint32_t sx = c.t % NX, ux = c.t / NX;
         if (c.t >= NX) ok = wait_bar(bar(B_XE + sx), (ux - 1) & 1u, p, abort_flag);
         if (!ok) break;
-        mbar_expect_tx(bar(B_XF + sx), kTile);
+        mbar_expect_tx(bar(B_XF + sx), kKV ? kTile + 512u : kTile);
         ++x_issued;
+        if (kKV)
+          bulk_load(base + LY::W + sx * 512u, p.sd + (size_t(c.bh) * p.Lp + y) * 2, 512u,
+                    bar(B_XF + sx));  // this tile's 64 queries: 16-byte aligned (y % 64 == 0)
         tma_load_3d(base + LY::X + sx * kTile, &tm_x, bar(B_XF + sx), 0, y, c.bh);
         tma_load_3d(base + LY::X + sx * kTile + kTHalf, &tm_x, bar(B_XF + sx), 64, y, c.bh);
         const uint32_t sy = c.t % NY, uy = c.t / NY;
@@ -335,30 +368,32 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       // First MMAs of tile t: S = A0 X^T (issuer A) or dP = A1 Y^T (issuer B).
       // ready: the stage barrier was already seen complete (a test this
       // thread ran during its previous accumulating MMAs).
-      auto issue_first = [&](const Cursor& c, bool s_mma, const Stage& st, bool ready) -> bool {
-        const uint32_t b = c.t & 1u;
+      // bs: the S/dP buffer of c.t (index and use parity).
+      auto issue_first = [&](const Cursor& c, bool s_mma, const Stage& st, const Stage& bs,
+                             bool ready) -> bool {
+        const uint32_t b = bs.s;
         if (c.j == 0 && !wait_w(bar(B_AF), c.item_idx & 1)) return false;
         uint32_t stage;
         uint64_t bdesc;
         if (s_mma) {
-          // Buffer b last held tile t-2: issuer A issued acc(t-2), which
-          // reads its S part, before this in its own order.
+          // dQ pass: S part b last held tile t-3; issuer A issued acc(t-3),
+          // which reads it, before this in its own order. dK/dV pass: the S^T
+          // part of buffer b, read by gV(t-2), likewise.
           stage = st.s;
           if (!__all_sync(0xffffffffu, ready) && !wait_w(bar(B_XF + stage), st.ph)) return false;
           bdesc = xk_desc + stage * (kTile >> 4);
         } else {
-          // dP(t) overwrites the dP part of buffer b. dQ pass: the softmax
-          // read dP(t-2) from it before publishing tile t-2 (acc reads only
-          // the S part there). dK/dV pass: gK(t-2), which reads dS^T from
-          // it, was issued by this thread first.
-          if (!kKV && c.t >= 2 && !wait_w(bar(B_PF + b), ((c.t >> 1) - 1) & 1u))
-            return false;
+          // dP(t) overwrites a dP part. dQ pass: the one dP part, once the
+          // softmax warps have loaded dP(t-1) from it (dS goes to the S
+          // part). dK/dV pass: gK(t-2), which reads dS^T from buffer b's dP
+          // part, was issued by this thread first.
+          if (!kKV && c.t >= 1 && !wait_w(bar(B_DR), (c.t - 1) & 1u)) return false;
           stage = st.s;
           if (!__all_sync(0xffffffffu, ready) && !wait_w(bar(B_YF + stage), st.ph)) return false;
           bdesc = yk_desc + stage * (kTile >> 4);
         }
         tc_fence_after();
-        const uint32_t d = tmem + b * 128u + (s_mma ? 0u : 64u);
+        const uint32_t d = tmem + (s_mma ? s_col<kKV>(b) : dp_col<kKV>(b));
         // k-steps 4h .. 4h+3 (head-dim columns [64 h, 64 h + 64), one
         // swizzled half of each operand), four MMAs per elect.
 #pragma unroll
@@ -391,18 +426,18 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       // latency overlaps the issue. A completed phase stays complete until
       // this thread has issued the MMAs that read the stage, and every
       // earlier use of the stage completed under this thread's own waits.
-      auto issue_acc = [&](const Cursor& c, bool s_part, const Stage& st, uint32_t next_bar,
-                           uint32_t next_ph, bool& next_ready) -> bool {
+      auto issue_acc = [&](const Cursor& c, bool s_part, const Stage& st, const Stage& bs,
+                           uint32_t next_bar, uint32_t next_ph, bool& next_ready) -> bool {
         // X stage of tile t; in the dK/dV pass (NX == NY) also its Y stage.
-        const uint32_t b = c.t & 1u, sx = st.s, sy = st.s;
+        const uint32_t b = bs.s, sx = st.s, sy = st.s;
         if (c.j == 0 && c.item_idx > 0 &&
             !wait_w(bar(B_CF), (c.item_idx - 1) & 1))
           return false;
-        if (!wait_w(bar(B_PF + b), (c.t >> 1) & 1u)) return false;
+        if (!wait_w(bar(B_PF + b), bs.ph)) return false;
         next_ready = next_bar != 0u && mbar_test(next_bar, next_ph);
         tc_fence_after();
         const uint32_t first = c.j == 0 ? 0u : 1u;
-        const uint32_t a_p = tmem + b * 128u + (s_part ? 0u : 64u);
+        const uint32_t a_p = tmem + (s_part ? s_col<kKV>(b) : dp_col<kKV>(b));
         // B operand: dQ pass K (X); dK/dV pass G (Y) for gV, Q (X) for gK.
         const uint64_t bm = (!kKV || !s_part) ? xm_desc + sx * (kTile >> 4)
                                               : ym_desc + sy * (kTile >> 4);
@@ -428,7 +463,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         // pass) are stored only after this item's epilogue, which waits for
         // this item's last acc.
         Cursor cs, ca;
-        Stage ss, sa;  // X stages of cs.t and ca.t
+        Stage ss, sa;    // X stages of cs.t and ca.t
+        Stage bss, bsa;  // S/dP buffers of cs.t and ca.t
         cs.start(p, ring, kConsumerWarp);
         ca.start(p, ring, kConsumerWarp);
         // Failure-detection test: wait on the drain barrier's first phase,
@@ -437,46 +473,52 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         if (p.stall_test) ok = __all_sync(0xffffffffu, wait_bar(bar(B_DRAIN + 0), 0u, p, abort_flag));
         bool xr = false;  // XF of cs.t seen complete
         while (ok && ca.valid) {
-          while (ok && cs.valid && cs.t < ca.t + 2 && cs.item_idx == ca.item_idx) {
-            ok = issue_first(cs, true, ss, xr);
+          while (ok && cs.valid && cs.t < ca.t + kBufs<kKV> && cs.item_idx == ca.item_idx) {
+            ok = issue_first(cs, true, ss, bss, xr);
             xr = false;
             cs.next(p, ring, kConsumerWarp);
             ss.step(NX);
+            bss.step(kBufs<kKV>);
           }
           if (!ok) break;
-          ok = issue_acc(ca, true, sa, cs.valid ? bar(B_XF + ss.s) : 0u, ss.ph, xr);
+          ok = issue_acc(ca, true, sa, bsa, cs.valid ? bar(B_XF + ss.s) : 0u, ss.ph, xr);
           ca.next(p, ring, kConsumerWarp);
           sa.step(NX);
+          bsa.step(kBufs<kKV>);
         }
       } else if (!kKV) {
         // dP of every tile, as soon as its buffer part is free.
         Cursor c;
-        Stage sc;  // Y stage of c.t
+        Stage sc, bsc;  // Y stage and S/dP buffer of c.t
         c.start(p, ring, kConsumerWarp);
         while (c.valid && ok) {
-          ok = issue_first(c, false, sc, false);
+          ok = issue_first(c, false, sc, bsc, false);
           c.next(p, ring, kConsumerWarp);
           sc.step(NY);
+          bsc.step(kBufs<kKV>);
         }
       } else {
         // gK(t), then dP^T(t+2) in this thread's order (it overwrites the dP
         // part gK(t) reads), as issuer A does with the S part.
         Cursor cd, ck;
-        Stage sd, sk;  // stages (X and Y alike) of cd.t and ck.t
+        Stage sd, sk;    // stages (X and Y alike) of cd.t and ck.t
+        Stage bsd, bsk;  // S/dP buffers of cd.t and ck.t
         cd.start(p, ring, kConsumerWarp);
         ck.start(p, ring, kConsumerWarp);
         bool yr = false;  // YF of cd.t seen complete
         while (ok && ck.valid) {
-          while (ok && cd.valid && cd.t < ck.t + 2 && cd.item_idx == ck.item_idx) {
-            ok = issue_first(cd, false, sd, yr);
+          while (ok && cd.valid && cd.t < ck.t + kBufs<kKV> && cd.item_idx == ck.item_idx) {
+            ok = issue_first(cd, false, sd, bsd, yr);
             yr = false;
             cd.next(p, ring, kConsumerWarp);
             sd.step(NY);
+            bsd.step(kBufs<kKV>);
           }
           if (!ok) break;
-          ok = issue_acc(ck, false, sk, cd.valid ? bar(B_YF + sd.s) : 0u, sd.ph, yr);
+          ok = issue_acc(ck, false, sk, bsk, cd.valid ? bar(B_YF + sd.s) : 0u, sd.ph, yr);
           ck.next(p, ring, kConsumerWarp);
           sk.step(NX);
+          bsk.step(kBufs<kKV>);
         }
       }
       if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
@@ -495,6 +537,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
     const int chunk = p.mask.chunk < 1 ? 1 : p.mask.chunk;
     const float kLog2e = 1.4426950408889634f;
     Cursor c;
+    Stage bsm;  // S/dP buffer of c.t
     c.start(p, ring, kConsumerWarp);
     RowKeys rk{0, 0, 0, 0};
     int grow = 0;
@@ -571,23 +614,33 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       // Column indices of this thread's 32 elements: keys (dQ pass) or
       // queries (dK/dV pass) [col0, col0 + 32).
       const int col0 = c.kt * BT + 32 * hw;
-      // dK/dV pass: -LSE2 and -D of the 32 queries as 16 row pairs, the same
-      // for every lane (col0 + 32 <= Lp; 16-byte aligned as col0 and Lp are even).
-      float4 w[16];
+      // dK/dV pass: -LSE2 and -D of this warpgroup's 32 queries, 16 query
+      // pairs of {-LSE2 pair, -D pair} (two packed fp32 pairs each, the same
+      // for every lane), read from the tile's shared-memory slice where they
+      // are used.
+      const ulonglong2* wsrc = nullptr;
       if (kKV) {
-        const float4* src =
-            reinterpret_cast<const float4*>(p.sd + (size_t(c.bh) * p.Lp + col0) * 2);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = __ldg(src + i);
+        // The slice arrived with the tile's Q stage; that stage's barrier is
+        // still in this tile's phase (the stage is reloaded only after this
+        // tile's accumulating MMAs, which wait for these warps).
+        const uint32_t sx = c.t % NX;
+        ok = wait_bar(bar(B_XF + sx), (c.t / NX) & 1u, p, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        wsrc = reinterpret_cast<const ulonglong2*>(base_ptr + LY::W + sx * 512u) + 16 * hw;
       }
-      const uint32_t b = c.t & 1u;
-      ok = wait_bar(bar(B_SF + b), (c.t >> 1) & 1u, p, abort_flag);
+      const uint32_t b = bsm.s;
+      ok = wait_bar(bar(B_SF + b), bsm.ph, p, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       uint32_t sr[32], dr[32];
-      tmem_ld32(tl + b * 128u + 32u * hw, sr);
-      tmem_ld32(tl + b * 128u + 64u + 32u * hw, dr);
+      tmem_ld32(tl + s_col<kKV>(b) + 32u * hw, sr);
+      tmem_ld32(tl + dp_col<kKV>(b) + 32u * hw, dr);
       tmem_wait_ld();
+      if (!kKV) {
+        // dQ pass: the dP part may take the next tile's dP.
+        tc_fence_before();
+        mbar_arrive(bar(B_DR));
+      }
       uint32_t pp[16], pd[16];
       // Elements (2i, 2i+1) as one packed fp32 pair: P = 2^(c2 S - LSE2),
       // dS = P (dP - D), each rounded as the scalar expression would be;
@@ -595,8 +648,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       const uint64_t c2v = f2pack(p.c2, p.c2);
       const uint64_t nl_row = f2pack(-lse2, -lse2), nd_row = f2pack(-dval, -dval);  // dQ pass
       auto pair = [&](int i, bool masked) {
-        const uint64_t nl = kKV ? f2pack(w[i].x, w[i].y) : nl_row;
-        const uint64_t nd = kKV ? f2pack(w[i].z, w[i].w) : nd_row;
+        ulonglong2 wv = make_ulonglong2(nl_row, nd_row);
+        if (kKV) wv = wsrc[i];
+        const uint64_t nl = wv.x, nd = wv.y;
         float x0, x1, e0, e1, d0, d1;
         f2unpack(fma2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), c2v, nl),
                  x0, x1);
@@ -621,10 +675,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         for (int i = 0; i < 16; ++i) pair(i, false);
       }
       if (!kKV) {
-        tmem_st16(tl + b * 128u + 32u * hw, pd);  // dS over this warpgroup's S columns
+        tmem_st16(tl + s_col<kKV>(b) + 32u * hw, pd);  // dS over this warpgroup's S columns
       } else {
-        tmem_st16(tl + b * 128u + 32u * hw, pp);        // P^T over its S^T columns
-        tmem_st16(tl + b * 128u + 64u + 32u * hw, pd);  // dS^T over its dP^T columns
+        tmem_st16(tl + s_col<kKV>(b) + 32u * hw, pp);   // P^T over its S^T columns
+        tmem_st16(tl + dp_col<kKV>(b) + 32u * hw, pd);  // dS^T over its dP^T columns
       }
       tmem_wait_st();
       tc_fence_before();
@@ -670,6 +724,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         mbar_arrive(bar(B_CF));
       }
       c.next(p, ring, kConsumerWarp);
+      bsm.step(kBufs<kKV>);
     }
   }
 
