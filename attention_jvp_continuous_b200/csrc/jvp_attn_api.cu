@@ -374,7 +374,7 @@ int jvp_attn_bwd(const void* q, const void* k, const void* v, const void* o, con
   a.wait_limit_ns = wait_limit_ns();
   a.stall_test = stall_test();
   WorkList wq, wkv;
-  rc = get_worklist(dev, mask, L, &wq, 128, 64, 0);
+  rc = get_worklist(dev, mask, L, &wq, 128, 128, 0);
   if (rc != JVP_OK) return rc;
   rc = get_worklist(dev, mask, L, &wkv, 64, 128, 1);
   if (rc != JVP_OK) return rc;

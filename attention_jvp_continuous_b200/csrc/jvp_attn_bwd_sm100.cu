@@ -5,10 +5,9 @@
 //   dP = G V^T,  dS = P o (dP - D),  gQ = c dS K,  gK = c dS^T Q,  gV = P^T G.
 //
 // Two persistent tcgen05 kernels over the same admissible-tile work lists:
-//  * dQ pass (query-stationary, 128 query rows per item, 64-key tiles):
-//      S = Q K^T, dP = G V^T   (N = 64; Q and G rows held in TMEM as the
-//                               A operands, K and V tiles from shared memory;
-//                               three S parts, one dP part)
+//  * dQ pass (query-stationary, 128 query rows per item, 128-key tiles):
+//      S = Q K^T, dP = G V^T   (N = 128, both operands in shared memory; two
+//                               S parts and one dP part in TMEM)
 //      softmax warps: P, dS    (one row per thread, bf16 dS back to TMEM)
 //      gQ += dS K              (A = dS in TMEM, N = 128, accumulator in TMEM)
 //    and it writes -LSE2 and -D_i per row pair to a scratch vector for the
@@ -49,13 +48,14 @@ using pipe::kRing;
 using pipe::wait_bar;
 
 constexpr int BR = 128;  // stationary rows per item (TMEM lanes)
-constexpr int BT = 64;   // streamed rows per tile
 constexpr int D = 128;
 constexpr int kThreads = 384;
+// Streamed rows per tile: 128 keys (dQ pass), 64 queries (dK/dV pass).
+template <bool kKV> constexpr int kBT = kKV ? 64 : 128;
 
 constexpr uint32_t kRHalf = BR * 128;  // 16 KB: 128 rows x 64 head-dim columns
-constexpr uint32_t kTHalf = BT * 128;  //  8 KB: 64 rows x 64 columns
-constexpr uint32_t kTile = 2 * kTHalf; // 16 KB: one streamed 64-row operand
+template <bool kKV> constexpr uint32_t kTHalf = kBT<kKV> * 128;  // rows x 64 columns
+template <bool kKV> constexpr uint32_t kTile = 2 * kTHalf<kKV>;   // one streamed operand
 // Readers of the work-item ring: issuer A's two cursors, issuer B's one (dQ)
 // or two (dK/dV), 8 softmax warps.
 template <bool kKV> constexpr uint32_t kReaders = (kKV ? 4 : 3) + 8;
@@ -109,34 +109,35 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-// Shared memory: the dK/dV pass's two stationary operands (A0, A1; the dQ
-// pass keeps its stationary Q and G in TMEM), then the streamed operands in
-// two rings X and Y, and in the dK/dV pass each X stage's per-query slice
-// of the scratch (W: 32 row pairs {-LSE2, -LSE2, -D, -D}, 512 B), loaded
-// with the stage. Stages: dQ pass, K feeds S(t) and gQ(t) and S runs up to
-// three tiles ahead of gQ: 6; V feeds dP only: 4. dK/dV pass: Q and G feed
-// one first and one accumulating batch each, the first batch one tile ahead
-// of the accumulating one: 4 each.
+// Shared memory: the item's two stationary operands (A0, A1: Q and G, or K
+// and V, 32 KB each), then the streamed operands in two rings X and Y, and
+// in the dK/dV pass each X stage's per-query slice of the scratch (W: 32 row
+// pairs {-LSE2, -LSE2, -D, -D}, 512 B), loaded with the stage. Stages: dQ
+// pass (32 KB tiles of 128 keys), K feeds S(t) and gQ(t), S one tile ahead
+// of gQ: 3; V feeds dP only: 2. dK/dV pass (16 KB tiles of 64 queries): Q
+// and G feed one first and one accumulating batch each, the first batch one
+// tile ahead of the accumulating one: 4 each.
 template <bool kKV>
 struct Layout {
-  static constexpr uint32_t NX = kKV ? 4 : 6;  // dQ: K    dK/dV: Q
-  static constexpr uint32_t NY = 4;            // dQ: V    dK/dV: G
+  static constexpr uint32_t NX = kKV ? 4 : 3;  // dQ: K    dK/dV: Q
+  static constexpr uint32_t NY = kKV ? 4 : 2;  // dQ: V    dK/dV: G
   static constexpr uint32_t A0 = 0;
-  static constexpr uint32_t A1 = kKV ? 2 * kRHalf : 0;
-  static constexpr uint32_t X = kKV ? 4 * kRHalf : 0;
-  static constexpr uint32_t Y = X + NX * kTile;
-  static constexpr uint32_t W = Y + NY * kTile;
-  static constexpr uint32_t BAR = W + (kKV ? NX * 512 : 0);  // 160 KB (dQ) / 194 KB (dK/dV)
+  static constexpr uint32_t A1 = 2 * kRHalf;
+  static constexpr uint32_t X = 4 * kRHalf;
+  static constexpr uint32_t Y = X + NX * kTile<kKV>;
+  static constexpr uint32_t W = Y + NY * kTile<kKV>;
+  static constexpr uint32_t BAR = W + (kKV ? NX * 512 : 0);  // 224 KB (dQ) / 194 KB (dK/dV)
   static constexpr uint32_t TMEM_SLOT = BAR + 8 * 44;
   static constexpr uint32_t ABORT = TMEM_SLOT + 4;
   static constexpr uint32_t RING = ABORT + 4;
   static constexpr uint32_t kBytes = BAR + 512 + 1024;  // + alignment slack
 };
-static_assert(Layout<true>::kBytes <= 232448, "shared memory over the per-block limit");
+static_assert(Layout<true>::kBytes <= 232448 && Layout<false>::kBytes <= 232448,
+              "shared memory over the per-block limit");
 
 enum : uint32_t {
-  B_AF = 0,      // stationary operands ready (TMA bytes, or TMEM rows stored)
-  B_AE = 1,      // dK/dV: stationary smem operands may be overwritten (2 issuers)
+  B_AF = 0,      // stationary operands ready (TMA bytes)
+  B_AE = 1,      // stationary operands may be overwritten (2 issuers)
   B_XF = 2,      // 6
   B_XE = 8,      // 6 (dK/dV pass: releases the X and the Y stage)
   B_YF = 14,     // 5
@@ -157,26 +158,23 @@ static_assert(Layout<true>::NX == Layout<true>::NY, "dK/dV pass: X and Y stages 
 static_assert(kNumBars <= 44, "barrier slots");
 static_assert(Layout<false>::RING + 16 <= Layout<false>::BAR + 512, "barrier area overflow");
 
-// TMEM columns [0, 256): dK/dV pass, two buffers (buffer b at 128 b: S^T at
-// +0, dP^T at +64); dQ pass, three S parts (part b at 64 b) and one dP part
-// at 192, since the softmax warps are done with dP as soon as they have
-// loaded it, while the S part holds dS until the accumulating MMAs have read
-// it. Then the accumulators C0 and C1, and in the dQ pass the stationary bf16
-// Q and G rows (A operands of the first MMAs) in place of C1.
-template <bool kKV> constexpr uint32_t kBufs = kKV ? 2 : 3;
-template <bool kKV> __device__ __forceinline__ uint32_t s_col(uint32_t b) {
-  return kKV ? 128u * b : 64u * b;
-}
+// TMEM columns. dQ pass: two 128-column S parts (part b at 128 b) and one
+// dP part at 256, since the softmax warps are done with dP as soon as they
+// have loaded it, while an S part holds dS until the accumulating MMAs have
+// read it; gQ at 384. dK/dV pass: two buffers (buffer b at 128 b: S^T at +0,
+// dP^T at +64), gV at 256 and gK at 384.
+template <bool kKV> constexpr uint32_t kBufs = 2;
+template <bool kKV> __device__ __forceinline__ uint32_t s_col(uint32_t b) { return 128u * b; }
 template <bool kKV> __device__ __forceinline__ uint32_t dp_col(uint32_t b) {
-  return kKV ? 128u * b + 64u : 192u;
+  return kKV ? 128u * b + 64u : 256u;
 }
-constexpr uint32_t TM_C0 = 256;  // gQ, or gV
+template <bool kKV> constexpr uint32_t kC0 = kKV ? 256u : 384u;  // gV, or gQ
 constexpr uint32_t TM_C1 = 384;  // gK
-constexpr uint32_t TM_QA = 384;  // dQ pass: Q rows, 64 columns of bf16 pairs
-constexpr uint32_t TM_GA = 448;  // dQ pass: G rows
 
-constexpr uint32_t IDESC_N64 = ptx::idesc_bf16(BR, BT, false, false);  // 128 x 64, K-major B
-constexpr uint32_t IDESC_MN = ptx::idesc_bf16(BR, D, false, true);     // 128 x 128, MN-major B
+// First MMAs: 128 x 128 (dQ pass) or 128 x 64 (dK/dV pass), K-major B.
+template <bool kKV>
+constexpr uint32_t kIdescFirst = ptx::idesc_bf16(BR, kBT<kKV>, false, false);
+constexpr uint32_t IDESC_MN = ptx::idesc_bf16(BR, D, false, true);  // 128 x 128, MN-major B
 
 struct Params {
   const int4* qtiles;  // work entries {outer tile, seg_begin, seg_count, inner tiles}
@@ -192,8 +190,8 @@ struct Params {
   // written by the dQ pass (rows past L: LSE2 = +inf, D = 0), read by the
   // dK/dV pass as packed fp32 pairs.
   float* sd;
-  const __nv_bfloat16* q;  // dQ pass: stationary rows, stored into TMEM
-  const __nv_bfloat16* g;  // cotangent: stationary rows and D (dQ pass)
+  const __nv_bfloat16* q;  // query rows
+  const __nv_bfloat16* g;  // cotangent rows, for D (dQ pass)
   const __nv_bfloat16* o;  // forward output, for D (dQ pass)
   __nv_bfloat16* out0;     // gQ (dQ pass) or gK (dK/dV pass)
   __nv_bfloat16* out1;     // gV (dK/dV pass)
@@ -222,9 +220,9 @@ struct Stage {
 // through completions, so the warp that reads a TMEM part in tile t's
 // accumulating MMAs is the one that overwrites it at tile t+2:
 //   dQ pass:    issuer A (warp 1): gQ(t) once the softmax warps have written
-//               tile t's dS into the S part, then S(t+2) = A0 X(t+2)^T into
-//               that part; issuer B (warp 2): dP(t) = A1 Y(t)^T into the dP
-//               part of buffer t&1 once the softmax has read dP(t-2) there.
+//               tile t's dS into S part t&1, then S(t+2) = A0 X(t+2)^T into
+//               that part; issuer B (warp 2): dP(t) = A1 Y(t)^T into the one
+//               dP part once the softmax warps have loaded dP(t-1) from it.
 //   dK/dV pass: issuer A: gV(t) (P^T, S part) then S^T(t+2); issuer B:
 //               gK(t) (dS^T, dP part) then dP^T(t+2).
 // One thread's MMAs run in issue order; every hand-over between the issuers
@@ -234,10 +232,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
            const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
            const __grid_constant__ Params p) {
-  // dQ pass:  A0 = Q, A1 = G (stationary, TMEM);  X = K, Y = V (smem rings).
-  // dK/dV:    A0 = K, A1 = V (stationary, smem);  X = Q, Y = G.
+  // dQ pass:  A0 = Q, A1 = G (stationary);  X = K, Y = V (rings).
+  // dK/dV:    A0 = K, A1 = V (stationary);  X = Q, Y = G.
   using LY = Layout<kKV>;
   constexpr uint32_t NX = LY::NX, NY = LY::NY;
+  constexpr int BT = kBT<kKV>;
+  constexpr uint32_t kTH = kTHalf<kKV>, kTL = kTile<kKV>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -249,7 +249,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
 
   if (threadIdx.x == 0) {
     // dQ: the 256 softmax threads store Q / G rows and arrive; dK/dV: TMA bytes.
-    mbar_init(bar(B_AF), kKV ? 1 : 2 * BR);
+    mbar_init(bar(B_AF), 1);
     mbar_init(bar(B_AE), 2);
     // dK/dV pass: a stage pair (Q and G of one tile) is released and an
     // item's accumulation is complete once both issuers have committed
@@ -278,10 +278,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    if (kKV) {
-      tma_prefetch_map(&tm_a0);
-      tma_prefetch_map(&tm_a1);
-    }
+    tma_prefetch_map(&tm_a0);
+    tma_prefetch_map(&tm_a1);
     tma_prefetch_map(&tm_x);
     tma_prefetch_map(&tm_y);
   }
@@ -304,7 +302,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       uint32_t a_armed = 0, x_issued = 0, y_issued = 0;
       bool ok = true;
       while (c.valid && ok) {
-        if (kKV && c.j == 0) {
+        if (c.j == 0) {
           if (c.item_idx > 0) ok = wait_bar(bar(B_AE), (c.item_idx - 1) & 1, p, abort_flag);
           if (!ok) break;
           mbar_expect_tx(bar(B_AF), 4 * kRHalf);
@@ -319,20 +317,20 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         const uint32_t sx = c.t % NX, ux = c.t / NX;
         if (c.t >= NX) ok = wait_bar(bar(B_XE + sx), (ux - 1) & 1u, p, abort_flag);
         if (!ok) break;
-        mbar_expect_tx(bar(B_XF + sx), kKV ? kTile + 512u : kTile);
+        mbar_expect_tx(bar(B_XF + sx), kKV ? kTL + 512u : kTL);
         ++x_issued;
         if (kKV)
           bulk_load(base + LY::W + sx * 512u, p.sd + (size_t(c.bh) * p.Lp + y) * 2, 512u,
                     bar(B_XF + sx));  // this tile's 64 queries: 16-byte aligned (y % 64 == 0)
-        tma_load_3d(base + LY::X + sx * kTile, &tm_x, bar(B_XF + sx), 0, y, c.bh);
-        tma_load_3d(base + LY::X + sx * kTile + kTHalf, &tm_x, bar(B_XF + sx), 64, y, c.bh);
+        tma_load_3d(base + LY::X + sx * kTL, &tm_x, bar(B_XF + sx), 0, y, c.bh);
+        tma_load_3d(base + LY::X + sx * kTL + kTH, &tm_x, bar(B_XF + sx), 64, y, c.bh);
         const uint32_t sy = c.t % NY, uy = c.t / NY;
         if (!kKV && c.t >= NY) ok = wait_bar(bar(B_YE + sy), (uy - 1) & 1u, p, abort_flag);
         if (!ok) break;
-        mbar_expect_tx(bar(B_YF + sy), kTile);
+        mbar_expect_tx(bar(B_YF + sy), kTL);
         ++y_issued;
-        tma_load_3d(base + LY::Y + sy * kTile, &tm_y, bar(B_YF + sy), 0, y, c.bh);
-        tma_load_3d(base + LY::Y + sy * kTile + kTHalf, &tm_y, bar(B_YF + sy), 64, y, c.bh);
+        tma_load_3d(base + LY::Y + sy * kTL, &tm_y, bar(B_YF + sy), 0, y, c.bh);
+        tma_load_3d(base + LY::Y + sy * kTL + kTH, &tm_y, bar(B_YF + sy), 64, y, c.bh);
         c.next(p, ring, kProducer);
       }
       if (!ok || *abort_flag) {
@@ -362,9 +360,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       const uint64_t a0_desc = sdesc_sw128(base + LY::A0, 16, 1024);
       const uint64_t a1_desc = sdesc_sw128(base + LY::A1, 16, 1024);
       const uint64_t xk_desc = sdesc_sw128(base + LY::X, 16, 1024);       // K-major view
-      const uint64_t xm_desc = sdesc_sw128(base + LY::X, kTHalf, 1024);   // MN-major view
+      const uint64_t xm_desc = sdesc_sw128(base + LY::X, kTH, 1024);      // MN-major view
       const uint64_t yk_desc = sdesc_sw128(base + LY::Y, 16, 1024);
-      const uint64_t ym_desc = sdesc_sw128(base + LY::Y, kTHalf, 1024);
+      const uint64_t ym_desc = sdesc_sw128(base + LY::Y, kTH, 1024);
       // First MMAs of tile t: S = A0 X^T (issuer A) or dP = A1 Y^T (issuer B).
       // ready: the stage barrier was already seen complete (a test this
       // thread ran during its previous accumulating MMAs).
@@ -376,12 +374,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         uint32_t stage;
         uint64_t bdesc;
         if (s_mma) {
-          // dQ pass: S part b last held tile t-3; issuer A issued acc(t-3),
-          // which reads it, before this in its own order. dK/dV pass: the S^T
-          // part of buffer b, read by gV(t-2), likewise.
+          // S part b (dQ pass) or buffer b's S^T part (dK/dV pass) last held
+          // tile t-2; issuer A issued acc(t-2), which reads it, before this
+          // in its own order.
           stage = st.s;
           if (!__all_sync(0xffffffffu, ready) && !wait_w(bar(B_XF + stage), st.ph)) return false;
-          bdesc = xk_desc + stage * (kTile >> 4);
+          bdesc = xk_desc + stage * (kTL >> 4);
         } else {
           // dP(t) overwrites a dP part. dQ pass: the one dP part, once the
           // softmax warps have loaded dP(t-1) from it (dS goes to the S
@@ -390,7 +388,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
           if (!kKV && c.t >= 1 && !wait_w(bar(B_DR), (c.t - 1) & 1u)) return false;
           stage = st.s;
           if (!__all_sync(0xffffffffu, ready) && !wait_w(bar(B_YF + stage), st.ph)) return false;
-          bdesc = yk_desc + stage * (kTile >> 4);
+          bdesc = yk_desc + stage * (kTL >> 4);
         }
         tc_fence_after();
         const uint32_t d = tmem + (s_mma ? s_col<kKV>(b) : dp_col<kKV>(b));
@@ -398,28 +396,24 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         // swizzled half of each operand), four MMAs per elect.
 #pragma unroll
         for (int h = 0; h < D / 64; ++h) {
-          const uint64_t bh = bdesc + ((h * kTHalf) >> 4);
-          if (!kKV) {
-            const uint32_t ah = tmem + (s_mma ? TM_QA : TM_GA) + 32u * h;
-            mma_ts4_elect(d, ah, ah + 8u, ah + 16u, ah + 24u, bh, bh + 2, bh + 4, bh + 6, IDESC_N64,
-                          h > 0);
-          } else {
-            const uint64_t ah = (s_mma ? a0_desc : a1_desc) + ((h * kRHalf) >> 4);
-            mma_ss4_elect(d, ah, ah + 2, ah + 4, ah + 6, bh, bh + 2, bh + 4, bh + 6, IDESC_N64, h > 0);
-          }
+          const uint64_t bh = bdesc + ((h * kTH) >> 4);
+          const uint64_t ah = (s_mma ? a0_desc : a1_desc) + ((h * kRHalf) >> 4);
+          mma_ss4_elect(d, ah, ah + 2, ah + 4, ah + 6, bh, bh + 2, bh + 4, bh + 6, kIdescFirst<kKV>,
+                        h > 0);
         }
         mma_commit_elect(bar(B_SF + b));
         if (!s_mma && !kKV) mma_commit_elect(bar(B_YE + stage));  // dQ pass: V feeds dP only
-        if (kKV && c.j == c.n - 1) mma_commit_elect(bar(B_AE));   // done with A0 (S) / A1 (dP)
+        if (c.j == c.n - 1) mma_commit_elect(bar(B_AE));   // done with A0 (S) / A1 (dP)
         return true;
       };
-      // Accumulating MMAs. The bf16 operands of a tile sit in TMEM columns
-      // {0, 8} and {32, 40} (one pair of 16-wide k-steps per warpgroup) of
-      // the S part (dQ pass: dS; dK/dV pass: P^T) and, dK/dV pass, of the dP
-      // part (dS^T). dQ pass: gQ += dS K, issuer A. dK/dV pass: gV += P^T G
-      // by issuer A (it reads the S part), gK += dS^T Q by issuer B (the dP
-      // part), each followed in its own thread by the first MMA that
-      // overwrites that part two tiles later.
+      // Accumulating MMAs. The bf16 operands of a tile sit at the start of
+      // each 32-column step of S columns the softmax warps read (k-step ks at
+      // column 32 (ks >> 1) + 8 (ks & 1)) in the S part (dQ pass: dS; dK/dV
+      // pass: P^T) and, dK/dV pass, in the dP part (dS^T). dQ pass: gQ += dS
+      // K, issuer A. dK/dV pass: gV += P^T G by issuer A (it reads the S
+      // part), gK += dS^T Q by issuer B (the dP part), each followed in its
+      // own thread by the first MMA that overwrites that part two tiles
+      // later.
       // next_bar / next_ph: the stage barrier of this issuer's next first
       // MMAs (0: none). It is tested here, before this tile's MMAs are
       // issued, and the result is used only after them, so the test's
@@ -439,13 +433,16 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         const uint32_t first = c.j == 0 ? 0u : 1u;
         const uint32_t a_p = tmem + (s_part ? s_col<kKV>(b) : dp_col<kKV>(b));
         // B operand: dQ pass K (X); dK/dV pass G (Y) for gV, Q (X) for gK.
-        const uint64_t bm = (!kKV || !s_part) ? xm_desc + sx * (kTile >> 4)
-                                              : ym_desc + sy * (kTile >> 4);
-        const uint32_t acc = (!kKV || s_part) ? TM_C0 : TM_C1;
-        // k-steps 0..3: TMEM columns {0, 8, 32, 40}; B rows 16 ks.
-        static_assert(BT == 64, "four accumulating k-steps per tile");
+        const uint64_t bm = (!kKV || !s_part) ? xm_desc + sx * (kTL >> 4)
+                                              : ym_desc + sy * (kTL >> 4);
+        const uint32_t acc = (!kKV || s_part) ? kC0<kKV> : TM_C1;
+        // k-step ks of 16 streamed rows: A columns 32 (ks >> 1) + 8 (ks & 1),
+        // B rows 16 ks (eight steps in the dQ pass, four in the dK/dV pass).
         mma_ts4_elect(tmem + acc, a_p, a_p + 8u, a_p + 32u, a_p + 40u, bm, bm + 128, bm + 256,
                       bm + 384, IDESC_MN, first);
+        if (!kKV)
+          mma_ts4_elect(tmem + acc, a_p + 64u, a_p + 72u, a_p + 96u, a_p + 104u, bm + 512,
+                        bm + 640, bm + 768, bm + 896, IDESC_MN, 1u);
         // Stage release: dQ pass, this thread read X(t) (also with S(t),
         // earlier) and Y(t) only through dP(t); dK/dV pass, both issuers
         // commit to the pair's one barrier (X and Y feed one MMA batch of
@@ -459,9 +456,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       if (issuer_a) {
         // acc(t), then S(t+2) in this thread's order: S(t+2) overwrites the
         // S part of the buffer acc(t) reads. S runs up to two tiles ahead of
-        // acc but not into the next item: that item's stationary rows (dQ
-        // pass) are stored only after this item's epilogue, which waits for
-        // this item's last acc.
+        // acc but not into the next item, whose stationary operands are
+        // loaded once both issuers are done with this item's.
         Cursor cs, ca;
         Stage ss, sa;    // X stages of cs.t and ca.t
         Stage bss, bsa;  // S/dP buffers of cs.t and ca.t
@@ -578,42 +574,15 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
             sdp[0] = -lse2;
             sdp[2] = -dval;
           }
-          // The item's stationary rows into TMEM, as bf16 pairs (the A
-          // operands of the first MMAs): warpgroup 0 stores Q, warpgroup 1
-          // G; rows past L are zero. The previous item's S and dP MMAs all
-          // completed before its last tile reached these warps, and neither
-          // issuer starts this item's before B_AF completes.
-          const __nv_bfloat16* src = hw == 0 ? p.q : p.g;
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t rv[32];
-            if (grow < p.L) {
-              const uint4* s4 = reinterpret_cast<const uint4*>(src + roff * D) + half * 8;
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const uint4 v4 = s4[i];
-                rv[4 * i] = v4.x;
-                rv[4 * i + 1] = v4.y;
-                rv[4 * i + 2] = v4.z;
-                rv[4 * i + 3] = v4.w;
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) rv[i] = 0u;
-            }
-            tmem_st32(tl + (hw == 0 ? TM_QA : TM_GA) + 32u * half, rv);
-          }
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(bar(B_AF));
         } else {
           rk = key_queries(p.mask.mode, p.mask.tokens_per_frame, p.mask.n_frames, chunk, p.L,
                            grow);
         }
       }
-      // Column indices of this thread's 32 elements: keys (dQ pass) or
-      // queries (dK/dV pass) [col0, col0 + 32).
-      const int col0 = c.kt * BT + 32 * hw;
+      // Column indices of this thread's 32 elements of a step: keys (dQ
+      // pass: two steps, columns 64 hw + 32 h2 of the 128-key tile) or
+      // queries (dK/dV pass: one step, columns 32 hw) [col0, col0 + 32).
+      int col0 = c.kt * BT + 32 * hw;
       // dK/dV pass: -LSE2 and -D of this warpgroup's 32 queries, 16 query
       // pairs of {-LSE2 pair, -D pair} (two packed fp32 pairs each, the same
       // for every lane), read from the tile's shared-memory slice where they
@@ -632,15 +601,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
       ok = wait_bar(bar(B_SF + b), bsm.ph, p, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      uint32_t sr[32], dr[32];
-      tmem_ld32(tl + s_col<kKV>(b) + 32u * hw, sr);
-      tmem_ld32(tl + dp_col<kKV>(b) + 32u * hw, dr);
-      tmem_wait_ld();
-      if (!kKV) {
-        // dQ pass: the dP part may take the next tile's dP.
-        tc_fence_before();
-        mbar_arrive(bar(B_DR));
-      }
+      uint32_t sr[32] = {}, dr[32] = {};
       uint32_t pp[16], pd[16];
       // Elements (2i, 2i+1) as one packed fp32 pair: P = 2^(c2 S - LSE2),
       // dS = P (dP - D), each rounded as the scalar expression would be;
@@ -667,16 +628,39 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         pp[i] = pack_bf16(e0, e1);
         pd[i] = pack_bf16(d0, d1);
       };
-      if (c.partial) {
+      auto step = [&]() {
+        if (c.partial) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pair(i, true);
-      } else {
+          for (int i = 0; i < 16; ++i) pair(i, true);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pair(i, false);
-      }
+          for (int i = 0; i < 16; ++i) pair(i, false);
+        }
+      };
       if (!kKV) {
-        tmem_st16(tl + s_col<kKV>(b) + 32u * hw, pd);  // dS over this warpgroup's S columns
+        // dQ pass: warpgroup hw takes keys [64 hw, 64 hw + 64) of the tile in
+        // two steps of 32; dS goes back over the start of each step's S
+        // columns (packed column 32 (ks >> 1) + 8 (ks & 1) for k-step ks).
+#pragma unroll 1
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const uint32_t col = 64u * hw + 32u * h2;
+          col0 = c.kt * BT + int(col);
+          tmem_ld32(tl + s_col<kKV>(b) + col, sr);
+          tmem_ld32(tl + dp_col<kKV>(b) + col, dr);
+          tmem_wait_ld();
+          if (h2 == 1) {
+            // The dP part may take the next tile's dP.
+            tc_fence_before();
+            mbar_arrive(bar(B_DR));
+          }
+          step();
+          tmem_st16(tl + s_col<kKV>(b) + col, pd);
+        }
       } else {
+        tmem_ld32(tl + s_col<kKV>(b) + 32u * hw, sr);
+        tmem_ld32(tl + dp_col<kKV>(b) + 32u * hw, dr);
+        tmem_wait_ld();
+        step();
         tmem_st16(tl + s_col<kKV>(b) + 32u * hw, pp);   // P^T over its S^T columns
         tmem_st16(tl + dp_col<kKV>(b) + 32u * hw, pd);  // dS^T over its dP^T columns
       }
@@ -698,7 +682,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
 #pragma unroll 1
         for (int oi = 0; oi < (kKV ? 2 : 1); ++oi) {
           // dQ pass: gQ = c * C0. dK/dV pass: gK = c * C1, gV = C0.
-          const uint32_t acc_col = !kKV ? TM_C0 : (oi == 0 ? TM_C1 : TM_C0);
+          const uint32_t acc_col = !kKV ? kC0<kKV> : (oi == 0 ? TM_C1 : kC0<kKV>);
           const float mul = (!kKV || oi == 0) ? p.scale : 1.f;
           __nv_bfloat16* dst = (!kKV || oi == 0) ? p.out0 : p.out1;
 #pragma unroll 1
@@ -773,7 +757,7 @@ static int launch_pass(const BwdArgs& a, const WorkList& w, int num_sms, unsigne
   const void* sx = kKV ? a.q : a.k;
   const void* sy = kKV ? a.g : a.v;
   if (!make_map(&m0, s0, a.L, BH, BR) || !make_map(&m1, s1, a.L, BH, BR) ||
-      !make_map(&mx, sx, a.L, BH, BT) || !make_map(&my, sy, a.L, BH, BT))
+      !make_map(&mx, sx, a.L, BH, kBT<kKV>) || !make_map(&my, sy, a.L, BH, kBT<kKV>))
     return JVP_ERR_LAUNCH_FAILED;
   Params p;
   p.qtiles = w.qtiles;
@@ -784,7 +768,7 @@ static int launch_pass(const BwdArgs& a, const WorkList& w, int num_sms, unsigne
   if (items > 0x7fffffffLL) return JVP_ERR_TOO_LARGE;
   p.n_items = int(items);
   p.n_qt = (a.L + BR - 1) / BR;
-  p.n_kt = (a.L + BT - 1) / BT;
+  p.n_kt = (a.L + kBT<kKV> - 1) / kBT<kKV>;
   p.L = a.L;
   p.mask = a.mask;
   p.scale = a.scale;
