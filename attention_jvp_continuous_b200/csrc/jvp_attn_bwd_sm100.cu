@@ -641,20 +641,29 @@ bwd_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CU
         // dQ pass: warpgroup hw takes keys [64 hw, 64 hw + 64) of the tile in
         // two steps of 32; dS goes back over the start of each step's S
         // columns (packed column 32 (ks >> 1) + 8 (ks & 1) for k-step ks).
-#pragma unroll 1
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const uint32_t col = 64u * hw + 32u * h2;
-          col0 = c.kt * BT + int(col);
+        // Both steps' dP are loaded up front, so the dP part is released
+        // before any arithmetic, and the second step's S load is in flight
+        // while the first step's dS is stored.
+        {
+          const uint32_t col = 64u * hw;
+          uint32_t dr1[32];
           tmem_ld32(tl + s_col<kKV>(b) + col, sr);
           tmem_ld32(tl + dp_col<kKV>(b) + col, dr);
+          tmem_ld32(tl + dp_col<kKV>(b) + col + 32u, dr1);
           tmem_wait_ld();
-          if (h2 == 1) {
-            // The dP part may take the next tile's dP.
-            tc_fence_before();
-            mbar_arrive(bar(B_DR));
-          }
+          // Both steps' dP are in registers: the dP part may take the next tile's dP.
+          tc_fence_before();
+          mbar_arrive(bar(B_DR));
+          col0 = c.kt * BT + int(col);
           step();
           tmem_st16(tl + s_col<kKV>(b) + col, pd);
+          tmem_ld32(tl + s_col<kKV>(b) + col + 32u, sr);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) dr[i] = dr1[i];
+          tmem_wait_ld();
+          col0 = c.kt * BT + int(col) + 32;
+          step();
+          tmem_st16(tl + s_col<kKV>(b) + col + 32u, pd);
         }
       } else {
         tmem_ld32(tl + s_col<kKV>(b) + 32u * hw, sr);
