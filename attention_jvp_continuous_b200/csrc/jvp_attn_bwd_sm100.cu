@@ -20,10 +20,10 @@
 //                               with each Q tile)
 //      gV += P^T G, gK += dS^T Q (A in TMEM, N = 128)
 // Warp roles: warp 0 TMA, warps 1 and 2 issue MMAs (whole warps, one
-// elected lane issuing), warps 4-11 two warpgroups taking 32 of each tile's
-// 64 columns. Each
-// warpgroup writes its bf16 operands into the TMEM columns it has just read
-// itself, so no exchange between the warpgroups is needed.
+// elected lane issuing), warps 4-11 two warpgroups taking half of each
+// tile's columns (64 of 128 keys in the dQ pass, 32 of 64 queries in the
+// dK/dV pass). Each warpgroup writes its bf16 operands into the TMEM columns
+// it has just read itself, so no exchange between the warpgroups is needed.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
