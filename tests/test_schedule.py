@@ -49,7 +49,14 @@ for n in range(24):
                   int(rng.choice([8, 16, 64]))))
 
 
-@pytest.mark.parametrize("mode,T,F,ch,bm,bn", CASES)
+# The backward's query pass runs 128 x 128 tiles: ragged lengths, lengths
+# below one tile, and each mask mode.
+QCASES = [(ja.TEACHER_FORCING, 200, 3, 1, 128, 128), (ja.TEACHER_FORCING, 100, 5, 2, 128, 128),
+          (ja.FRAME_CAUSAL, 130, 5, 1, 128, 128), (ja.CHUNK_CAUSAL, 70, 7, 3, 128, 128),
+          (ja.DENSE, 64, 4, 1, 128, 128), (ja.TEACHER_FORCING, 5, 2, 1, 128, 128)]
+
+
+@pytest.mark.parametrize("mode,T,F,ch,bm,bn", CASES + QCASES)
 def test_tile_classes_match_brute_force(mode, T, F, ch, bm, bn):
     spec = MaskSpec(mode, T, F, ch)
     got = ja.tile_classes(ja.Mask(mode, T, F, ch), bm=bm, bn=bn)
@@ -60,7 +67,7 @@ def test_tile_classes_match_brute_force(mode, T, F, ch, bm, bn):
     assert (full, partial, empty) == tuple(int((want == c).sum()) for c in (1, 2, 0))
 
 
-@pytest.mark.parametrize("mode,T,F,ch,bm,bn", CASES[:12])
+@pytest.mark.parametrize("mode,T,F,ch,bm,bn", CASES[:12] + QCASES)
 def test_schedule_covers_nonempty_tiles_in_order(mode, T, F, ch, bm, bn):
     mk = ja.Mask(mode, T, F, ch)
     cls = ja.tile_classes(mk, bm=bm, bn=bn)
